@@ -1,0 +1,393 @@
+"""Benchmark: decode step of IsoQuant compressed-space attention on B200.
+
+Workload (default): GQA decode, batch 16, 32 query / 4 KV heads, d = 128,
+context 32768 (bf16 heavy-tailed K/V compressed into a paged 3-bit cache
+with 256-token pages and a shuffled page table).  One step = append one new
+token per sequence (isoquant_compress_kv), rotate the queries
+(isoquant_rotate_q), split-context attention over the packed codes
+(isoquant_attend_partial) and the combine with the inverse rotation
+(isoquant_attend_combine): every row of the hot path.
+
+Metric: KV-token x KV-head pairs attended per second (sum over sequences of
+the context length times the KV heads, per step), and the achieved HBM
+bandwidth of the attention kernel on the 108 compressed bytes per KV
+token-head, against the measured copy bandwidth of this GPU.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 it is launched with torchrun, one rank per GPU; every rank runs its
+own shard (weak scaling) and rank 0 prints the line.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+BYTES_PER_KV_TOKEN_HEAD = 2 * (13 * 4 + 2)  # K and V: 13 words + fp16 norm
+METRIC = "decode attention KV-token·heads/s on packed 3-bit KV; achieved HBM GB/s vs ~8 TB/s"
+UNIT = "KV-token·heads/s"
+DEFAULT_WORKLOAD = "gqa_b16_q32_kv4_L32768_paged"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            mp = json.load(f)
+        return float(mp["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_src):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, or None when the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "attend_partial_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("source_hash") != source_hash(*kernel_src):
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons, n = [], [], set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                except ValueError:
+                    continue
+                n += 1
+                for nm, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import compressed_space_decode_b200 as csd
+    from compressed_space_decode_b200 import multi, synthetic
+    from compressed_space_decode_b200.workload import DecodeState
+
+    rank, local_rank, world = multi.env_rank()
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    wl = multi.shard_workload(synthetic.workloads()[args.workload], rank, world)
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    growth = args.warmup + args.steps + e2e_steps + 2
+    st = DecodeState(wl, growth=growth, device=dev)
+    B, H, Hq, nq = st.B, st.H, st.Hq, wl.nq
+    stream = torch.cuda.current_stream(dev)
+
+    # per-step inputs, generated up front (device-resident for the kernel metric)
+    n_total = args.warmup + args.steps
+    lens0 = list(st.seq_lens)
+    k_all = torch.empty((n_total, B, H, 128), dtype=torch.bfloat16, device=dev)
+    v_all = torch.empty_like(k_all)
+    for b in range(B):
+        k, v = st.kv_tokens(b, lens0[b], lens0[b] + n_total)
+        k_all[:, b] = k
+        v_all[:, b] = v
+    q_all = synthetic.gaussian(wl.seed, 20_000_000, (n_total, B * nq, Hq, 128), device=dev, dtype=torch.bfloat16)
+    slots_all = st.slot_matrix(lens0, n_total)
+    lens_all = torch.tensor([[L + s + 1 for L in lens0] for s in range(n_total)], dtype=torch.int32, device=dev)
+    q_rot = torch.empty((B, nq, Hq, 128), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q_rot)
+    ws = csd.alloc_workspace(st.ctx, B, nq, Hq, device=dev)
+    launches = [0]
+
+    def step(s, k, v, q, slots, lens):
+        csd.isoquant_compress_kv(st.ctx, st.cache, k, v, slots, stream=stream)
+        launches[0] += csd.isoquant_last_launch_count(st.ctx)
+        csd.isoquant_rotate_q(st.ctx, q, q_rot.view(B * nq, Hq, 128), stream=stream)
+        launches[0] += csd.isoquant_last_launch_count(st.ctx)
+        ev = attn_events[s] if attn_events is not None else None
+        if ev is not None:
+            ev[0].record(stream)
+        csd.isoquant_attend_partial(st.ctx, st.cache, q_rot, st.page_table, lens, ws, causal=wl.causal,
+                                    stream=stream)
+        launches[0] += csd.isoquant_last_launch_count(st.ctx)
+        if ev is not None:
+            ev[1].record(stream)
+        csd.isoquant_attend_combine(st.ctx, B, nq, Hq, lens, st.ps, ws, out, stream=stream)
+        launches[0] += csd.isoquant_last_launch_count(st.ctx)
+
+    attn_events = None
+    for s in range(args.warmup):
+        step(s, k_all[s], v_all[s], q_all[s], slots_all[s], lens_all[s])
+    torch.cuda.synchronize(dev)
+
+    attn_events = {s: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for s in range(args.warmup, n_total)}
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    launches[0] = 0
+    multi.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.warmup, n_total):
+        step(s, k_all[s], v_all[s], q_all[s], slots_all[s], lens_all[s])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    multi.barrier()
+    ms_local = t_start.elapsed_time(t_end)
+    kernel_launches = launches[0]
+    attn_ms = [attn_events[s][0].elapsed_time(attn_events[s][1]) for s in range(args.warmup, n_total)]
+    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+
+    units_local = sum(int(lens_all[s].sum().item()) * H for s in range(args.warmup, n_total))
+    ms = multi.max_over_ranks(ms_local, device=dev)
+    units = multi.sum_over_ranks(units_local, device=dev)
+    value = units / (ms / 1e3)
+
+    # roofline of the attention kernel: algorithmic bytes per launch / duration
+    bytes_per_launch = BYTES_PER_KV_TOKEN_HEAD * units_local / args.steps
+    achieved = bytes_per_launch / (attn_avg_ms / 1e3) / 1e9
+    peak, peak_kind = peaks()
+    traffic = profiled_traffic(["compressed_space_decode_b200/csrc/attend.cu",
+                                "compressed_space_decode_b200/csrc/isoquant_internal.cuh"])
+
+    # end to end through the public API from pinned host buffers
+    attn_events = None
+    st.seq_lens = [L + n_total for L in lens0]
+    base = n_total
+    kh = torch.empty((e2e_steps, B, H, 128), dtype=torch.bfloat16).pin_memory()
+    vh = torch.empty_like(kh).pin_memory()
+    for b in range(B):
+        k, v = st.kv_tokens(b, lens0[b] + base, lens0[b] + base + e2e_steps)
+        kh[:, b] = k.cpu()
+        vh[:, b] = v.cpu()
+    qh = q_all[:e2e_steps].cpu().pin_memory()
+    slots_h = st.slot_matrix([L + base for L in lens0], e2e_steps).cpu().pin_memory()
+    lens_h = torch.tensor([[L + base + s + 1 for L in lens0] for s in range(e2e_steps)], dtype=torch.int32).pin_memory()
+    out_h = torch.empty((e2e_steps, B, nq, Hq, 128), dtype=torch.float32).pin_memory()
+    kd, vd = torch.empty_like(k_all[0]), torch.empty_like(v_all[0])
+    qd, sd, ld = torch.empty_like(q_all[0]), torch.empty_like(slots_all[0]), torch.empty_like(lens_all[0])
+    h2d = (kd.numel() * 2 + vd.numel() * 2 + qd.numel() * 2 + sd.numel() * 8 + ld.numel() * 4)
+    d2h = out.numel() * 4
+    multi.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(e2e_steps):
+        kd.copy_(kh[s], non_blocking=True)
+        vd.copy_(vh[s], non_blocking=True)
+        qd.copy_(qh[s], non_blocking=True)
+        sd.copy_(slots_h[s], non_blocking=True)
+        ld.copy_(lens_h[s], non_blocking=True)
+        step(0, kd, vd, qd, sd, ld)
+        out_h[s].copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = multi.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    e2e_units = multi.sum_over_ranks(sum(int(lens_h[s].sum().item()) * H for s in range(e2e_steps)), device=dev)
+    e2e_value = e2e_units / (e2e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 accumulate (3-bit codes -> f16 centroids, hi/lo f16 queries on mma.sync)",
+        "data": "synthetic (seeded bf16 Student-t(4) K/V, log-uniform channel scales, x20 outliers)",
+        "config": {"workload": wl.name.split("@")[0], "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
+                   "context_start": lens0[0], "page_size": st.ps, "page_table": "shuffled",
+                   "step": "append 1 token/seq + rotate_q + attend_partial + attend_combine",
+                   "l2": f"packed cache {bytes_per_launch / 1e6:.0f} MB > 126 MB L2; no flush",
+                   "parallelism": f"dp{world} (independent shards)"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "roofline": {"bound": "hbm", "kernel": "isoquant_attend_partial", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+                     "bytes_per_launch": bytes_per_launch, "avg_launch_ms": attn_avg_ms,
+                     "frac_of_8TBps": achieved / 8000.0},
+        "gpu_launches": kernel_launches,
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line))
+
+
+def oracle_sample(wl, b, h):
+    """Oracle state for one (sequence, KV head) of workload `wl`: its own
+    codes of the context, the appended token and the step's query rows.
+    Inputs come from the seeded generators only."""
+    import oracle
+    from compressed_space_decode_b200 import synthetic
+    L = wl.seq_lens[b]
+    G = wl.group
+    k, v = synthetic.workload_kv_tokens(wl, b, 0, L + 1, device="cuda")
+    signs, quats = synthetic.rotation_params(wl.seed, wl.kv_heads)
+    s, qt = signs[h].numpy(), quats[h].numpy()
+    kc, kn, _, _ = oracle.compress(s, qt, k[:L, h].double().cpu().numpy())
+    vc, vn, _, _ = oracle.compress(s, qt, v[:L, h].double().cpu().numpy())
+    newk = k[L:L + 1, h].double().cpu().numpy()
+    newv = v[L:L + 1, h].double().cpu().numpy()
+    q = synthetic.workload_queries(wl, 0, device="cuda")[b, 0, h * G:(h + 1) * G].double().cpu().numpy()
+    return dict(s=s, qt=qt, kc=kc, kn=kn, vc=vc, vn=vn, newk=newk, newv=newv, q=q, L=L, G=G)
+
+
+def oracle_step(o):
+    """One decode step of the oracle for one (sequence, KV head): compress
+    the appended K/V token, then attend over L+1 tokens."""
+    import numpy as np
+
+    import oracle
+    kc1, kn1, _, _ = oracle.compress(o["s"], o["qt"], o["newk"])
+    vc1, vn1, _, _ = oracle.compress(o["s"], o["qt"], o["newv"])
+    kc = np.concatenate([o["kc"], kc1])
+    kn = np.concatenate([o["kn"], kn1])
+    vc = np.concatenate([o["vc"], vc1])
+    vn = np.concatenate([o["vn"], vn1])
+    R = o["q"].shape[0]
+    return oracle.attend(o["s"], o["qt"], o["q"], kc, kn, vc, vn, [o["L"] + 1] * R)
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    """The fp64 oracle, as it stands, on the host cores: a bounded sample of
+    the same decode step (whole (sequence, KV head) units, repeated)."""
+    o = oracle_sample(wl, 0, 0)
+    units, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        oracle_step(o)
+        units += o["L"] + 1
+    dt = time.perf_counter() - t0
+    return {"value": units / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"sequence 0, KV head 0 of the workload (context {o['L'] + 1}, {o['G']} query rows): "
+                      f"compress the appended token + attend, repeated {units // (o['L'] + 1)}x in {dt:.1f} s"}
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args):
+    """The fp64 oracle as the reference arm (there is no reference code to
+    install: the pages describe the method only).  Rank 0 only."""
+    rank, local_rank, world = (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+                               int(os.environ.get("WORLD_SIZE", "1")))
+    if rank != 0:
+        return
+    import torch
+
+    from compressed_space_decode_b200 import synthetic
+    torch.cuda.set_device(local_rank)
+    wl = synthetic.workloads()[args.workload]
+    o = oracle_sample(wl, 0, 0)
+    for _ in range(args.warmup):
+        oracle_step(o)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(o)
+    dt = time.perf_counter() - t0
+    units = args.steps * (o["L"] + 1)
+    value = units / dt
+    sample = (f"each step: sequence 0, KV head 0 of {wl.name} (context {o['L'] + 1}, {o['G']} query rows), "
+              f"compress the appended token + attend")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.q_heads, "kv_heads": wl.kv_heads,
+                   "head_dim": 128, "context_start": wl.seq_lens[0], "page_size": wl.page_size},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

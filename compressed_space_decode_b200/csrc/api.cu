@@ -1,0 +1,338 @@
+// api.cu -- C ABI entry points: argument checks, parameter block, codebook,
+// launch sequencing.  See include/isoquant.h for the contract of each call.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "isoquant_internal.cuh"
+
+namespace isoquant {
+
+// Lloyd's conditions for the 8-level minimum-MSE quantizer of N(0,1): each
+// decision threshold is the midpoint of its neighbouring levels and each
+// level is the mean of the standard normal restricted to its cell,
+// (pdf(a) - pdf(b)) / (cdf(b) - cdf(a)).  Iterated from evenly spaced levels;
+// the levels are then rounded to fp16 (the stored decode values) and the
+// thresholds taken as midpoints of the rounded levels.
+int build_codebook(Codebook *cb) {
+  const double inv_sqrt2pi = 0.39894228040143267794;
+  auto pdf = [&](double z) { return inv_sqrt2pi * std::exp(-0.5 * z * z); };
+  auto cdf = [](double z) { return 0.5 * std::erfc(-z * 0.70710678118654752440); };
+  double lv[kLevels], th[kLevels - 1];
+  for (int i = 0; i < kLevels; ++i) lv[i] = 3.0 * (2.0 * i + 1.0 - kLevels) / kLevels;
+  for (int iter = 0; iter < 100000; ++iter) {
+    for (int k = 0; k < kLevels - 1; ++k) th[k] = 0.5 * (lv[k] + lv[k + 1]);
+    double moved = 0.0;
+    for (int i = 0; i < kLevels; ++i) {
+      const double pa = i == 0 ? 0.0 : pdf(th[i - 1]);
+      const double pb = i == kLevels - 1 ? 0.0 : pdf(th[i]);
+      const double ca = i == 0 ? 0.0 : cdf(th[i - 1]);
+      const double cbv = i == kLevels - 1 ? 1.0 : cdf(th[i]);
+      const double c = (pa - pb) / (cbv - ca);
+      moved = std::fmax(moved, std::fabs(c - lv[i]));
+      lv[i] = c;
+    }
+    if (moved < 1e-15) break;
+  }
+  for (int i = 0; i < kLevels; ++i) {
+    const __half h = __double2half(lv[i]);
+    cb->level16[i] = __half_as_ushort(h);
+    cb->level[i] = __half2float(h);
+  }
+  for (int k = 0; k < kLevels - 1; ++k) {
+    cb->threshold64[k] = 0.5 * (static_cast<double>(cb->level[k]) + cb->level[k + 1]);
+    cb->threshold[k] = static_cast<float>(cb->threshold64[k]);
+  }
+  return 0;
+}
+
+namespace {
+
+// left multiplication by a: a (x) v = L(a) v;  right multiplication by c:
+// v (x) c = Rm(c) v  (Hamilton product, quaternions as (w, x, y, z)).
+void left_matrix(const double a[4], double m[16]) {
+  const double t[16] = {a[0], -a[1], -a[2], -a[3], a[1], a[0], -a[3], a[2],
+                        a[2], a[3],  a[0], -a[1], a[3], -a[2], a[1], a[0]};
+  std::memcpy(m, t, sizeof(t));
+}
+void right_matrix(const double c[4], double m[16]) {
+  const double t[16] = {c[0], -c[1], -c[2], -c[3], c[1], c[0], c[3], -c[2],
+                        c[2], -c[3], c[0],  c[1], c[3], c[2], -c[1], c[0]};
+  std::memcpy(m, t, sizeof(t));
+}
+
+bool build_head(const int8_t *signs, const float *quats, HeadParams *hp) {
+  std::memset(hp, 0, sizeof(*hp));
+  for (int j = 0; j < kD; ++j) {
+    if (signs[j] != 1 && signs[j] != -1) return false;
+    if (signs[j] < 0) hp->sign_bits[j >> 5] |= 1u << (j & 31);
+  }
+  for (int b = 0; b < kBlocks; ++b) {
+    double ql[4], qr[4];
+    for (int s = 0; s < 2; ++s) {
+      const float *q = quats + (b * 2 + s) * 4;
+      double n2 = 0.0;
+      for (int c = 0; c < 4; ++c) {
+        if (!std::isfinite(q[c])) return false;
+        n2 += static_cast<double>(q[c]) * q[c];
+      }
+      if (!(n2 > 0.0)) return false;
+      const double inv = 1.0 / std::sqrt(n2);
+      double *dst = s == 0 ? ql : qr;
+      for (int c = 0; c < 4; ++c) dst[c] = q[c] * inv;
+    }
+    // block b: v -> qL (x) v (x) conj(qR) = L(qL) Rm(conj qR) v
+    const double cr[4] = {qr[0], -qr[1], -qr[2], -qr[3]};
+    double Lm[16], Rm[16];
+    left_matrix(ql, Lm);
+    right_matrix(cr, Rm);
+    for (int r = 0; r < 4; ++r)
+      for (int c = 0; c < 4; ++c) {
+        double acc = 0.0;
+        for (int k = 0; k < 4; ++k) acc += Lm[4 * r + k] * Rm[4 * k + c];
+        hp->m64[b][4 * r + c] = acc;
+        hp->m32[b][4 * r + c] = static_cast<float>(acc);
+      }
+  }
+  return true;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool valid_page_size(int ps) { return ps == 32 || ps == 64 || ps == 128 || ps == 256; }
+
+int make_shape(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, int page_size, int causal,
+               AttendShape *s) {
+  if (batch < 0 || nq < 1 || num_q_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
+  if (num_q_heads % ctx->num_kv_heads != 0) return ISOQUANT_ERR_INVALID_ARG;
+  s->batch = batch;
+  s->nq = nq;
+  s->q_heads = num_q_heads;
+  s->kv_heads = ctx->num_kv_heads;
+  s->group = num_q_heads / ctx->num_kv_heads;
+  s->rows = nq * s->group;
+  s->row_groups = (s->rows + 7) / 8;
+  s->page_size = page_size;
+  s->causal = causal ? 1 : 0;
+  s->n_cta = ctx->num_sms;
+  s->slots = static_cast<size_t>(s->n_cta) +
+             static_cast<size_t>(s->row_groups) * static_cast<size_t>(batch) * ctx->num_kv_heads;
+  return ISOQUANT_OK;
+}
+
+int check_cache(const isoquant_cache *cache) {
+  if (cache == nullptr || cache->codes == nullptr || cache->norms == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  if (cache->num_pages < 1) return ISOQUANT_ERR_INVALID_ARG;
+  if (!valid_page_size(cache->page_size)) return ISOQUANT_ERR_UNSUPPORTED;
+  if (!aligned(cache->codes, 16) || !aligned(cache->norms, 16)) return ISOQUANT_ERR_ALIGNMENT;
+  return ISOQUANT_OK;
+}
+
+int dtype_bytes(int dtype) {
+  switch (dtype) {
+    case ISOQUANT_F32: return 4;
+    case ISOQUANT_BF16: return 2;
+    case ISOQUANT_F16: return 2;
+    default: return 0;
+  }
+}
+
+}  // namespace
+}  // namespace isoquant
+
+using namespace isoquant;
+
+extern "C" {
+
+const char *isoquant_strerror(int status) {
+  switch (status) {
+    case ISOQUANT_OK: return "ok";
+    case ISOQUANT_ERR_INVALID_ARG: return "invalid argument";
+    case ISOQUANT_ERR_UNSUPPORTED: return "unsupported (head_dim must be 128; dtype F32/BF16/F16; page size 32/64/128/256)";
+    case ISOQUANT_ERR_OUT_OF_RANGE: return "index or length out of range";
+    case ISOQUANT_ERR_WORKSPACE: return "workspace too small";
+    case ISOQUANT_ERR_CUDA: return "CUDA runtime error";
+    case ISOQUANT_ERR_ALIGNMENT: return "pointer not aligned (16 bytes required)";
+    default: return "unknown status";
+  }
+}
+
+int isoquant_codebook(float levels[8], float thresholds[7]) {
+  if (levels == nullptr || thresholds == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  Codebook cb;
+  build_codebook(&cb);
+  for (int i = 0; i < kLevels; ++i) levels[i] = cb.level[i];
+  for (int k = 0; k < kLevels - 1; ++k) thresholds[k] = cb.threshold[k];
+  return ISOQUANT_OK;
+}
+
+int isoquant_init(isoquant_ctx **out, int num_kv_heads, int head_dim, const int8_t *signs, const float *quats) {
+  if (out == nullptr || signs == nullptr || quats == nullptr || num_kv_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (head_dim != kD) return ISOQUANT_ERR_UNSUPPORTED;
+  std::vector<HeadParams> host(static_cast<size_t>(num_kv_heads));
+  for (int h = 0; h < num_kv_heads; ++h)
+    if (!build_head(signs + static_cast<size_t>(h) * kD, quats + static_cast<size_t>(h) * kBlocks * 8, &host[h]))
+      return ISOQUANT_ERR_INVALID_ARG;
+  isoquant_ctx *ctx = new (std::nothrow) isoquant_ctx();
+  if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  build_codebook(&ctx->codebook);
+  ctx->num_kv_heads = num_kv_heads;
+  if (cudaGetDevice(&ctx->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess ||
+      cudaMalloc(&ctx->params, sizeof(HeadParams) * num_kv_heads) != cudaSuccess ||
+      cudaMalloc(&ctx->status, 16) != cudaSuccess ||
+      cudaMemcpy(ctx->params, host.data(), sizeof(HeadParams) * num_kv_heads, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemset(ctx->status, 0, 16) != cudaSuccess) {
+    if (ctx->params) cudaFree(ctx->params);
+    if (ctx->status) cudaFree(ctx->status);
+    delete ctx;
+    return ISOQUANT_ERR_CUDA;
+  }
+  *out = ctx;
+  return ISOQUANT_OK;
+}
+
+void isoquant_destroy(isoquant_ctx *ctx) {
+  if (ctx == nullptr) return;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(ctx->device);
+  cudaDeviceSynchronize();
+  cudaFree(ctx->params);
+  cudaFree(ctx->status);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete ctx;
+}
+
+int isoquant_cache_bytes(const isoquant_ctx *ctx, int num_pages, int page_size, size_t *code_bytes,
+                         size_t *norm_bytes) {
+  if (ctx == nullptr || code_bytes == nullptr || norm_bytes == nullptr || num_pages < 0) return ISOQUANT_ERR_INVALID_ARG;
+  if (!valid_page_size(page_size)) return ISOQUANT_ERR_UNSUPPORTED;
+  const size_t vecs = static_cast<size_t>(num_pages) * 2 * ctx->num_kv_heads * page_size;
+  *code_bytes = vecs * kWords * sizeof(uint32_t);
+  *norm_bytes = vecs * sizeof(uint16_t);
+  return ISOQUANT_OK;
+}
+
+int isoquant_compress_kv(isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v, int dtype,
+                         int n_tok, const int64_t *slot_mapping, void *stream) {
+  if (ctx == nullptr || n_tok < 0) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 0;
+  int st = check_cache(cache);
+  if (st != ISOQUANT_OK) return st;
+  const int eb = dtype_bytes(dtype);
+  if (eb == 0) return ISOQUANT_ERR_UNSUPPORTED;
+  if (n_tok == 0) return ISOQUANT_OK;
+  if (k == nullptr || v == nullptr || slot_mapping == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  const uintptr_t need = eb == 4 ? 16 : 8;
+  if (!aligned(k, need) || !aligned(v, need) || !aligned(slot_mapping, 8)) return ISOQUANT_ERR_ALIGNMENT;
+  cudaError_t e = launch_compress(ctx, cache, k, v, dtype, n_tok, slot_mapping, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
+  ctx->last_launches = 1;
+  return ISOQUANT_OK;
+}
+
+int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows, int num_q_heads, float *q_rot,
+                      void *stream) {
+  if (ctx == nullptr || n_rows < 0 || num_q_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 0;
+  if (num_q_heads % ctx->num_kv_heads != 0) return ISOQUANT_ERR_INVALID_ARG;
+  const int eb = dtype_bytes(dtype);
+  if (eb == 0) return ISOQUANT_ERR_UNSUPPORTED;
+  if (n_rows == 0) return ISOQUANT_OK;
+  if (q == nullptr || q_rot == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  if (!aligned(q, eb == 4 ? 16 : 8) || !aligned(q_rot, 16)) return ISOQUANT_ERR_ALIGNMENT;
+  cudaError_t e = launch_rotate_q(ctx, q, dtype, n_rows, num_q_heads, q_rot, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
+  ctx->last_launches = 1;
+  return ISOQUANT_OK;
+}
+
+int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, size_t *bytes) {
+  if (ctx == nullptr || bytes == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  AttendShape s;
+  int st = make_shape(ctx, batch, nq, num_q_heads, 256, 0, &s);
+  if (st != ISOQUANT_OK) return st;
+  *bytes = attend_workspace_bytes(s);
+  return ISOQUANT_OK;
+}
+
+int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache, const float *q_rot, int batch, int nq,
+                            int num_q_heads, const int32_t *page_table, int max_pages, const int32_t *seq_lens,
+                            int causal, float scale, void *workspace, size_t ws_bytes, void *stream) {
+  if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 0;
+  int st = check_cache(cache);
+  if (st != ISOQUANT_OK) return st;
+  AttendShape s;
+  st = make_shape(ctx, batch, nq, num_q_heads, cache->page_size, causal, &s);
+  if (st != ISOQUANT_OK) return st;
+  if (!(scale >= 0.0f) || !std::isfinite(scale)) return ISOQUANT_ERR_INVALID_ARG;
+  if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(kD));
+  if (batch == 0) return ISOQUANT_OK;
+  if (q_rot == nullptr || page_table == nullptr || seq_lens == nullptr || workspace == nullptr || max_pages < 1)
+    return ISOQUANT_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16) || !aligned(q_rot, 4) || !aligned(page_table, 4) || !aligned(seq_lens, 4))
+    return ISOQUANT_ERR_ALIGNMENT;
+  if (ws_bytes < attend_workspace_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
+  cudaError_t e = launch_attend_partial(ctx, cache, s, q_rot, page_table, max_pages, seq_lens, scale, workspace,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
+  ctx->last_launches = 1;
+  return ISOQUANT_OK;
+}
+
+int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq, int num_q_heads, const int32_t *seq_lens,
+                            int page_size, const void *workspace, size_t ws_bytes, float *out, void *stream) {
+  if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 0;
+  if (!valid_page_size(page_size)) return ISOQUANT_ERR_UNSUPPORTED;
+  AttendShape s;
+  int st = make_shape(ctx, batch, nq, num_q_heads, page_size, 0, &s);
+  if (st != ISOQUANT_OK) return st;
+  if (batch == 0) return ISOQUANT_OK;
+  if (seq_lens == nullptr || workspace == nullptr || out == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16) || !aligned(out, 16) || !aligned(seq_lens, 4)) return ISOQUANT_ERR_ALIGNMENT;
+  if (ws_bytes < attend_workspace_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
+  cudaError_t e = launch_attend_combine(ctx, s, seq_lens, workspace, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
+  ctx->last_launches = 1;
+  return ISOQUANT_OK;
+}
+
+int isoquant_attend_decode(isoquant_ctx *ctx, const isoquant_cache *cache, const float *q_rot, int batch, int nq,
+                           int num_q_heads, const int32_t *page_table, int max_pages, const int32_t *seq_lens,
+                           int causal, float scale, void *workspace, size_t ws_bytes, float *out, void *stream) {
+  if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  if (out == nullptr && batch > 0) return ISOQUANT_ERR_INVALID_ARG;
+  if (out != nullptr && !aligned(out, 16)) return ISOQUANT_ERR_ALIGNMENT;
+  int st = isoquant_attend_partial(ctx, cache, q_rot, batch, nq, num_q_heads, page_table, max_pages, seq_lens,
+                                   causal, scale, workspace, ws_bytes, stream);
+  if (st != ISOQUANT_OK) return st;
+  const int first = ctx->last_launches;
+  st = isoquant_attend_combine(ctx, batch, nq, num_q_heads, seq_lens, cache->page_size, workspace, ws_bytes, out,
+                               stream);
+  ctx->last_launches += first;
+  return st;
+}
+
+int isoquant_get_status(isoquant_ctx *ctx, uint32_t *status, void *stream) {
+  if (ctx == nullptr || status == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t host = 0;
+  if (cudaMemcpyAsync(&host, ctx->status, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess || cudaMemsetAsync(ctx->status, 0, 16, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return ISOQUANT_ERR_CUDA;
+  *status = host;
+  return ISOQUANT_OK;
+}
+
+int isoquant_last_launch_count(const isoquant_ctx *ctx) { return ctx ? ctx->last_launches : 0; }
+
+}  // extern "C"

@@ -1,0 +1,711 @@
+// attend.cu -- isoquant_attend_partial / isoquant_attend_combine.
+//
+// RotaryQuant, Abstract: attention runs directly on the packed 3-bit
+// tensors, without materialising full-precision KV.  Scores and the
+// softmax-weighted V sum are formed in the rotated space from the codes; the
+// output is rotated back once, in the combine step.
+//
+// Partial kernel (one CTA per SM, persistent, split-K over pages):
+//   * work = pages of (row group, batch, KV head) pairs, laid end to end;
+//     CTA c takes pages [c*P/N, (c+1)*P/N) so that every SM streams the same
+//     number of pages whatever the length mix, and writes one partial
+//     (m, l, o) per pair it touches.
+//   * warp 8 is a producer: per page it issues 28 bulk copies (13 K code
+//     rows, 13 V code rows, 2 norm rows) into a 4-stage shared-memory ring
+//     with an mbarrier per stage.
+//   * warps 0..7 take 32-token slices of the page.  A GQA group of up to 8
+//     query rows shares every KV tile: Q.K^T is an m16n8k16 tensor-core
+//     product with the query split into fp16 high and low parts in the 16
+//     rows (so the score keeps ~22 bits), K codes become fp16 centroids
+//     through a 64-entry pair table held once per lane in shared memory, and
+//     P.V is a second m16n8k16 product with V^T as the A operand.
+//   * at the end of each pair, the 8 warps merge their (m, l, o) in shared
+//     memory and one record is written to the workspace.
+// Combine kernel: one warp per output row merges the records of its pair,
+// divides by l and applies R^-1 = D Hn B^T.
+#include <cuda_fp16.h>
+
+#include <cmath>
+
+#include "isoquant_internal.cuh"
+
+namespace isoquant {
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStages = 4;
+constexpr int kMaxPage = 256;
+// Shared-memory row strides (32-bit words) of the K and V code rows.  K rows
+// are read as word rows {3t, 3t+1, 3t+2} by the four threads of a quad; a
+// stride = 24 (mod 32) puts those rows in distinct 16-byte bank groups.  V
+// rows are read as rows {2p, 2p+1}; a stride = 4 (mod 32) interleaves them.
+constexpr int kStrideK = kMaxPage + 24;
+constexpr int kStrideV = kMaxPage + 4;
+constexpr int kStageKC = 0;
+constexpr int kStageVC = kStageKC + kWords * kStrideK * 4;
+constexpr int kStageKN = kStageVC + kWords * kStrideV * 4;
+constexpr int kStageVN = kStageKN + kMaxPage * 2;
+constexpr int kStageBytes = kStageVN + kMaxPage * 2;
+// merge scratch: o[8 warps][8 rows][128], m[8][8], l[8][8], e[8]
+constexpr int kScratchO = kStages * kStageBytes;
+constexpr int kScratchM = kScratchO + kConsumerWarps * 8 * kD * 4;
+constexpr int kScratchL = kScratchM + kConsumerWarps * 8 * 4;
+constexpr int kScratchE = kScratchL + kConsumerWarps * 8 * 4;
+constexpr int kBarriers = kScratchE + 8 * 4;
+constexpr int kLocate = kBarriers + 2 * kStages * 8;
+constexpr int kSmemBytes = kLocate + 64;
+static_assert(kStageBytes % 16 == 0, "stage alignment");
+
+constexpr uint32_t kSpinLimit = 1u << 25;
+
+struct PartialParams {
+  const uint32_t *codes;
+  const uint16_t *norms;
+  int num_pages, page_size;
+  const float *q_rot;
+  const int32_t *page_table;
+  int max_pages;
+  const int32_t *seq_lens;
+  int B, nq, Hq, H, G, R, RG, causal;
+  float qfold;  // scale * log2(e) / sqrt(128)
+  float level[kLevels];
+  float *records;
+  uint32_t *status;
+  int n_cta;
+};
+
+struct CombineParams {
+  const float *records;
+  const HeadParams *params;
+  const int32_t *seq_lens;
+  float *out;
+  int B, nq, Hq, H, G, RG, page_size, n_cta;
+};
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: gives up after kSpinLimit polls, raising the timeout bit.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
+                                          volatile int *abort_flag) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (i > 64) __nanosleep(64);
+  }
+  set_status(status, ISOQUANT_DEVERR_WAIT_TIMEOUT);
+  if (abort_flag != nullptr) *abort_flag = 1;
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// ------------------------------------------------------------ work walk
+__device__ __forceinline__ int pages_of(int L, int ps) { return L > 0 ? (L + ps - 1) / ps : 0; }
+
+__device__ __forceinline__ int64_t warp_sum64(int64_t v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// sum over b < b_end of pages_of(seq_lens[b]) (whole warp participates)
+__device__ int64_t pages_before(const int32_t *seq_lens, int b_end, int ps, int lane) {
+  int64_t s = 0;
+  for (int b0 = 0; b0 < b_end; b0 += 32) {
+    const int b = b0 + lane;
+    s += (b < b_end) ? pages_of(seq_lens[b], ps) : 0;
+  }
+  return warp_sum64(s);
+}
+
+// Find the batch b whose pages (H per page index) contain offset `rem` of a
+// row-group slab; returns b and H * (pages before b).
+__device__ void locate_batch(const int32_t *seq_lens, int B, int H, int ps, int64_t rem, int lane, int &b_out,
+                             int64_t &before_out) {
+  int64_t base = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const int64_t np = (b < B) ? static_cast<int64_t>(H) * pages_of(seq_lens[b], ps) : 0;
+    int64_t incl = np;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int64_t excl = incl - np;
+    const unsigned hit = __ballot_sync(0xffffffffu, base + excl <= rem && rem < base + incl);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      b_out = b0 + src;
+      before_out = __shfl_sync(0xffffffffu, base + excl, src);
+      return;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  b_out = B;
+  before_out = base;
+}
+
+struct Walk {
+  int rg, b, h, j, np, L;
+  __device__ void advance(const int32_t *seq_lens, int B, int H, int ps) {
+    if (++j < np) return;
+    j = 0;
+    if (++h < H) return;
+    h = 0;
+    do {
+      if (++b == B) { b = 0; ++rg; }
+      L = seq_lens[b];
+      np = pages_of(L, ps);
+    } while (np == 0);
+  }
+};
+
+// ------------------------------------------------------------ pair table
+// s_lut[idx * 32 + lane] = half2(C[idx & 7], C[idx >> 3]): one copy per lane
+// so that 32 lanes with 32 different indices hit 32 different banks.
+__shared__ __align__(16) uint32_t s_lut[64 * 32];
+
+// Byte offset of entry ((x >> sh) & 63) for this lane: the entry index lands
+// in bits 7..12 and the lane's bank in bits 2..6, so one AND-OR forms it.
+template <int SH>
+__device__ __forceinline__ uint32_t lut_off(uint32_t x, uint32_t lane4) {
+  const uint32_t y = (SH >= 0) ? (x >> (SH >= 0 ? SH : 0)) : (x << (SH < 0 ? -SH : 0));
+  return (y & 0x1F80u) | lane4;
+}
+__device__ __forceinline__ uint32_t lut_at(uint32_t off) {
+  return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(s_lut) + off);
+}
+// five adjacent-code pairs (2k, 2k+1), k = 0..4, of a packed word
+__device__ __forceinline__ void word_pairs(uint32_t w, uint32_t lane4, uint32_t *out) {
+  out[0] = lut_at(lut_off<-7>(w, lane4));
+  out[1] = lut_at(lut_off<-1>(w, lane4));
+  out[2] = lut_at(lut_off<5>(w, lane4));
+  out[3] = lut_at(lut_off<11>(w, lane4));
+  out[4] = lut_at(lut_off<17>(w, lane4));
+}
+
+__device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// ------------------------------------------------------------ partial kernel
+__global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gid = lane >> 2, tq = lane & 3;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarriers);
+  uint64_t *empty = full + kStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kLocate);
+  int64_t *loc = reinterpret_cast<int64_t *>(smem + kLocate + 8);
+  const int ps = p.page_size;
+
+  for (int e = tid; e < 64 * 32; e += kThreads) {
+    const int idx = e >> 5;
+    s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // CTA's page range [gs, ge) and where it starts
+  if (warp == 0) {
+    const int64_t pb = pages_before(p.seq_lens, p.B, ps, lane);
+    const int64_t p_rg = static_cast<int64_t>(p.H) * pb;
+    const int64_t total = p_rg * p.RG;
+    const int64_t gs = total * blockIdx.x / p.n_cta;
+    const int64_t ge = total * (blockIdx.x + 1) / p.n_cta;
+    int b = 0;
+    int64_t before = 0;
+    int64_t rem = 0, rg = 0;
+    if (gs < ge) {
+      rg = gs / p_rg;
+      rem = gs - rg * p_rg;
+      locate_batch(p.seq_lens, p.B, p.H, ps, rem, lane, b, before);
+    }
+    if (lane == 0) {
+      loc[0] = gs;
+      loc[1] = ge;
+      loc[2] = rg;
+      loc[3] = b;
+      loc[4] = rem - before;  // offset inside batch b's H * np pages
+    }
+  }
+  __syncthreads();
+  const int64_t gs = loc[0], ge = loc[1];
+  if (gs >= ge) return;
+  Walk wk;
+  wk.rg = static_cast<int>(loc[2]);
+  wk.b = static_cast<int>(loc[3]);
+  wk.L = p.seq_lens[wk.b];
+  wk.np = pages_of(wk.L, ps);
+  wk.h = static_cast<int>(loc[4] / wk.np);
+  wk.j = static_cast<int>(loc[4] - static_cast<int64_t>(wk.h) * wk.np);
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    int64_t it = 0;
+    for (int64_t g = gs; g < ge; ++g, ++it) {
+      const int stage = static_cast<int>(it % kStages);
+      const uint32_t round = static_cast<uint32_t>(it / kStages);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&empty[stage], (round & 1u) ^ 1u, p.status, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      int phys = -1;
+      if (wk.j < p.max_pages) phys = p.page_table[static_cast<int64_t>(wk.b) * p.max_pages + wk.j];
+      if (phys < 0 || phys >= p.num_pages) {
+        if (lane == 0) set_status(p.status, ISOQUANT_DEVERR_PAGE_RANGE);
+        phys = 0;
+      }
+      uint8_t *st = smem + static_cast<size_t>(stage) * kStageBytes;
+      if (lane == 0) mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(108 * ps));
+      __syncwarp();
+      const int64_t kblk = (static_cast<int64_t>(phys) * 2 + 0) * p.H + wk.h;
+      const int64_t vblk = (static_cast<int64_t>(phys) * 2 + 1) * p.H + wk.h;
+      if (lane < kWords) {
+        bulk_g2s(st + kStageKC + lane * kStrideK * 4, p.codes + (kblk * kWords + lane) * ps,
+                 static_cast<uint32_t>(ps * 4), &full[stage]);
+      } else if (lane < 2 * kWords) {
+        const int w = lane - kWords;
+        bulk_g2s(st + kStageVC + w * kStrideV * 4, p.codes + (vblk * kWords + w) * ps,
+                 static_cast<uint32_t>(ps * 4), &full[stage]);
+      } else if (lane == 2 * kWords) {
+        bulk_g2s(st + kStageKN, p.norms + kblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
+      } else if (lane == 2 * kWords + 1) {
+        bulk_g2s(st + kStageVN, p.norms + vblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
+      }
+      if (g + 1 < ge) wk.advance(p.seq_lens, p.B, p.H, ps);
+    }
+    // wait (bounded) for every copy still in flight before the CTA exits
+    if (lane == 0) {
+      const int64_t issued = it;
+      for (int64_t k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
+        mbar_wait(&full[k % kStages], static_cast<uint32_t>((k / kStages) & 1), p.status, nullptr);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+  float *sm_o = reinterpret_cast<float *>(smem + kScratchO);
+  float *sm_m = reinterpret_cast<float *>(smem + kScratchM);
+  float *sm_l = reinterpret_cast<float *>(smem + kScratchL);
+  float *sm_e = reinterpret_cast<float *>(smem + kScratchE);
+
+  // dims this thread feeds to Q.K^T: pair k (k = 0..15) = coordinates
+  // (kdim(k), kdim(k) + 1); pairs 0..14 come from words 3tq..3tq+2, pair 15
+  // from word 12.
+  auto kdim = [&](int k) -> int {
+    return k < 15 ? 10 * (3 * tq + k / 5) + 2 * (k % 5) : 120 + 2 * tq;
+  };
+  // dims this thread feeds to P.V (rows gid / gid+8 of each 16-dim tile):
+  // word gid fully, half of word 8 + gid/2, code gid of word 12.
+  const int par = gid & 1;
+  auto vdim = [&](int k) -> int {
+    if (k < 5) return 10 * gid + 2 * k;
+    if (k < 10) return 10 * gid + 2 * (k - 5) + 1;
+    if (k < 15) return 10 * (8 + (gid >> 1)) + par + 2 * (k - 10);
+    return 120 + gid;
+  };
+
+  uint32_t qa[8][4];
+  float acc[8][4];
+  float m_run = -INFINITY, l_run = 0.f, inv2e = 1.f;
+  int lim = 0, lim_min = 0, lim_max = 0;
+
+  int64_t it = 0;
+  for (int64_t g = gs; g < ge; ++g, ++it) {
+    const bool seg_start = (g == gs) || (wk.j == 0);
+    const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
+    if (seg_start) {
+      // load this pair's query rows as hi/lo fp16 A fragments
+      const int r = wk.rg * 8 + gid;
+      const bool valid = r < p.R;
+      const int qi = valid ? r / p.G : 0;
+      const int hq = wk.h * p.G + (valid ? r % p.G : 0);
+      const float *qp = p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD;
+      float qv[32];
+      float mx = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int d0 = kdim(k);
+        qv[2 * k] = valid ? qp[d0] * p.qfold : 0.f;
+        qv[2 * k + 1] = valid ? qp[d0 + 1] * p.qfold : 0.f;
+        mx = fmaxf(mx, fmaxf(fabsf(qv[2 * k]), fabsf(qv[2 * k + 1])));
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      // power-of-two prescale: the largest |q| lands in [2^14, 2^15)
+      int ex = 0;
+      if (mx > 0.f) frexpf(mx, &ex);
+      ex = max(ex, -100);
+      const float up = ldexpf(1.f, 15 - ex);
+      inv2e = ldexpf(1.f, ex - 15);
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float a = qv[2 * k] * up, b = qv[2 * k + 1] * up;
+        const __half ah = __float2half_rn(a), bh = __float2half_rn(b);
+        hi[k] = pack_half2(__half2float(ah), __half2float(bh));
+        lo[k] = pack_half2(a - __half2float(ah), b - __half2float(bh));
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        qa[c][0] = hi[2 * c];
+        qa[c][1] = lo[2 * c];
+        qa[c][2] = hi[2 * c + 1];
+        qa[c][3] = lo[2 * c + 1];
+      }
+      const int L = wk.L;
+      lim = valid ? (p.causal ? L - p.nq + qi + 1 : L) : L;
+      lim = max(lim, 0);
+      lim_min = p.causal ? max(L - p.nq + 1, 0) : L;
+      lim_max = L;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+      m_run = -INFINITY;
+      l_run = 0.f;
+    }
+
+    const int stage = static_cast<int>(it % kStages);
+    const uint32_t round = static_cast<uint32_t>(it / kStages);
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(&full[stage], round & 1u, p.status, abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    const uint8_t *st = smem + static_cast<size_t>(stage) * kStageBytes;
+    const uint32_t *kc = reinterpret_cast<const uint32_t *>(st + kStageKC);
+    const uint32_t *vc = reinterpret_cast<const uint32_t *>(st + kStageVC);
+    const __half *kn = reinterpret_cast<const __half *>(st + kStageKN);
+    const __half *vn = reinterpret_cast<const __half *>(st + kStageVN);
+
+    for (int sc = warp; ok && sc * 32 < ps; sc += kConsumerWarps) {
+      const int t0 = sc * 32;                       // token offset in the page
+      const int tok0 = wk.j * ps + t0;              // absolute position
+      if (tok0 >= lim_max) break;
+
+      // ---- scores: 4 n-tiles, tile j column n = token 4n + j
+      const uint4 kw0 = *reinterpret_cast<const uint4 *>(kc + (3 * tq + 0) * kStrideK + t0 + 4 * gid);
+      const uint4 kw1 = *reinterpret_cast<const uint4 *>(kc + (3 * tq + 1) * kStrideK + t0 + 4 * gid);
+      const uint4 kw2 = *reinterpret_cast<const uint4 *>(kc + (3 * tq + 2) * kStrideK + t0 + 4 * gid);
+      const uint4 kw3 = *reinterpret_cast<const uint4 *>(kc + 12 * kStrideK + t0 + 4 * gid);
+      float x[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t bf[16];
+        word_pairs(u4_at(kw0, j), lane4, bf + 0);
+        word_pairs(u4_at(kw1, j), lane4, bf + 5);
+        word_pairs(u4_at(kw2, j), lane4, bf + 10);
+        bf[15] = lut_at((((u4_at(kw3, j) << 7) >> (6 * tq)) & 0x1F80u) | lane4);
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mma16816(d, qa[c][0], qa[c][1], qa[c][2], qa[c][3], bf[2 * c], bf[2 * c + 1]);
+        x[j] = d[0] + d[2];        // token 8tq + j
+        x[4 + j] = d[1] + d[3];    // token 8tq + 4 + j
+      }
+      // ---- norms, masking, online softmax (row gid, tokens 8tq + i)
+      const uint4 knv = *reinterpret_cast<const uint4 *>(kn + t0 + 8 * tq);
+      const uint4 vnv = *reinterpret_cast<const uint4 *>(vn + t0 + 8 * tq);
+      float nk[8], nv[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&reinterpret_cast<const uint32_t *>(&knv)[i]));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&reinterpret_cast<const uint32_t *>(&vnv)[i]));
+        nk[2 * i] = a.x; nk[2 * i + 1] = a.y;
+        nv[2 * i] = b.x; nv[2 * i + 1] = b.y;
+      }
+      const bool mask = tok0 + 32 > lim_min;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float v = x[i] * nk[i];
+        if (mask && tok0 + 8 * tq + i >= lim) v = -INFINITY;
+        x[i] = v;
+        mx = fmaxf(mx, v);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run, mx);
+      if (__any_sync(0xffffffffu, m_new > m_run)) {
+        const float corr = (m_run == -INFINITY) ? 0.f : exp2f((m_run - m_new) * inv2e);
+        l_run *= corr;
+        const float c0 = __shfl_sync(0xffffffffu, corr, (2 * tq) * 4);
+        const float c1 = __shfl_sync(0xffffffffu, corr, (2 * tq + 1) * 4);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          acc[m][0] *= c0; acc[m][1] *= c1; acc[m][2] *= c0; acc[m][3] *= c1;
+        }
+        m_run = m_new;
+      }
+      const float mm = (m_run == -INFINITY) ? 0.f : m_run * inv2e;
+      float pv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float pr = exp2f(fmaf(x[i], inv2e, -mm));
+        l_run += pr;
+        pv[i] = pr > 0.f ? pr * nv[i] : 0.f;
+      }
+      // ---- P.V: O^T[16 dims x 8 rows] += V^T[16 dims x 16 tok] P^T
+      const uint4 va0 = *reinterpret_cast<const uint4 *>(vc + gid * kStrideV + t0 + 8 * tq);
+      const uint4 va1 = *reinterpret_cast<const uint4 *>(vc + gid * kStrideV + t0 + 8 * tq + 4);
+      const uint4 vb0 = *reinterpret_cast<const uint4 *>(vc + (8 + (gid >> 1)) * kStrideV + t0 + 8 * tq);
+      const uint4 vb1 = *reinterpret_cast<const uint4 *>(vc + (8 + (gid >> 1)) * kStrideV + t0 + 8 * tq + 4);
+      const uint4 vz0 = *reinterpret_cast<const uint4 *>(vc + 12 * kStrideV + t0 + 8 * tq);
+      const uint4 vz1 = *reinterpret_cast<const uint4 *>(vc + 12 * kStrideV + t0 + 8 * tq + 4);
+      constexpr uint32_t M = 0x071C71C7u;  // even-indexed 3-bit fields
+#pragma unroll
+      for (int kap = 0; kap < 2; ++kap) {
+        uint32_t va[2][16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int tp = 2 * kap + half;  // token pair (2tp, 2tp+1) of this thread's 8
+          const uint4 &A = tp < 2 ? va0 : va1;
+          const uint4 &Bv = tp < 2 ? vb0 : vb1;
+          const uint4 &Z = tp < 2 ? vz0 : vz1;
+          const int e0 = (tp & 1) * 2;
+          const uint32_t wa = u4_at(A, e0), wa1 = u4_at(A, e0 + 1);
+          const uint32_t wb = u4_at(Bv, e0), wb1 = u4_at(Bv, e0 + 1);
+          const uint32_t wz = u4_at(Z, e0), wz1 = u4_at(Z, e0 + 1);
+          // merge two tokens' words: 6-bit slot k = (code of tok a, code of tok b)
+          const uint32_t e_even = (wa & M) | ((wa1 << 3) & ~M);
+          const uint32_t e_odd = ((wa >> 3) & M) | (wa1 & ~M);
+          const uint32_t e_half = ((wb >> (3 * par)) & M) | ((wb1 << (3 - 3 * par)) & ~M);
+          word_pairs(e_even, lane4, va[half] + 0);
+          word_pairs(e_odd, lane4, va[half] + 5);
+          word_pairs(e_half, lane4, va[half] + 10);
+          const uint32_t z12 = (((wz >> (3 * gid)) & 7u) << 7) | (((wz1 >> (3 * gid)) & 7u) << 10);
+          va[half][15] = lut_at(z12 | lane4);
+        }
+        const uint32_t b0 = pack_half2(pv[4 * kap + 0], pv[4 * kap + 1]);
+        const uint32_t b1 = pack_half2(pv[4 * kap + 2], pv[4 * kap + 3]);
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          mma16816(acc[m], va[0][2 * m], va[0][2 * m + 1], va[1][2 * m], va[1][2 * m + 1], b0, b1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+
+    if (seg_end) {
+      // ---- merge the 8 warps' states and write one record
+      float l_tot = l_run;
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
+      l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+      float *o_w = sm_o + warp * 8 * kD;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        o_w[(2 * tq) * kD + vdim(2 * m)] = acc[m][0];
+        o_w[(2 * tq + 1) * kD + vdim(2 * m)] = acc[m][1];
+        o_w[(2 * tq) * kD + vdim(2 * m + 1)] = acc[m][2];
+        o_w[(2 * tq + 1) * kD + vdim(2 * m + 1)] = acc[m][3];
+      }
+      if (tq == 0) {
+        sm_m[warp * 8 + gid] = m_run;
+        sm_l[warp * 8 + gid] = l_tot;
+        if (warp == 0) sm_e[gid] = inv2e;
+      }
+      named_bar_sync(1, kConsumerWarps * 32);
+      const int row = tid >> 5, d0 = (tid & 31) * 4;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * 8 + row]);
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      float l = 0.f;
+      if (M != -INFINITY) {
+        const float e = sm_e[row];
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float s = exp2f((sm_m[w * 8 + row] - M) * e);
+          l += s * sm_l[w * 8 + row];
+          const float4 ow = *reinterpret_cast<const float4 *>(sm_o + (w * 8 + row) * kD + d0);
+          o.x += s * ow.x; o.y += s * ow.y; o.z += s * ow.z; o.w += s * ow.w;
+        }
+        M *= e;  // to log2 units
+      }
+      const int64_t pair = (static_cast<int64_t>(wk.rg) * p.B + wk.b) * p.H + wk.h;
+      float *rec = p.records + (blockIdx.x + pair) * static_cast<int64_t>(kRecordFloats);
+      if ((tid & 31) == 0) {
+        rec[2 * row] = M;
+        rec[2 * row + 1] = l;
+      }
+      *reinterpret_cast<float4 *>(rec + 16 + row * kD + d0) = o;
+      named_bar_sync(1, kConsumerWarps * 32);
+    }
+    if (g + 1 < ge) wk.advance(p.seq_lens, p.B, p.H, ps);
+  }
+}
+
+// ------------------------------------------------------------ combine kernel
+__global__ void __launch_bounds__(256) k_attend_combine(const CombineParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_rows = static_cast<int64_t>(p.B) * p.nq * p.Hq;
+  if (row_id >= n_rows) return;
+  const int hq = static_cast<int>(row_id % p.Hq);
+  const int64_t bi = row_id / p.Hq;
+  const int i = static_cast<int>(bi % p.nq);
+  const int b = static_cast<int>(bi / p.nq);
+  const int h = hq / p.G, g = hq % p.G;
+  const int r = i * p.G + g, rg = r >> 3, rr = r & 7;
+  const int ps = p.page_size;
+  float *dst = p.out + row_id * kD + 4 * lane;
+
+  const int np = pages_of(p.seq_lens[b], ps);
+  const int64_t p_rg = static_cast<int64_t>(p.H) * pages_before(p.seq_lens, p.B, ps, lane);
+  if (np == 0) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const int64_t total = p_rg * p.RG;
+  const int64_t g0 = rg * p_rg + static_cast<int64_t>(p.H) * pages_before(p.seq_lens, b, ps, lane) +
+                     static_cast<int64_t>(h) * np;
+  const int64_t N = p.n_cta;
+  auto cta_of = [&](int64_t gg) -> int64_t { return ((gg + 1) * N + total - 1) / total - 1; };
+  const int64_t c_lo = cta_of(g0), c_hi = cta_of(g0 + np - 1);
+  const int64_t pair = (static_cast<int64_t>(rg) * p.B + b) * p.H + h;
+
+  // CTAs with an empty page range (possible when there are fewer pages than
+  // CTAs) wrote no record: skip them
+  auto empty_cta = [&](int64_t c) -> bool { return c * total / N == (c + 1) * total / N; };
+  float M = -INFINITY;
+  for (int64_t c = c_lo; c <= c_hi; ++c)
+    if (!empty_cta(c)) M = fmaxf(M, p.records[(c + pair) * kRecordFloats + 2 * rr]);
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  float l = 0.f;
+  if (M != -INFINITY) {
+    for (int64_t c = c_lo; c <= c_hi; ++c) {
+      if (empty_cta(c)) continue;
+      const float *rec = p.records + (c + pair) * kRecordFloats;
+      const float s = exp2f(rec[2 * rr] - M);
+      l += s * rec[2 * rr + 1];
+      const float4 v = *reinterpret_cast<const float4 *>(rec + 16 + rr * kD + 4 * lane);
+      o[0] += s * v.x; o[1] += s * v.y; o[2] += s * v.z; o[3] += s * v.w;
+    }
+  }
+  if (M == -INFINITY || !(l > 0.f)) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  // o~ = sum p n C / (l sqrt(128)); then R^-1 = D Hn B^T, Hn = H / sqrt(128)
+  const float inv = 1.f / (l * 128.f);
+  const HeadParams &hp = p.params[h];
+  const float *mb = hp.m32[lane];
+  float y[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    y[c] = fmaf(mb[12 + c], o[3], fmaf(mb[8 + c], o[2], fmaf(mb[4 + c], o[1], mb[c] * o[0])));
+  wht128<float>(y, lane);
+  const uint32_t sn = (hp.sign_bits[lane >> 3] >> (4 * (lane & 7))) & 0xFu;
+  float res[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) res[c] = __uint_as_float(__float_as_uint(y[c] * inv) ^ (((sn >> c) & 1u) << 31));
+  *reinterpret_cast<float4 *>(dst) = make_float4(res[0], res[1], res[2], res[3]);
+}
+
+}  // namespace
+
+size_t attend_workspace_bytes(const AttendShape &s) {
+  return kWsHeader + s.slots * kRecordFloats * sizeof(float);
+}
+
+cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache, const AttendShape &s,
+                                  const float *q_rot, const int32_t *page_table, int max_pages,
+                                  const int32_t *seq_lens, float scale, void *ws, cudaStream_t stream) {
+  static int configured_device = -1;
+  if (configured_device != ctx->device) {
+    cudaError_t e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = ctx->device;
+  }
+  PartialParams p{};
+  p.codes = cache->codes;
+  p.norms = cache->norms;
+  p.num_pages = cache->num_pages;
+  p.page_size = cache->page_size;
+  p.q_rot = q_rot;
+  p.page_table = page_table;
+  p.max_pages = max_pages;
+  p.seq_lens = seq_lens;
+  p.B = s.batch;
+  p.nq = s.nq;
+  p.Hq = s.q_heads;
+  p.H = s.kv_heads;
+  p.G = s.group;
+  p.R = s.rows;
+  p.RG = s.row_groups;
+  p.causal = s.causal;
+  p.qfold = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 / std::sqrt(128.0));
+  for (int i = 0; i < kLevels; ++i) p.level[i] = ctx->codebook.level[i];
+  p.records = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
+  p.status = ctx->status;
+  p.n_cta = s.n_cta;
+  k_attend_partial<<<s.n_cta, kThreads, kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s, const int32_t *seq_lens,
+                                  const void *ws, float *out, cudaStream_t stream) {
+  CombineParams p{};
+  p.records = reinterpret_cast<const float *>(static_cast<const char *>(ws) + kWsHeader);
+  p.params = ctx->params;
+  p.seq_lens = seq_lens;
+  p.out = out;
+  p.B = s.batch;
+  p.nq = s.nq;
+  p.Hq = s.q_heads;
+  p.H = s.kv_heads;
+  p.G = s.group;
+  p.RG = s.row_groups;
+  p.page_size = s.page_size;
+  p.n_cta = s.n_cta;
+  const int64_t rows = static_cast<int64_t>(s.batch) * s.nq * s.q_heads;
+  const int64_t blocks = (rows * 32 + 255) / 256;
+  if (blocks == 0) return cudaSuccess;
+  k_attend_combine<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace isoquant

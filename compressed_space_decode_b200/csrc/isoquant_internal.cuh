@@ -1,0 +1,106 @@
+// isoquant_internal.cuh -- shared definitions of the CUDA library (sm_100a).
+//
+// Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via
+// Fused Compressed-Space Attention", Abstract (WHT + block-diagonal SO(4)
+// isotropization, 3-bit scalar quantization, attention on packed codes).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/isoquant.h"
+
+namespace isoquant {
+
+constexpr int kD = 128;
+constexpr int kBlocks = 32;
+constexpr int kWords = 13;
+constexpr int kLevels = 8;
+
+// Per-head parameter block in device memory.
+struct HeadParams {
+  float m32[kBlocks][16];    // SO(4) block matrices, row-major, y' = M y
+  double m64[kBlocks][16];   // same in fp64 (exact re-check near thresholds)
+  uint32_t sign_bits[4];     // bit j set <=> sign_j = -1
+  uint32_t pad[4];
+};
+
+// Codebook handed to the kernels by value.
+struct Codebook {
+  float level[kLevels];       // fp16-rounded Lloyd-Max levels, ascending
+  float threshold[kLevels - 1];
+  double threshold64[kLevels - 1];
+  uint16_t level16[kLevels];  // fp16 bits of the levels
+};
+
+}  // namespace isoquant
+
+struct isoquant_ctx {
+  int device;
+  int num_kv_heads;
+  int num_sms;
+  isoquant::HeadParams *params;  // device [num_kv_heads]
+  uint32_t *status;              // device, 16 bytes
+  isoquant::Codebook codebook;
+  int last_launches;
+};
+
+namespace isoquant {
+
+// ------------------------------------------------------------ host helpers
+int build_codebook(Codebook *cb);
+
+// launchers (defined in compress.cu / attend.cu)
+cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k,
+                            const void *v, int dtype, int n_tok, const int64_t *slot_mapping,
+                            cudaStream_t stream);
+cudaError_t launch_rotate_q(const isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
+                            int num_q_heads, float *q_rot, cudaStream_t stream);
+
+struct AttendShape {
+  int batch, nq, q_heads, kv_heads, group, rows, row_groups, page_size, causal;
+  int n_cta;
+  size_t slots;       // partial records
+};
+constexpr size_t kWsHeader = 256;
+constexpr size_t kRecordFloats = 8 * 2 + 8 * kD;  // (m,l) x 8 rows, o[8][128]
+
+size_t attend_workspace_bytes(const AttendShape &s);
+cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache,
+                                  const AttendShape &s, const float *q_rot, const int32_t *page_table,
+                                  int max_pages, const int32_t *seq_lens, float scale, void *ws,
+                                  cudaStream_t stream);
+cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
+                                  const int32_t *seq_lens, const void *ws, float *out,
+                                  cudaStream_t stream);
+
+// ------------------------------------------------------------ device helpers
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void set_status(uint32_t *status, uint32_t bits) {
+  atomicOr(status, bits);
+}
+
+// Sylvester WHT (unnormalised) of 128 values held 4 per lane, lane l holding
+// elements 4l..4l+3.  Strides 1 and 2 are inside a lane; strides 4..64 pair
+// lanes l and l^(stride/4).  The lower index of each butterfly keeps a+b,
+// the upper one a-b.
+template <typename T>
+__device__ __forceinline__ void wht128(T (&v)[4], int lane) {
+  T a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
+  v[0] = a0 + a2; v[1] = a1 + a3; v[2] = a0 - a2; v[3] = a1 - a3;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      T p = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? (p - v[i]) : (v[i] + p);
+    }
+  }
+}
+
+}  // namespace isoquant

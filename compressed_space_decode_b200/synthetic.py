@@ -165,3 +165,53 @@ def workloads(small: bool = False) -> dict:
         layers=48 if not small else 2, shuffle_pages=False,
         note="bulk compression of a 32768-token prompt x 8 KV heads x 48 layers (K and V)")
     return w
+
+
+# ------------------------------------------------------- workload streams
+CHUNK = 4096  # tokens per independently seeded K/V chunk
+
+
+def workload_scales(wl):
+    """(K scales, V scales) of a heavy-tailed workload, or (None, None)."""
+    if wl.kind != "heavy":
+        return None, None
+    return channel_scales(wl.seed, 0, wl.kv_heads), channel_scales(wl.seed, 1, wl.kv_heads)
+
+
+def workload_kv_chunk(wl, b, c, device="cpu", scales=None):
+    """K, V [CHUNK][H][128] of tokens [c*CHUNK, (c+1)*CHUNK) of sequence b."""
+    sid = (b * 100003 + c) * 2
+    if wl.kind == "heavy":
+        ks, vs = scales if scales is not None else workload_scales(wl)
+        return (heavy_tailed(wl.seed, sid, CHUNK, ks, device=device),
+                heavy_tailed(wl.seed, sid + 1, CHUNK, vs, device=device))
+    return (gaussian_with_outliers(wl.seed, sid, CHUNK, wl.kv_heads, device=device),
+            gaussian_with_outliers(wl.seed, sid + 1, CHUNK, wl.kv_heads, device=device))
+
+
+def workload_kv_tokens(wl, b, t0, t1, device="cpu", scales=None):
+    """K, V of tokens [t0, t1) of sequence b, chunk by chunk."""
+    ks, vs = [], []
+    t = t0
+    while t < t1:
+        c = t // CHUNK
+        k, v = workload_kv_chunk(wl, b, c, device=device, scales=scales)
+        a, e = t - c * CHUNK, min(t1 - c * CHUNK, CHUNK)
+        ks.append(k[a:e])
+        vs.append(v[a:e])
+        t = c * CHUNK + e
+    if not ks:
+        shape = (0, wl.kv_heads, D)
+        dt = torch.bfloat16 if wl.kind == "heavy" else torch.float32
+        return torch.empty(shape, dtype=dt, device=device), torch.empty(shape, dtype=dt, device=device)
+    return torch.cat(ks), torch.cat(vs)
+
+
+def workload_queries(wl, step, device="cpu", nq=None):
+    """Queries [B][nq][Hq][128] of decode step `step` (N(0,1); fp32 with the
+    x10 outlier channels for the Gaussian workload, bf16 otherwise)."""
+    nq = nq or wl.nq
+    if wl.kind == "gaussian":
+        return gaussian_with_outliers(wl.seed, 10_000_000 + step, wl.batch * nq, wl.q_heads,
+                                      device=device).reshape(wl.batch, nq, wl.q_heads, D)
+    return gaussian(wl.seed, 10_000_000 + step, (wl.batch, nq, wl.q_heads, D), device=device, dtype=torch.bfloat16)

@@ -1,0 +1,183 @@
+/*
+ * isoquant.h -- C ABI of the IsoQuant compressed-space attention library
+ * (B200 / sm_100a).
+ *
+ * Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via
+ * Fused Compressed-Space Attention" (arXiv 2608.08081), Abstract.  Each K/V
+ * head vector (d = 128) is isotropized by a Walsh-Hadamard transform
+ * followed by 32 block-diagonal SO(4) rotations (256 stored parameters per
+ * head), then quantized to 3-bit scalar codes; attention runs directly on
+ * the packed codes, and full-precision KV is never materialised.
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   R = B * Hn * D: D = diag(signs), Hn = Sylvester Hadamard / sqrt(128)
+ *   (natural order), B = 32 SO(4) blocks, block b acting on coordinates
+ *   4b..4b+3 as the quaternion (w,x,y,z) by v -> qL (x) v (x) conj(qR).
+ *   Per vector: n = ||x||_2 (fp64) stored as fp16 (nearest even, saturating
+ *   at 65504); z = sqrt(128) * (R x) / n; code_j = #{k : z_j > t_k} with the
+ *   8-level Lloyd-Max levels for N(0,1) rounded to fp16 (ascending, code 0 =
+ *   most negative) and t_k the midpoints of adjacent levels.  Ten codes per
+ *   32-bit word, code j at bits 3*(j%10) of word j/10, 13 words per vector.
+ *   Attention: s_t = scale * (n16_t / sqrt(128)) * <R q, C[code_t]>,
+ *   softmax over visible tokens, o = R^-1 sum_t p_t (n16v_t/sqrt(128))
+ *   C[codev_t].
+ *
+ * Memory: every device buffer is owned by the caller, except the per-head
+ * parameter block and a 16-byte status word that isoquant_init allocates and
+ * isoquant_destroy frees.  No call below allocates, frees or synchronises,
+ * except isoquant_init, isoquant_destroy and isoquant_get_status.
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ * default stream); all work is enqueued asynchronously on it.
+ * Errors: every call returns an isoquant_status.  Argument errors are found
+ * on the host before anything is launched; a failed launch returns
+ * ISOQUANT_ERR_CUDA.  Errors the host cannot see (a device index out of
+ * range, a bounded device-side wait that expired) set bits in the context's
+ * status word, read with isoquant_get_status.
+ */
+#ifndef ISOQUANT_H
+#define ISOQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ISOQUANT_HEAD_DIM 128
+#define ISOQUANT_WORDS_PER_VECTOR 13
+#define ISOQUANT_PARAMS_PER_HEAD 256
+
+typedef enum {
+  ISOQUANT_OK = 0,
+  ISOQUANT_ERR_INVALID_ARG = -1,   /* null pointer, bad count or size */
+  ISOQUANT_ERR_UNSUPPORTED = -2,   /* head_dim != 128, unknown dtype, page size */
+  ISOQUANT_ERR_OUT_OF_RANGE = -3,  /* an index or length outside its buffer */
+  ISOQUANT_ERR_WORKSPACE = -4,     /* workspace too small */
+  ISOQUANT_ERR_CUDA = -5,          /* a CUDA runtime call failed */
+  ISOQUANT_ERR_ALIGNMENT = -6      /* a pointer is not 16-byte aligned */
+} isoquant_status;
+
+/* device status bits (isoquant_get_status) */
+#define ISOQUANT_DEVERR_WAIT_TIMEOUT 1u   /* a bounded pipeline wait expired */
+#define ISOQUANT_DEVERR_PAGE_RANGE 2u     /* page_table entry outside [0, num_pages) */
+#define ISOQUANT_DEVERR_SLOT_RANGE 4u     /* slot_mapping entry outside the cache */
+
+typedef enum {
+  ISOQUANT_F32 = 0,
+  ISOQUANT_BF16 = 1,
+  ISOQUANT_F16 = 2
+} isoquant_dtype;
+
+typedef struct isoquant_ctx isoquant_ctx;
+
+/* Paged packed KV cache, caller-owned device memory.
+ *   codes: uint32 [num_pages][2 (K,V)][num_kv_heads][13][page_size]
+ *          (word-major inside a page: word w of every token, then word w+1)
+ *   norms: uint16 (fp16 bits) [num_pages][2][num_kv_heads][page_size]
+ * Token t of a sequence lives in page page_table[b][t / page_size] at
+ * offset t % page_size.  page_size must be 32, 64, 128 or 256; both
+ * pointers 16-byte aligned.  Bytes per token and KV head: 2 * (52 + 2). */
+typedef struct {
+  uint32_t *codes;
+  uint16_t *norms;
+  int32_t num_pages;
+  int32_t page_size;
+} isoquant_cache;
+
+/* Create a context for `num_kv_heads` heads on the current CUDA device.
+ *   head_dim: must be 128 (RotaryQuant, Abstract: 256 parameters per head
+ *             = 32 SO(4) blocks x 2 unit quaternions x 4).
+ *   signs:    host int8 [num_kv_heads][128], each +1 or -1 (the D of R).
+ *   quats:    host float [num_kv_heads][32][2][4], (w,x,y,z), left then
+ *             right quaternion of each block; normalised here in fp64.
+ * Allocates the device parameter block (per head: 2 KB fp32 and 4 KB fp64
+ * block matrices, 16 B of sign bits) and the status word.  Synchronous.
+ * Errors: INVALID_ARG (null, num_kv_heads < 1, a sign not +-1, a zero or
+ * non-finite quaternion), UNSUPPORTED (head_dim), CUDA. */
+int isoquant_init(isoquant_ctx **out, int num_kv_heads, int head_dim,
+                  const int8_t *signs, const float *quats);
+
+/* Free the context and its device memory (synchronises the device). */
+void isoquant_destroy(isoquant_ctx *ctx);
+
+/* Human-readable text for an isoquant_status. */
+const char *isoquant_strerror(int status);
+
+/* The library's own codebook (host only, no device work): the 8 fp16-
+ * rounded Lloyd-Max levels for N(0,1), ascending, widened to float, and the
+ * 7 decision thresholds (midpoints, exact in float). */
+int isoquant_codebook(float levels[8], float thresholds[7]);
+
+/* Bytes of the two cache arrays for `num_pages` pages. */
+int isoquant_cache_bytes(const isoquant_ctx *ctx, int num_pages, int page_size,
+                         size_t *code_bytes, size_t *norm_bytes);
+
+/* Rotate, quantize, pack and append K and V vectors into the paged cache.
+ *   k, v:  device [n_tok][num_kv_heads][128] of `dtype` (F32, BF16, F16),
+ *          contiguous, 8-byte aligned.
+ *   slot_mapping: device int64 [n_tok], slot = page * page_size + offset;
+ *          a negative slot skips that token; a slot beyond the cache sets
+ *          ISOQUANT_DEVERR_SLOT_RANGE and is skipped.
+ * Writes 13 code words and one fp16 norm per (token, head, K/V).
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA. */
+int isoquant_compress_kv(isoquant_ctx *ctx, const isoquant_cache *cache,
+                         const void *k, const void *v, int dtype, int n_tok,
+                         const int64_t *slot_mapping, void *stream);
+
+/* q_rot = R q for every row: q device [n_rows][num_q_heads][128] of dtype,
+ * q_rot device float [n_rows][num_q_heads][128].  Query head h uses the
+ * rotation of KV head h / (num_q_heads / num_kv_heads). */
+int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
+                      int num_q_heads, float *q_rot, void *stream);
+
+/* Workspace bytes isoquant_attend_decode needs for this shape. */
+int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
+                            int num_q_heads, size_t *bytes);
+
+/* Split-context decode attention over the packed cache, then the combine
+ * step that merges the splits and applies R^-1 once.
+ *   q_rot:      device float [batch][nq][num_q_heads][128] (from rotate_q)
+ *   page_table: device int32 [batch][max_pages]
+ *   seq_lens:   device int32 [batch]; tokens 0..seq_lens[b]-1 are in the
+ *               cache (including the nq query positions' own K/V)
+ *   causal:     if nonzero, query position i sees tokens
+ *               t <= seq_lens[b] - nq + i; otherwise all seq_lens[b] tokens
+ *   scale:      softmax scale; 0 selects 1/sqrt(128)
+ *   workspace:  device, >= isoquant_workspace_size bytes, 16-byte aligned
+ *   out:        device float [batch][nq][num_q_heads][128]
+ * A row that sees no token outputs zeros.  Rows of heads in one GQA group
+ * share each KV tile.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE,
+ * ALIGNMENT, CUDA. */
+int isoquant_attend_decode(isoquant_ctx *ctx, const isoquant_cache *cache,
+                           const float *q_rot, int batch, int nq,
+                           int num_q_heads, const int32_t *page_table,
+                           int max_pages, const int32_t *seq_lens, int causal,
+                           float scale, void *workspace, size_t ws_bytes,
+                           float *out, void *stream);
+
+/* The two halves of isoquant_attend_decode, for callers that schedule them
+ * separately (same arguments; the partial half fills the workspace, the
+ * combine half reads it and writes `out`). */
+int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache,
+                            const float *q_rot, int batch, int nq,
+                            int num_q_heads, const int32_t *page_table,
+                            int max_pages, const int32_t *seq_lens, int causal,
+                            float scale, void *workspace, size_t ws_bytes,
+                            void *stream);
+int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq,
+                            int num_q_heads, const int32_t *seq_lens,
+                            int page_size, const void *workspace,
+                            size_t ws_bytes, float *out, void *stream);
+
+/* Copy the device status word to *status and clear it (synchronises the
+ * stream).  0 means no device-side error since the last call. */
+int isoquant_get_status(isoquant_ctx *ctx, uint32_t *status, void *stream);
+
+/* Number of kernels the most recent call on this context launched. */
+int isoquant_last_launch_count(const isoquant_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ISOQUANT_H */

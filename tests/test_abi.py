@@ -1,0 +1,68 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+declared in include/isoquant.h, and its host-only parts behave (CPU only:
+no device work is started here)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "isoquant.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:int|void|const char \*)\s*\*?\s*(isoquant_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def native():
+    from compressed_space_decode_b200 import build
+    build.build()
+    import compressed_space_decode_b200 as csd
+    return csd
+
+
+def test_header_declares_the_four_calls():
+    syms = declared_symbols()
+    for name in ("isoquant_init", "isoquant_compress_kv", "isoquant_rotate_q", "isoquant_attend_decode"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(native):
+    L = native.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert sorted(native.SYMBOLS) == declared_symbols()
+
+
+def test_codebook_matches_oracle(native):
+    lv, th = native.isoquant_codebook()
+    ol, ot = oracle.codebook()
+    np.testing.assert_array_equal(np.array(lv, dtype=np.float64), ol)
+    np.testing.assert_array_equal(np.array(th, dtype=np.float64), ot)
+
+
+def test_strerror_and_argument_errors(native):
+    L = native.lib()
+    assert native.strerror(0) == "ok"
+    assert "workspace" in native.strerror(-4)
+    h = ctypes.c_void_p()
+    signs = np.ones((1, 128), np.int8)
+    quats = np.zeros((1, 32, 2, 4), np.float32)
+    quats[..., 0] = 1
+    # rejected on the host before any CUDA call
+    assert L.isoquant_init(None, 1, 128, signs.ctypes.data, quats.ctypes.data) == -1
+    assert L.isoquant_init(ctypes.byref(h), 1, 64, signs.ctypes.data, quats.ctypes.data) == -2
+    assert L.isoquant_init(ctypes.byref(h), 0, 128, signs.ctypes.data, quats.ctypes.data) == -1
+    bad = signs.copy()
+    bad[0, 3] = 0
+    assert L.isoquant_init(ctypes.byref(h), 1, 128, bad.ctypes.data, quats.ctypes.data) == -1
+    zq = np.zeros_like(quats)
+    assert L.isoquant_init(ctypes.byref(h), 1, 128, signs.ctypes.data, zq.ctypes.data) == -1
+    assert L.isoquant_compress_kv(None, None, None, None, 0, 1, None, None) == -1
+    assert L.isoquant_attend_decode(None, None, None, 1, 1, 8, None, 1, None, 0, 0.0, None, 0, None, None) == -1

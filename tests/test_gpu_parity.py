@@ -1,0 +1,241 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bit-exact packed codes and fp16 norms (coordinates within 1e-6 of a decision
+threshold counted and exempt), and attention outputs within 2e-3 normwise
+per row, on every workload at sizes the oracle finishes in seconds, plus
+full-size runs checked on sampled (sequence, KV head) pairs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity import ATTN_TOL, compare_compressed, oracle_rows, rowwise_rel_err
+
+pytestmark = pytest.mark.gpu
+
+D = 128
+
+
+def _ws(csd, st):
+    # NaN-filled so that reading a record nobody wrote shows up as NaN
+    return csd.alloc_workspace(st.ctx, st.B, st.wl.nq, st.Hq).fill_(0x7FC00000)
+
+
+def run_attend(csd, st, step=0, scale=0.0, q=None):
+    wl = st.wl
+    nq = wl.nq
+    if q is None:
+        q = st.queries(step)
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    csd.isoquant_rotate_q(st.ctx, q.reshape(st.B * nq, st.Hq, D), q_rot.view(st.B * nq, st.Hq, D))
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    ws = _ws(csd, st)
+    csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, ws, out,
+                               causal=wl.causal, scale=scale)
+    torch.cuda.synchronize()
+    assert csd.isoquant_get_status(st.ctx) == 0
+    return q.float().cpu(), q_rot.cpu(), out.cpu()
+
+
+def limits(wl):
+    if wl.causal:
+        return lambda L, i: max(L - wl.nq + i + 1, 0)
+    return lambda L, i: L
+
+
+def check_pair(st, b, h, q_cpu, out, scale=None, report=None):
+    L = st.seq_lens[b]
+    k, v = st.kv_tokens(b, 0, L) if L > 0 else (None, None)
+    s, qt = st.signs[h].numpy(), st.quats[h].numpy()
+    if L > 0:
+        gkc, gkn = st.gather(b, h, 0, 0, L)
+        gvc, gvn = st.gather(b, h, 1, 0, L)
+        k64 = k[:, h].to(torch.float64).cpu().numpy()
+        v64 = v[:, h].to(torch.float64).cpu().numpy()
+        ks, kc, kn = compare_compressed(k64, s, qt, gkc.numpy(), gkn.numpy())
+        vs, vc, vn = compare_compressed(v64, s, qt, gvc.numpy(), gvn.numpy())
+        if report is not None:
+            report.append((b, h, ks, vs))
+    else:
+        kc = vc = np.zeros((0, 13), np.uint32)
+        kn = vn = np.zeros(0, np.uint16)
+    ref, idx = oracle_rows(st, b, h, q_cpu, limits(st.wl), (kc, kn, vc, vn), scale=scale)
+    got = np.stack([out[b, i, hq].numpy() for (i, hq) in idx])
+    err = rowwise_rel_err(got, ref)
+    assert np.isfinite(got).all()
+    assert err.max() <= ATTN_TOL, f"b={b} h={h} max row rel err {err.max():.3e}"
+    return err.max()
+
+
+SMALL = ["single_head_d128_L1024", "gqa_b1_q32_kv8_L4096", "gqa_b16_q32_kv4_L32768_paged",
+         "long_b4_q64_kv8_L64k_128k_ragged", "verify_b8_nq16_q32_kv8_L16384"]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_attend_small(cuda_lib, name):
+    from compressed_space_decode_b200.workload import DecodeState
+    wl = cuda_lib.synthetic.workloads(small=True)[name]
+    st = DecodeState(wl)
+    q, _, out = run_attend(cuda_lib, st)
+    rng = np.random.default_rng(0)
+    pairs = [(b, h) for b in range(st.B) for h in range(st.H)]
+    if len(pairs) > 6:
+        pairs = [pairs[i] for i in rng.choice(len(pairs), 6, replace=False)]
+    worst = max(check_pair(st, b, h, q, out) for b, h in pairs)
+    print(f"{name}: worst row rel err {worst:.2e}")
+
+
+def test_compress_bit_exact_all_dtypes(cuda_lib):
+    """Heavy-tailed, Gaussian, zero, tiny and huge vectors; fp32/bf16/fp16 inputs."""
+    from compressed_space_decode_b200 import synthetic
+    H, n = 2, 3000
+    signs, quats = synthetic.rotation_params(77, H)
+    ctx = cuda_lib.isoquant_init(signs, quats)
+    cache = cuda_lib.PagedCache.allocate(H, (n + 255) // 256, 256)
+    sc = synthetic.channel_scales(78, 0, H)
+    base = synthetic.heavy_tailed(79, 0, n, sc, device="cuda", dtype=torch.float32)
+    base[:200] = synthetic.gaussian(80, 0, (200, H, D), device="cuda")
+    base[200] = 0.0
+    base[201] = 1e-3 * base[202]
+    base[203, :, 5] = 70000.0  # saturating norm
+    for dtype in (torch.float32, torch.bfloat16, torch.float16):
+        x = base.to(dtype)
+        if dtype == torch.float16:
+            x = torch.nan_to_num(x, posinf=60000.0, neginf=-60000.0).clamp(-60000, 60000)
+        slots = torch.arange(n, dtype=torch.int64, device="cuda")
+        cuda_lib.isoquant_compress_kv(ctx, cache, x, x.flip(0).contiguous(), slots)
+        torch.cuda.synchronize()
+        assert cuda_lib.isoquant_get_status(ctx) == 0
+        for h in range(H):
+            codes = cache.codes[:, 0, h].permute(0, 2, 1).reshape(-1, 13)[:n]
+            norms = cache.norms[:, 0, h].reshape(-1)[:n]
+            gc = codes.cpu().numpy().view(np.uint32)
+            gn = norms.cpu().numpy().view(np.uint16)
+            x64 = x[:, h].to(torch.float64).cpu().numpy()
+            stats, _, _ = compare_compressed(x64, signs[h].numpy(), quats[h].numpy(), gc, gn)
+            print(dtype, h, stats)
+
+
+def test_compress_slot_rules(cuda_lib):
+    from compressed_space_decode_b200 import synthetic
+    H = 1
+    signs, quats = synthetic.rotation_params(5, H)
+    ctx = cuda_lib.isoquant_init(signs, quats)
+    cache = cuda_lib.PagedCache.allocate(H, 2, 32)
+    cache.codes.fill_(-1)
+    x = synthetic.gaussian(6, 0, (3, H, D), device="cuda")
+    slots = torch.tensor([-1, 5, 64], dtype=torch.int64, device="cuda")  # skip, write, out of range
+    cuda_lib.isoquant_compress_kv(ctx, cache, x, x, slots)
+    torch.cuda.synchronize()
+    st = cuda_lib.isoquant_get_status(ctx)
+    assert st & cuda_lib.DEVERR_SLOT_RANGE
+    written = (cache.codes[0, 0, 0, :, :] != -1).any(dim=0).cpu()
+    assert written.tolist() == [i == 5 for i in range(32)]
+    assert cuda_lib.isoquant_get_status(ctx) == 0  # cleared by the read
+
+
+def test_rotate_q_matches_oracle(cuda_lib):
+    from compressed_space_decode_b200 import synthetic
+    H, Hq = 4, 16
+    signs, quats = synthetic.rotation_params(11, H)
+    ctx = cuda_lib.isoquant_init(signs, quats)
+    q = synthetic.gaussian(12, 0, (5, Hq, D), device="cuda") * 7.0
+    out = torch.empty_like(q)
+    cuda_lib.isoquant_rotate_q(ctx, q, out)
+    torch.cuda.synchronize()
+    qc, oc = q.double().cpu().numpy(), out.double().cpu().numpy()
+    for hq in range(Hq):
+        h = hq // (Hq // H)
+        ref = oracle.rotate(signs[h].numpy(), quats[h].numpy(), qc[:, hq])
+        err = np.abs(oc[:, hq] - ref).max() / np.abs(ref).max()
+        assert err < 2e-6, (hq, err)
+
+
+@pytest.mark.parametrize("ps", [32, 64, 128, 256])
+def test_attend_edge_lengths(cuda_lib, ps):
+    """Empty, single-token, ragged, page-multiple and split-boundary lengths."""
+    from compressed_space_decode_b200.synthetic import Workload
+    from compressed_space_decode_b200.workload import DecodeState
+    lens = [0, 1, 31, 32, 33, ps - 1, ps, ps + 1, 3 * ps + 17, 700]
+    wl = Workload(f"edge_ps{ps}", len(lens), 8, 2, lens, page_size=ps, seed=4242)
+    st = DecodeState(wl)
+    q, _, out = run_attend(cuda_lib, st)
+    for b in range(len(lens)):
+        for h in range(2):
+            if lens[b] == 0:
+                assert torch.all(out[b] == 0)
+                continue
+            check_pair(st, b, h, q, out)
+
+
+def test_attend_mixing_softmax(cuda_lib):
+    """Scale chosen so the score spread is O(1): many tokens share the weight."""
+    from compressed_space_decode_b200.workload import DecodeState
+    wl = cuda_lib.synthetic.workloads(small=True)["gqa_b1_q32_kv8_L4096"]
+    st = DecodeState(wl)
+    # the heavy-tailed keys have norms of a few hundred: a scale of 1e-3
+    # brings the scores to a spread of about 2
+    q, _, out = run_attend(cuda_lib, st, scale=1e-3)
+    for h in range(st.H):
+        check_pair(st, 0, h, q, out, scale=1e-3)
+
+
+def test_append_steps_then_attend(cuda_lib):
+    """Decode steps: append one token per sequence via compress_kv, attend."""
+    from compressed_space_decode_b200.workload import DecodeState
+    wl = cuda_lib.synthetic.workloads(small=True)["gqa_b16_q32_kv4_L32768_paged"]
+    st = DecodeState(wl, growth=40)
+    for step in range(40):
+        k = torch.stack([st.kv_tokens(b, st.seq_lens[b], st.seq_lens[b] + 1)[0][0] for b in range(st.B)])
+        v = torch.stack([st.kv_tokens(b, st.seq_lens[b], st.seq_lens[b] + 1)[1][0] for b in range(st.B)])
+        slots = torch.cat([st.slots(b, st.seq_lens[b], st.seq_lens[b] + 1) for b in range(st.B)])
+        cuda_lib.isoquant_compress_kv(st.ctx, st.cache, k.contiguous(), v.contiguous(), slots)
+        st.seq_lens = [L + 1 for L in st.seq_lens]
+        st.seq_lens_dev += 1
+        q, _, out = run_attend(cuda_lib, st, step=step)
+    for b, h in [(0, 0), (7, 3), (15, 1)]:
+        check_pair(st, b, h, q, out)
+
+
+def test_attend_allocates_nothing(cuda_lib):
+    from compressed_space_decode_b200.workload import DecodeState
+    wl = cuda_lib.synthetic.workloads(small=True)["gqa_b1_q32_kv8_L4096"]
+    st = DecodeState(wl)
+    q = st.queries(0)
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    out = torch.empty_like(q_rot)
+    ws = _ws(cuda_lib, st)
+    torch.cuda.synchronize()
+    before = torch.cuda.memory_allocated()
+    cuda_lib.isoquant_rotate_q(st.ctx, q.reshape(-1, st.Hq, D), q_rot.view(-1, st.Hq, D))
+    cuda_lib.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, ws, out)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == before
+    # the workspace holds partial (m, l, o) records only: far smaller than the
+    # fp16 K/V this cache stands for (no full-precision KV is materialised)
+    assert ws.numel() * 4 < sum(st.seq_lens) * st.H * 2 * D * 2
+
+
+@pytest.mark.parametrize("name,pairs", [
+    ("gqa_b1_q32_kv8_L4096", "all"),
+    ("gqa_b16_q32_kv4_L32768_paged", 2),
+    ("long_b4_q64_kv8_L64k_128k_ragged", 1),
+    ("verify_b8_nq16_q32_kv8_L16384", 2),
+])
+def test_attend_full_size_sampled(cuda_lib, name, pairs):
+    from compressed_space_decode_b200.workload import DecodeState
+    wl = cuda_lib.synthetic.workloads()[name]
+    st = DecodeState(wl)
+    q, _, out = run_attend(cuda_lib, st)
+    assert torch.isfinite(out).all()
+    allp = [(b, h) for b in range(st.B) for h in range(st.H)]
+    rng = np.random.default_rng(1)
+    sel = allp if pairs == "all" else [allp[i] for i in rng.choice(len(allp), pairs, replace=False)]
+    if name.startswith("long"):
+        b_short = int(np.argmin(st.seq_lens))
+        sel = [(b_short, int(rng.integers(st.H)))]
+    for b, h in sel:
+        check_pair(st, b, h, q, out)
