@@ -33,6 +33,7 @@ SYMBOLS = [
     "isoquant_init", "isoquant_destroy", "isoquant_strerror", "isoquant_codebook", "isoquant_cache_bytes",
     "isoquant_compress_kv", "isoquant_rotate_q", "isoquant_workspace_size", "isoquant_attend_decode",
     "isoquant_attend_partial", "isoquant_attend_combine", "isoquant_get_status", "isoquant_last_launch_count",
+    "isoquant_attend_decode_static",
 ]
 
 
@@ -73,6 +74,8 @@ def lib():
             "isoquant_attend_combine": ([vp, i32, i32, i32, vp, i32, vp, sz, vp, vp], i32),
             "isoquant_get_status": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i32),
             "isoquant_last_launch_count": ([vp], i32),
+            "isoquant_attend_decode_static": ([vp, cp, vp, i32, i32, i32, vp, i32, vp, i32, ctypes.c_float, vp, vp],
+                                              i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -221,6 +224,20 @@ def isoquant_attend_decode(ctx, cache, q_rot, page_table, seq_lens, workspace, o
                                         _ptr(seq_lens), int(bool(causal)), float(scale), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
            "isoquant_attend_decode")
+
+
+def isoquant_attend_decode_static(ctx, cache, q_rot, page_table, seq_lens, out, causal=False, scale=0.0,
+                                  stream=None):
+    """isoquant_attend_decode for callers that cannot allocate device memory
+    or lend a workspace: the split records go to a fixed 4 MiB array inside
+    the library.  Its first call on a device must precede any stream
+    capture; calls that overlap on the GPU race on the shared array."""
+    B, nq, Hq, maxp = _attend_args(q_rot, page_table, seq_lens)
+    cs = cache.c_struct()
+    _check(lib().isoquant_attend_decode_static(ctx.handle, ctypes.byref(cs), _ptr(q_rot), B, nq, Hq,
+                                               _ptr(page_table), maxp, _ptr(seq_lens), int(bool(causal)),
+                                               float(scale), _ptr(out), _stream(stream)),
+           "isoquant_attend_decode_static")
 
 
 def isoquant_attend_partial(ctx, cache, q_rot, page_table, seq_lens, workspace, causal=False, scale=0.0,

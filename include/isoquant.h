@@ -156,6 +156,25 @@ int isoquant_attend_decode(isoquant_ctx *ctx, const isoquant_cache *cache,
                            float scale, void *workspace, size_t ws_bytes,
                            float *out, void *stream);
 
+/* isoquant_attend_decode without a workspace argument, for callers that can
+ * neither allocate device memory nor lend the library a buffer (a serving
+ * process whose memory pool owns all device memory, or a decode loop that
+ * must not risk the device-wide synchronisation of cudaMalloc/cudaFree).
+ * The paper has no counterpart to this call; it is a deployment aid.
+ * Same arguments and result as isoquant_attend_decode.  The split records
+ * live in a 4 MiB array compiled into the library (held by every GPU that
+ * loads it until exit); a shape whose isoquant_workspace_size exceeds 4 MiB
+ * is rejected with ISOQUANT_ERR_WORKSPACE.  The first call on a device looks
+ * up the array's device address and must come before any stream capture.
+ * Calls share the array: calls whose kernels overlap on the GPU race and
+ * must be ordered by the caller.  Allocates and frees nothing. */
+int isoquant_attend_decode_static(isoquant_ctx *ctx, const isoquant_cache *cache,
+                                  const float *q_rot, int batch, int nq,
+                                  int num_q_heads, const int32_t *page_table,
+                                  int max_pages, const int32_t *seq_lens,
+                                  int causal, float scale, float *out,
+                                  void *stream);
+
 /* The two halves of isoquant_attend_decode, for callers that schedule them
  * separately (same arguments; the partial half fills the workspace, the
  * combine half reads it and writes `out`). */
