@@ -118,7 +118,7 @@ int make_shape(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, int 
   s->row_groups = (s->rows + 7) / 8;
   s->page_size = page_size;
   s->causal = causal ? 1 : 0;
-  s->n_cta = ctx->num_sms;
+  s->n_cta = ctx->num_sms * attend_ctas_per_sm();
   s->slots = static_cast<size_t>(s->n_cta) +
              static_cast<size_t>(s->row_groups) * static_cast<size_t>(batch) * ctx->num_kv_heads;
   return ISOQUANT_OK;

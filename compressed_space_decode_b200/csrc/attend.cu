@@ -5,21 +5,22 @@
 // softmax-weighted V sum are formed in the rotated space from the codes; the
 // output is rotated back once, in the combine step.
 //
-// Partial kernel (one CTA per SM, persistent, split-K over pages):
+// Partial kernel (two CTAs per SM, persistent, split-K over pages):
 //   * work = pages of (row group, batch, KV head) pairs, laid end to end;
 //     CTA c takes pages [c*P/N, (c+1)*P/N) so that every SM streams the same
 //     number of pages whatever the length mix, and writes one partial
 //     (m, l, o) per pair it touches.
-//   * warp 8 is a producer: per page it issues 28 bulk copies (13 K code
-//     rows, 13 V code rows, 2 norm rows) into a 4-stage shared-memory ring
+//   * warp 4 is a producer: per page it issues 28 bulk copies (13 K code
+//     rows, 13 V code rows, 2 norm rows) into a 3-stage shared-memory ring
 //     with an mbarrier per stage.
-//   * warps 0..7 take 32-token slices of the page.  A GQA group of up to 8
-//     query rows shares every KV tile: Q.K^T is an m16n8k16 tensor-core
+//   * warps 0..3 each take a 64-token unit of the page.  A GQA group of up to
+//     8 query rows shares every KV tile: Q.K^T is an m16n8k16 tensor-core
 //     product with the query split into fp16 high and low parts in the 16
 //     rows (so the score keeps ~22 bits), K codes become fp16 centroids
 //     through a 64-entry pair table held once per lane in shared memory, and
-//     P.V is a second m16n8k16 product with V^T as the A operand.
-//   * at the end of each pair, the 8 warps merge their (m, l, o) in shared
+//     P.V is a second m16n8k16 product with V^T as the A operand.  The eight
+//     4-token tiles of a unit run their mma chains interleaved.
+//   * at the end of each pair, the warps merge their (m, l, o) in shared
 //     memory and one record is written to the workspace.
 // Combine kernel: one warp per output row merges the records of its pair,
 // divides by l and applies R^-1 = D Hn B^T.
@@ -32,9 +33,16 @@
 namespace isoquant {
 namespace {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 4;
+#ifndef ISOQUANT_ATTEND_CTAS_PER_SM
+#define ISOQUANT_ATTEND_CTAS_PER_SM 2
+#endif
+constexpr int kCtasPerSm = ISOQUANT_ATTEND_CTAS_PER_SM;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 4;
+#ifndef ISOQUANT_ATTEND_STAGES
+#define ISOQUANT_ATTEND_STAGES 3
+#endif
+constexpr int kStages = ISOQUANT_ATTEND_STAGES;
 constexpr int kMaxPage = 256;
 // Shared-memory row strides (32-bit words) of the K and V code rows.  K rows
 // are read as word rows {3t, 3t+1, 3t+2} by the four threads of a quad; a
@@ -47,12 +55,15 @@ constexpr int kStageVC = kStageKC + kWords * kStrideK * 4;
 constexpr int kStageKN = kStageVC + kWords * kStrideV * 4;
 constexpr int kStageVN = kStageKN + kMaxPage * 2;
 constexpr int kStageBytes = kStageVN + kMaxPage * 2;
-// merge scratch: o[8 warps][8 rows][128], m[8][8], l[8][8], e[8]
-constexpr int kScratchO = kStages * kStageBytes;
+// Merge scratch (o[warps][8 rows][128], m[warps][8], l[warps][8], e[8]) is
+// placed in the stage buffer being retired when a pair ends, after every
+// consumer warp has finished reading it and before the stage is released.
+constexpr int kScratchO = 0;
 constexpr int kScratchM = kScratchO + kConsumerWarps * 8 * kD * 4;
 constexpr int kScratchL = kScratchM + kConsumerWarps * 8 * 4;
 constexpr int kScratchE = kScratchL + kConsumerWarps * 8 * 4;
-constexpr int kBarriers = kScratchE + 8 * 4;
+static_assert(kScratchE + 8 * 4 <= kStageBytes, "merge scratch must fit in one stage");
+constexpr int kBarriers = kStages * kStageBytes;
 constexpr int kLocate = kBarriers + 2 * kStages * 8;
 constexpr int kSmemBytes = kLocate + 64;
 static_assert(kStageBytes % 16 == 0, "stage alignment");
@@ -133,6 +144,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// 2^x by the SFU (ex2.approx, relative error below 2^-22; 2^-inf = +0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -205,8 +222,8 @@ struct Walk {
 // so that 32 lanes with 32 different indices hit 32 different banks.
 __shared__ __align__(16) uint32_t s_lut[64 * 32];
 
-// Byte offset of entry ((x >> sh) & 63) for this lane: the entry index lands
-// in bits 7..12 and the lane's bank in bits 2..6, so one AND-OR forms it.
+// Byte offset of entry ((x >> (SH + 7)) & 63) for this lane: the entry index
+// lands in bits 7..12 and the lane's bank in bits 2..6, so one AND-OR forms it.
 template <int SH>
 __device__ __forceinline__ uint32_t lut_off(uint32_t x, uint32_t lane4) {
   const uint32_t y = (SH >= 0) ? (x >> (SH >= 0 ? SH : 0)) : (x << (SH < 0 ? -SH : 0));
@@ -228,8 +245,40 @@ __device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
   return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
+// Q.K^T B-fragment register for pair k (0..15) of token j of a 4-token group:
+// pairs 0..14 are adjacent codes (2(k%5), 2(k%5)+1) of words 3tq + k/5;
+// pair 15 is codes (2tq, 2tq+1) of word 12 (shift sh12 = 6tq).
+template <int K>
+__device__ __forceinline__ uint32_t k_pair_c(const uint4 (&kw)[4], int j, uint32_t sh12, uint32_t lane4) {
+  if constexpr (K < 15) {
+    return lut_at(lut_off<6 * (K % 5) - 7>(u4_at(kw[K / 5], j), lane4));
+  } else {
+    return lut_at((((u4_at(kw[3], j) << 7) >> sh12) & 0x1F80u) | lane4);
+  }
+}
+__device__ __forceinline__ uint32_t k_pair(const uint4 (&kw)[4], int j, int k, uint32_t sh12, uint32_t lane4) {
+  switch (k) {
+    case 0: return k_pair_c<0>(kw, j, sh12, lane4);
+    case 1: return k_pair_c<1>(kw, j, sh12, lane4);
+    case 2: return k_pair_c<2>(kw, j, sh12, lane4);
+    case 3: return k_pair_c<3>(kw, j, sh12, lane4);
+    case 4: return k_pair_c<4>(kw, j, sh12, lane4);
+    case 5: return k_pair_c<5>(kw, j, sh12, lane4);
+    case 6: return k_pair_c<6>(kw, j, sh12, lane4);
+    case 7: return k_pair_c<7>(kw, j, sh12, lane4);
+    case 8: return k_pair_c<8>(kw, j, sh12, lane4);
+    case 9: return k_pair_c<9>(kw, j, sh12, lane4);
+    case 10: return k_pair_c<10>(kw, j, sh12, lane4);
+    case 11: return k_pair_c<11>(kw, j, sh12, lane4);
+    case 12: return k_pair_c<12>(kw, j, sh12, lane4);
+    case 13: return k_pair_c<13>(kw, j, sh12, lane4);
+    case 14: return k_pair_c<14>(kw, j, sh12, lane4);
+    default: return k_pair_c<15>(kw, j, sh12, lane4);
+  }
+}
+
 // ------------------------------------------------------------ partial kernel
-__global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialParams p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const PartialParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tq = lane & 3;
@@ -331,10 +380,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialPar
 
   // -------------------------------------------------------------- consumers
   const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
-  float *sm_o = reinterpret_cast<float *>(smem + kScratchO);
-  float *sm_m = reinterpret_cast<float *>(smem + kScratchM);
-  float *sm_l = reinterpret_cast<float *>(smem + kScratchL);
-  float *sm_e = reinterpret_cast<float *>(smem + kScratchE);
 
   // dims this thread feeds to Q.K^T: pair k (k = 0..15) = coordinates
   // (kdim(k), kdim(k) + 1); pairs 0..14 come from words 3tq..3tq+2, pair 15
@@ -357,8 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialPar
   float m_run = -INFINITY, l_run = 0.f, inv2e = 1.f;
   int lim = 0, lim_min = 0, lim_max = 0;
 
-  int64_t it = 0;
-  for (int64_t g = gs; g < ge; ++g, ++it) {
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int64_t g = gs; g < ge; ++g) {
     const bool seg_start = (g == gs) || (wk.j == 0);
     const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
     if (seg_start) {
@@ -411,10 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialPar
       l_run = 0.f;
     }
 
-    const int stage = static_cast<int>(it % kStages);
-    const uint32_t round = static_cast<uint32_t>(it / kStages);
     bool ok = true;
-    if (lane == 0) ok = mbar_wait(&full[stage], round & 1u, p.status, abort_flag);
+    if (lane == 0) ok = mbar_wait(&full[stage], phase, p.status, abort_flag);
     ok = __shfl_sync(0xffffffffu, ok, 0);
     const uint8_t *st = smem + static_cast<size_t>(stage) * kStageBytes;
     const uint32_t *kc = reinterpret_cast<const uint32_t *>(st + kStageKC);
@@ -422,55 +466,77 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialPar
     const __half *kn = reinterpret_cast<const __half *>(st + kStageKN);
     const __half *vn = reinterpret_cast<const __half *>(st + kStageVN);
 
-    for (int sc = warp; ok && sc * 32 < ps; sc += kConsumerWarps) {
-      const int t0 = sc * 32;                       // token offset in the page
+    // each warp takes 64-token units: two 32-token halves whose independent
+    // work interleaves, sharing one softmax reduction
+    for (int sc = warp; ok && sc * 64 < ps; sc += kConsumerWarps) {
+      const int t0 = sc * 64;                       // first token of the unit in the page
       const int tok0 = wk.j * ps + t0;              // absolute position
       if (tok0 >= lim_max) break;
+      // tokens past a row's limit (or past the end of a 32-token page) exist
+      // only in the last unit of a pair
+      const bool tail = (tok0 + 64 > lim_min) || (t0 + 64 > ps);
 
-      // ---- scores: 4 n-tiles, tile j column n = token 4n + j
-      const uint4 kw0 = *reinterpret_cast<const uint4 *>(kc + (3 * tq + 0) * kStrideK + t0 + 4 * gid);
-      const uint4 kw1 = *reinterpret_cast<const uint4 *>(kc + (3 * tq + 1) * kStrideK + t0 + 4 * gid);
-      const uint4 kw2 = *reinterpret_cast<const uint4 *>(kc + (3 * tq + 2) * kStrideK + t0 + 4 * gid);
-      const uint4 kw3 = *reinterpret_cast<const uint4 *>(kc + 12 * kStrideK + t0 + 4 * gid);
-      float x[8];
+      // ---- scores: tile t = 4h + j, column n = token t0 + 32h + 4n + j.  The
+      // k-chunk loop is outermost so that the 8 tiles' mma chains interleave.
+      uint4 kw[2][4];  // words 3tq, 3tq+1, 3tq+2 and 12 of tokens t0 + 32h + 4gid + {0..3}
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t bf[16];
-        word_pairs(u4_at(kw0, j), lane4, bf + 0);
-        word_pairs(u4_at(kw1, j), lane4, bf + 5);
-        word_pairs(u4_at(kw2, j), lane4, bf + 10);
-        bf[15] = lut_at((((u4_at(kw3, j) << 7) >> (6 * tq)) & 0x1F80u) | lane4);
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mma16816(d, qa[c][0], qa[c][1], qa[c][2], qa[c][3], bf[2 * c], bf[2 * c + 1]);
-        x[j] = d[0] + d[2];        // token 8tq + j
-        x[4 + j] = d[1] + d[3];    // token 8tq + 4 + j
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t *kb = kc + t0 + 32 * h + 4 * gid;
+        kw[h][0] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 0) * kStrideK);
+        kw[h][1] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 1) * kStrideK);
+        kw[h][2] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 2) * kStrideK);
+        kw[h][3] = *reinterpret_cast<const uint4 *>(kb + 12 * kStrideK);
       }
-      // ---- norms, masking, online softmax (row gid, tokens 8tq + i)
-      const uint4 knv = *reinterpret_cast<const uint4 *>(kn + t0 + 8 * tq);
-      const uint4 vnv = *reinterpret_cast<const uint4 *>(vn + t0 + 8 * tq);
-      float nk[8], nv[8];
+      const uint32_t sh12 = 6 * tq;
+      float d[8][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&reinterpret_cast<const uint32_t *>(&knv)[i]));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&reinterpret_cast<const uint32_t *>(&vnv)[i]));
-        nk[2 * i] = a.x; nk[2 * i + 1] = a.y;
-        nv[2 * i] = b.x; nv[2 * i + 1] = b.y;
-      }
-      const bool mask = tok0 + 32 > lim_min;
-      float mx = -INFINITY;
+      for (int t = 0; t < 8; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float v = x[i] * nk[i];
-        if (mask && tok0 + 8 * tq + i >= lim) v = -INFINITY;
-        x[i] = v;
-        mx = fmaxf(mx, v);
+      for (int c = 0; c < 8; ++c) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const uint32_t b0 = k_pair(kw[t >> 2], t & 3, 2 * c, sh12, lane4);
+          const uint32_t b1 = k_pair(kw[t >> 2], t & 3, 2 * c + 1, sh12, lane4);
+          mma16816(d[t], qa[c][0], qa[c][1], qa[c][2], qa[c][3], b0, b1);
+        }
       }
+      float x[16];  // x[8h + i] = token t0 + 32h + 8tq + i
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        x[8 * (t >> 2) + (t & 3)] = d[t][0] + d[t][2];      // hi + lo rows
+        x[8 * (t >> 2) + 4 + (t & 3)] = d[t][1] + d[t][3];
+      }
+      // ---- norms, masking, online softmax (row gid)
+      float nv[16];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint4 knv = *reinterpret_cast<const uint4 *>(kn + t0 + 32 * h + 8 * tq);
+        const uint4 vnv = *reinterpret_cast<const uint4 *>(vn + t0 + 32 * h + 8 * tq);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&reinterpret_cast<const uint32_t *>(&knv)[i]));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&reinterpret_cast<const uint32_t *>(&vnv)[i]));
+          x[8 * h + 2 * i] *= a.x;
+          x[8 * h + 2 * i + 1] *= a.y;
+          nv[8 * h + 2 * i] = b.x;
+          nv[8 * h + 2 * i + 1] = b.y;
+        }
+      }
+      if (tail) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int tin = t0 + 32 * (i >> 3) + 8 * tq + (i & 7);
+          if (wk.j * ps + tin >= lim || tin >= ps) x[i] = -INFINITY;
+        }
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int i = 1; i < 16; ++i) mx = fmaxf(mx, x[i]);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float m_new = fmaxf(m_run, mx);
       if (__any_sync(0xffffffffu, m_new > m_run)) {
-        const float corr = (m_run == -INFINITY) ? 0.f : exp2f((m_run - m_new) * inv2e);
+        const float corr = (m_run == -INFINITY) ? 0.f : ex2((m_run - m_new) * inv2e);
         l_run *= corr;
         const float c0 = __shfl_sync(0xffffffffu, corr, (2 * tq) * 4);
         const float c1 = __shfl_sync(0xffffffffu, corr, (2 * tq + 1) * 4);
@@ -481,56 +547,76 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialPar
         m_run = m_new;
       }
       const float mm = (m_run == -INFINITY) ? 0.f : m_run * inv2e;
-      float pv[8];
+      float pv[16], psum[2] = {0.f, 0.f};
+      if (!tail) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float pr = exp2f(fmaf(x[i], inv2e, -mm));
-        l_run += pr;
-        pv[i] = pr > 0.f ? pr * nv[i] : 0.f;
+        for (int i = 0; i < 16; ++i) {
+          const float pr = ex2(fmaf(x[i], inv2e, -mm));
+          psum[i & 1] += pr;
+          pv[i] = pr * nv[i];
+        }
+      } else {
+        // masked slots may hold stale norms: select, do not multiply
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float pr = ex2(fmaf(x[i], inv2e, -mm));
+          psum[i & 1] += pr;
+          pv[i] = pr > 0.f ? pr * nv[i] : 0.f;
+        }
       }
+      l_run += psum[0] + psum[1];
+
       // ---- P.V: O^T[16 dims x 8 rows] += V^T[16 dims x 16 tok] P^T
-      const uint4 va0 = *reinterpret_cast<const uint4 *>(vc + gid * kStrideV + t0 + 8 * tq);
-      const uint4 va1 = *reinterpret_cast<const uint4 *>(vc + gid * kStrideV + t0 + 8 * tq + 4);
-      const uint4 vb0 = *reinterpret_cast<const uint4 *>(vc + (8 + (gid >> 1)) * kStrideV + t0 + 8 * tq);
-      const uint4 vb1 = *reinterpret_cast<const uint4 *>(vc + (8 + (gid >> 1)) * kStrideV + t0 + 8 * tq + 4);
-      const uint4 vz0 = *reinterpret_cast<const uint4 *>(vc + 12 * kStrideV + t0 + 8 * tq);
-      const uint4 vz1 = *reinterpret_cast<const uint4 *>(vc + 12 * kStrideV + t0 + 8 * tq + 4);
       constexpr uint32_t M = 0x071C71C7u;  // even-indexed 3-bit fields
 #pragma unroll
-      for (int kap = 0; kap < 2; ++kap) {
-        uint32_t va[2][16];
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t *vb = vc + t0 + 32 * h + 8 * tq;
+        const uint4 va0 = *reinterpret_cast<const uint4 *>(vb + gid * kStrideV);
+        const uint4 va1 = *reinterpret_cast<const uint4 *>(vb + gid * kStrideV + 4);
+        const uint4 vb0 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * kStrideV);
+        const uint4 vb1 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * kStrideV + 4);
+        const uint4 vz0 = *reinterpret_cast<const uint4 *>(vb + 12 * kStrideV);
+        const uint4 vz1 = *reinterpret_cast<const uint4 *>(vb + 12 * kStrideV + 4);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int tp = 2 * kap + half;  // token pair (2tp, 2tp+1) of this thread's 8
-          const uint4 &A = tp < 2 ? va0 : va1;
-          const uint4 &Bv = tp < 2 ? vb0 : vb1;
-          const uint4 &Z = tp < 2 ? vz0 : vz1;
-          const int e0 = (tp & 1) * 2;
-          const uint32_t wa = u4_at(A, e0), wa1 = u4_at(A, e0 + 1);
-          const uint32_t wb = u4_at(Bv, e0), wb1 = u4_at(Bv, e0 + 1);
-          const uint32_t wz = u4_at(Z, e0), wz1 = u4_at(Z, e0 + 1);
-          // merge two tokens' words: 6-bit slot k = (code of tok a, code of tok b)
-          const uint32_t e_even = (wa & M) | ((wa1 << 3) & ~M);
-          const uint32_t e_odd = ((wa >> 3) & M) | (wa1 & ~M);
-          const uint32_t e_half = ((wb >> (3 * par)) & M) | ((wb1 << (3 - 3 * par)) & ~M);
-          word_pairs(e_even, lane4, va[half] + 0);
-          word_pairs(e_odd, lane4, va[half] + 5);
-          word_pairs(e_half, lane4, va[half] + 10);
-          const uint32_t z12 = (((wz >> (3 * gid)) & 7u) << 7) | (((wz1 >> (3 * gid)) & 7u) << 10);
-          va[half][15] = lut_at(z12 | lane4);
+        for (int kap = 0; kap < 2; ++kap) {
+          uint32_t va[2][16];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int tp = 2 * kap + half;  // token pair (2tp, 2tp+1) of this thread's 8
+            const uint4 &A = tp < 2 ? va0 : va1;
+            const uint4 &Bv = tp < 2 ? vb0 : vb1;
+            const uint4 &Z = tp < 2 ? vz0 : vz1;
+            const int e0 = (tp & 1) * 2;
+            const uint32_t wa = u4_at(A, e0), wa1 = u4_at(A, e0 + 1);
+            const uint32_t wb = u4_at(Bv, e0), wb1 = u4_at(Bv, e0 + 1);
+            const uint32_t wz = u4_at(Z, e0), wz1 = u4_at(Z, e0 + 1);
+            // merge two tokens' words: 6-bit slot k = (code of tok a, code of tok b)
+            const uint32_t e_even = (wa & M) | ((wa1 << 3) & ~M);
+            const uint32_t e_odd = ((wa >> 3) & M) | (wa1 & ~M);
+            const uint32_t e_half = ((wb >> (3 * par)) & M) | ((wb1 << (3 - 3 * par)) & ~M);
+            word_pairs(e_even, lane4, va[half] + 0);
+            word_pairs(e_odd, lane4, va[half] + 5);
+            word_pairs(e_half, lane4, va[half] + 10);
+            const uint32_t z12 = (((wz >> (3 * gid)) & 7u) << 7) | (((wz1 >> (3 * gid)) & 7u) << 10);
+            va[half][15] = lut_at(z12 | lane4);
+          }
+          const uint32_t b0 = pack_half2(pv[8 * h + 4 * kap + 0], pv[8 * h + 4 * kap + 1]);
+          const uint32_t b1 = pack_half2(pv[8 * h + 4 * kap + 2], pv[8 * h + 4 * kap + 3]);
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            mma16816(acc[m], va[0][2 * m], va[0][2 * m + 1], va[1][2 * m], va[1][2 * m + 1], b0, b1);
         }
-        const uint32_t b0 = pack_half2(pv[4 * kap + 0], pv[4 * kap + 1]);
-        const uint32_t b1 = pack_half2(pv[4 * kap + 2], pv[4 * kap + 3]);
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-          mma16816(acc[m], va[0][2 * m], va[0][2 * m + 1], va[1][2 * m], va[1][2 * m + 1], b0, b1);
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
-
     if (seg_end) {
-      // ---- merge the 8 warps' states and write one record
+      // ---- merge the consumer warps' states and write one record
+      // every warp is done reading this stage: reuse it as merge scratch
+      named_bar_sync(1, kConsumerWarps * 32);
+      uint8_t *scr = smem + static_cast<size_t>(stage) * kStageBytes;
+      float *sm_o = reinterpret_cast<float *>(scr + kScratchO);
+      float *sm_m = reinterpret_cast<float *>(scr + kScratchM);
+      float *sm_l = reinterpret_cast<float *>(scr + kScratchL);
+      float *sm_e = reinterpret_cast<float *>(scr + kScratchE);
       float l_tot = l_run;
       l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
       l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
@@ -548,50 +634,70 @@ __global__ void __launch_bounds__(kThreads, 1) k_attend_partial(const PartialPar
         if (warp == 0) sm_e[gid] = inv2e;
       }
       named_bar_sync(1, kConsumerWarps * 32);
-      const int row = tid >> 5, d0 = (tid & 31) * 4;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * 8 + row]);
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      float l = 0.f;
-      if (M != -INFINITY) {
-        const float e = sm_e[row];
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float s = exp2f((sm_m[w * 8 + row] - M) * e);
-          l += s * sm_l[w * 8 + row];
-          const float4 ow = *reinterpret_cast<const float4 *>(sm_o + (w * 8 + row) * kD + d0);
-          o.x += s * ow.x; o.y += s * ow.y; o.z += s * ow.z; o.w += s * ow.w;
-        }
-        M *= e;  // to log2 units
-      }
       const int64_t pair = (static_cast<int64_t>(wk.rg) * p.B + wk.b) * p.H + wk.h;
       float *rec = p.records + (blockIdx.x + pair) * static_cast<int64_t>(kRecordFloats);
-      if ((tid & 31) == 0) {
-        rec[2 * row] = M;
-        rec[2 * row + 1] = l;
+      for (int e = tid; e < 8 * 32; e += kConsumerWarps * 32) {
+        const int row = e >> 5, d0 = (e & 31) * 4;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * 8 + row]);
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        float l = 0.f;
+        if (M != -INFINITY) {
+          const float e2 = sm_e[row];
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float s = ex2((sm_m[w * 8 + row] - M) * e2);
+            l += s * sm_l[w * 8 + row];
+            const float4 ow = *reinterpret_cast<const float4 *>(sm_o + (w * 8 + row) * kD + d0);
+            o.x += s * ow.x; o.y += s * ow.y; o.z += s * ow.z; o.w += s * ow.w;
+          }
+          M *= e2;  // to log2 units
+        }
+        if ((e & 31) == 0) {
+          rec[2 * row] = M;
+          rec[2 * row + 1] = l;
+        }
+        *reinterpret_cast<float4 *>(rec + 16 + row * kD + d0) = o;
       }
-      *reinterpret_cast<float4 *>(rec + 16 + row * kD + d0) = o;
+      // the bulk copies that refill this stage must not overtake the
+      // scratch accesses above
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       named_bar_sync(1, kConsumerWarps * 32);
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+
     if (g + 1 < ge) wk.advance(p.seq_lens, p.B, p.H, ps);
   }
 }
 
 // ------------------------------------------------------------ combine kernel
+// CTA that owns global page g when P pages are split as [c P / N, (c+1) P / N)
+__device__ __forceinline__ int64_t cta_of_page(int64_t g, int64_t N, int64_t P) {
+  return ((g + 1) * N + P - 1) / P - 1;
+}
+__device__ __forceinline__ bool cta_empty(int64_t c, int64_t N, int64_t P) {
+  return c * P / N == (c + 1) * P / N;
+}
+
 __global__ void __launch_bounds__(256) k_attend_combine(const CombineParams p) {
   const int lane = threadIdx.x & 31;
-  const int64_t row_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_rows = static_cast<int64_t>(p.B) * p.nq * p.Hq;
+  const uint32_t row_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t n_rows = static_cast<uint32_t>(p.B) * p.nq * p.Hq;
   if (row_id >= n_rows) return;
-  const int hq = static_cast<int>(row_id % p.Hq);
-  const int64_t bi = row_id / p.Hq;
-  const int i = static_cast<int>(bi % p.nq);
-  const int b = static_cast<int>(bi / p.nq);
+  const int hq = static_cast<int>(row_id % static_cast<uint32_t>(p.Hq));
+  const uint32_t bi = row_id / static_cast<uint32_t>(p.Hq);
+  const int i = static_cast<int>(bi % static_cast<uint32_t>(p.nq));
+  const int b = static_cast<int>(bi / static_cast<uint32_t>(p.nq));
   const int h = hq / p.G, g = hq % p.G;
   const int r = i * p.G + g, rg = r >> 3, rr = r & 7;
   const int ps = p.page_size;
-  float *dst = p.out + row_id * kD + 4 * lane;
+  float *dst = p.out + static_cast<int64_t>(row_id) * kD + 4 * lane;
 
   const int np = pages_of(p.seq_lens[b], ps);
   const int64_t p_rg = static_cast<int64_t>(p.H) * pages_before(p.seq_lens, p.B, ps, lane);
@@ -603,27 +709,41 @@ __global__ void __launch_bounds__(256) k_attend_combine(const CombineParams p) {
   const int64_t g0 = rg * p_rg + static_cast<int64_t>(p.H) * pages_before(p.seq_lens, b, ps, lane) +
                      static_cast<int64_t>(h) * np;
   const int64_t N = p.n_cta;
-  auto cta_of = [&](int64_t gg) -> int64_t { return ((gg + 1) * N + total - 1) / total - 1; };
-  const int64_t c_lo = cta_of(g0), c_hi = cta_of(g0 + np - 1);
+  const int64_t c_lo = cta_of_page(g0, N, total), c_hi = cta_of_page(g0 + np - 1, N, total);
   const int64_t pair = (static_cast<int64_t>(rg) * p.B + b) * p.H + h;
 
   // CTAs with an empty page range (possible when there are fewer pages than
-  // CTAs) wrote no record: skip them
-  auto empty_cta = [&](int64_t c) -> bool { return c * total / N == (c + 1) * total / N; };
+  // CTAs) wrote no record: skip them.  Lane i reads the (m, l) of record
+  // c_lo + i, so the records' maxima and weights come from one round trip.
   float M = -INFINITY;
-  for (int64_t c = c_lo; c <= c_hi; ++c)
-    if (!empty_cta(c)) M = fmaxf(M, p.records[(c + pair) * kRecordFloats + 2 * rr]);
+  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
+    const int64_t c = c0 + lane;
+    if (c <= c_hi && !cta_empty(c, N, total)) M = fmaxf(M, p.records[(c + pair) * kRecordFloats + 2 * rr]);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float o[4] = {0.f, 0.f, 0.f, 0.f};
   float l = 0.f;
   if (M != -INFINITY) {
-    for (int64_t c = c_lo; c <= c_hi; ++c) {
-      if (empty_cta(c)) continue;
-      const float *rec = p.records + (c + pair) * kRecordFloats;
-      const float s = exp2f(rec[2 * rr] - M);
-      l += s * rec[2 * rr + 1];
-      const float4 v = *reinterpret_cast<const float4 *>(rec + 16 + rr * kD + 4 * lane);
-      o[0] += s * v.x; o[1] += s * v.y; o[2] += s * v.z; o[3] += s * v.w;
+    for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
+      const int64_t c = c0 + lane;
+      float s_mine = 0.f;
+      if (c <= c_hi && !cta_empty(c, N, total)) {
+        const float *rec = p.records + (c + pair) * kRecordFloats;
+        s_mine = ex2(rec[2 * rr] - M);
+        l += s_mine * rec[2 * rr + 1];
+      }
+      const int n = static_cast<int>(c_hi - c0 + 1 < 32 ? c_hi - c0 + 1 : 32);
+      for (int i = 0; i < n; ++i) {
+        const float s = __shfl_sync(0xffffffffu, s_mine, i);
+        if (s == 0.f) continue;  // empty CTA, or a record with nothing visible
+        const float4 v =
+            *reinterpret_cast<const float4 *>(p.records + (c0 + i + pair) * kRecordFloats + 16 + rr * kD + 4 * lane);
+        o[0] += s * v.x; o[1] += s * v.y; o[2] += s * v.z; o[3] += s * v.w;
+      }
     }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
   }
   if (M == -INFINITY || !(l > 0.f)) {
     *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -647,6 +767,8 @@ __global__ void __launch_bounds__(256) k_attend_combine(const CombineParams p) {
 
 }  // namespace
 
+int attend_ctas_per_sm() { return kCtasPerSm; }
+
 size_t attend_workspace_bytes(const AttendShape &s) {
   return kWsHeader + s.slots * kRecordFloats * sizeof(float);
 }
@@ -657,6 +779,9 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
   static int configured_device = -1;
   if (configured_device != ctx->device) {
     cudaError_t e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured_device = ctx->device;
   }

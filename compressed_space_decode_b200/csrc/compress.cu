@@ -2,10 +2,10 @@
 //
 // RotaryQuant, Abstract: a Walsh-Hadamard transform followed by
 // block-diagonal SO(4) rotations isotropizes each head vector before 3-bit
-// scalar quantization.  One warp handles one d = 128 vector, lane l holding
-// coordinates 4l..4l+3: the two smallest WHT strides stay inside the lane,
-// the other five are warp shuffles, and SO(4) block l is lane l's own 4x4
-// product, so the whole rotation stays in registers.
+// scalar quantization.  A warp rotates one d = 128 vector at a time, lane l
+// holding coordinates 4l..4l+3: the two smallest WHT strides stay inside the
+// lane, the other five are warp shuffles, and SO(4) block l is lane l's own
+// 4x4 product, so the whole rotation stays in registers.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -70,88 +70,148 @@ __device__ __forceinline__ void rotate_f64(const HeadParams &hp, int lane, const
     out[r] = fma(m[4 * r + 3], y[3], fma(m[4 * r + 2], y[2], fma(m[4 * r + 1], y[1], m[4 * r] * y[0])));
 }
 
+// One warp handles kVecPerWarp consecutive tokens of one (head, K/V): the
+// head's block matrices and sign bits are loaded once into registers and the
+// tokens' inputs are all requested before the first is rotated.
+constexpr int kVecPerWarp = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_compress(const HeadParams *__restrict__ params, Codebook cb,
                                                   const T *__restrict__ kin, const T *__restrict__ vin,
                                                   int n_tok, int H, const int64_t *__restrict__ slots,
                                                   uint32_t *__restrict__ codes,
                                                   uint16_t *__restrict__ norms, int num_pages,
-                                                  int page_size, uint32_t *status) {
+                                                  int ps_shift, uint32_t *status) {
   const int lane = threadIdx.x & 31;
-  const int64_t vec = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t per_kv = static_cast<int64_t>(n_tok) * H;
-  if (vec >= 2 * per_kv) return;
-  const int kv = static_cast<int>(vec / per_kv);
-  const int64_t rem = vec - kv * per_kv;
-  const int64_t t = rem / H;
-  const int h = static_cast<int>(rem - t * H);
-  const int64_t slot = slots[t];
-  if (slot < 0) return;
-  const int64_t page = slot / page_size;
-  const int off = static_cast<int>(slot - page * page_size);
-  if (page >= num_pages) {
-    if (lane == 0) set_status(status, ISOQUANT_DEVERR_SLOT_RANGE);
-    return;
-  }
+  const int kv = blockIdx.y;
+  const uint32_t w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const uint32_t groups = (static_cast<uint32_t>(n_tok) + kVecPerWarp - 1) / kVecPerWarp;
+  const uint32_t tg = w / static_cast<uint32_t>(H);
+  if (tg >= groups) return;
+  const int h = static_cast<int>(w - tg * static_cast<uint32_t>(H));
+  const int page_size = 1 << ps_shift;
   const HeadParams &hp = params[h];
+  const T *src = kv ? vin : kin;
 
-  float x[4];
-  load4((kv ? vin : kin) + (t * H + h) * kD + 4 * lane, x);
-
-  // ||x||_2 in fp64: squares of fp32 values are exact in fp64
-  double ss = static_cast<double>(x[0]) * x[0] + static_cast<double>(x[1]) * x[1] +
-              static_cast<double>(x[2]) * x[2] + static_cast<double>(x[3]) * x[3];
+  // this warp's tokens: inputs first, so their loads overlap
+  float x[kVecPerWarp][4];
+  int64_t slot[kVecPerWarp];
 #pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-  const double n = sqrt(ss);
-
-  // z = (B H D x) / n; sqrt(128) of the normalised Hn cancels against the
-  // sqrt(128) of z = sqrt(128) * y / n.
-  float yr[4];
-  rotate_f32(hp, lane, x, yr);
-  const float inv = n > 0.0 ? static_cast<float>(1.0 / n) : 0.0f;
-  uint32_t c[4];
-  bool near = false;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float z = yr[i] * inv;
-    uint32_t code = 0;
-#pragma unroll
-    for (int k = 0; k < kLevels - 1; ++k) {
-      code += (z > cb.threshold[k]) ? 1u : 0u;
-      near |= fabsf(z - cb.threshold[k]) < kRecheckBand;
-    }
-    c[i] = code;
-  }
-  if (__any_sync(0xffffffffu, near && n > 0.0)) {
-    double y64[4];
-    rotate_f64(hp, lane, x, y64);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const double z = n > 0.0 ? y64[i] / n : 0.0;
-      uint32_t code = 0;
-#pragma unroll
-      for (int k = 0; k < kLevels - 1; ++k) code += (z > cb.threshold64[k]) ? 1u : 0u;
-      c[i] = code;
+  for (int i = 0; i < kVecPerWarp; ++i) {
+    const int t = static_cast<int>(tg) * kVecPerWarp + i;
+    slot[i] = -1;
+    if (t < n_tok) {
+      slot[i] = slots[t];
+      load4(src + (static_cast<int64_t>(t) * H + h) * kD + 4 * lane, x[i]);
     }
   }
+  const uint32_t sn = lane_sign_nibble(hp, lane);
+  float mrow[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float4 row = reinterpret_cast<const float4 *>(hp.m32[lane])[r];
+    mrow[r][0] = row.x; mrow[r][1] = row.y; mrow[r][2] = row.z; mrow[r][3] = row.w;
+  }
+  const float t4 = cb.threshold[4], t5 = cb.threshold[5], t6 = cb.threshold[6];
 
-  // pack: word w holds codes 10w..10w+9, i.e. coordinates of lanes
-  // floor(10w/4) .. +2; an odd word starts two codes into its first lane.
-  const uint32_t c4 = c[0] | (c[1] << 3) | (c[2] << 6) | (c[3] << 9);
-  const int w = lane;
-  const int a = (5 * w) >> 1;
-  const uint32_t s0 = __shfl_sync(0xffffffffu, c4, a & 31);
-  const uint32_t s1 = __shfl_sync(0xffffffffu, c4, min(a + 1, 31));
-  const uint32_t s2 = __shfl_sync(0xffffffffu, c4, min(a + 2, 31));
-  const uint64_t comb = static_cast<uint64_t>(s0) | (static_cast<uint64_t>(s1) << 12) |
-                        (static_cast<uint64_t>(s2) << 24);
-  const uint32_t word =
-      static_cast<uint32_t>(comb >> ((w & 1) ? 6 : 0)) & (w == 12 ? 0x00FFFFFFu : 0x3FFFFFFFu);
+#pragma unroll
+  for (int i = 0; i < kVecPerWarp; ++i) {
+    if (slot[i] < 0) continue;  // past the end, or a skipped token (uniform)
+    const int64_t page = slot[i] >> ps_shift;
+    const int off = static_cast<int>(slot[i] & (page_size - 1));
+    if (page >= num_pages) {
+      if (lane == 0) set_status(status, ISOQUANT_DEVERR_SLOT_RANGE);
+      continue;
+    }
+    const float(&xv)[4] = x[i];
+    // ||x||^2 in fp32 (squares of bf16/fp16 inputs are exact; the tree sum is
+    // within 7 * 2^-24 relative).  The fp64 norm is only formed for the few
+    // vectors whose fp16 rounding the fp32 value cannot decide (below).
+    float ssf = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) ssf += __shfl_xor_sync(0xffffffffu, ssf, m);
+    const float n32 = sqrtf(ssf);
+    // fp16 norm, round to nearest even: decided in fp32 unless n lies within
+    // 1e-6 (relative) of a rounding midpoint, or is huge, tiny or not finite
+    const __half h32 = __float2half_rn(fminf(n32, 65504.f));
+    const float hv = __half2float(h32);
+    const uint16_t hb = __half_as_ushort(h32);
+    const float up = __half2float(__ushort_as_half(static_cast<uint16_t>(hb + 1)));
+    const float dn = hb > 0 ? __half2float(__ushort_as_half(static_cast<uint16_t>(hb - 1))) : 0.f;
+    const float mid = n32 >= hv ? 0.5f * (hv + up) : 0.5f * (hv + dn);
+    const bool exact_f32 = ssf > 1e-30f && n32 < 65000.f && fabsf(n32 - mid) > 1e-6f * n32;
+    uint16_t n16 = hb;
+    float inv;
+    if (__all_sync(0xffffffffu, exact_f32)) {
+      // 1/n: hardware reciprocal square root plus one Newton step (~1e-7)
+      const float r = rsqrtf(ssf);
+      inv = r * (1.5f - 0.5f * ssf * r * r);
+    } else {
+      double ss = static_cast<double>(xv[0]) * xv[0] + static_cast<double>(xv[1]) * xv[1] +
+                  static_cast<double>(xv[2]) * xv[2] + static_cast<double>(xv[3]) * xv[3];
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      const double n = sqrt(ss);
+      n16 = __half_as_ushort(__double2half(fmin(n, 65504.0)));
+      inv = n > 0.0 ? static_cast<float>(1.0 / n) : 0.0f;
+    }
 
-  const int64_t block = (page * 2 + kv) * H + h;
-  if (lane < kWords) codes[block * kWords * page_size + static_cast<int64_t>(w) * page_size + off] = word;
-  if (lane == 0) norms[block * page_size + off] = __half_as_ushort(__double2half(fmin(n, 65504.0)));
+    // z = (B H D x) / n; sqrt(128) of the normalised Hn cancels against the
+    // sqrt(128) of z = sqrt(128) * y / n.
+    float y[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) y[k] = __uint_as_float(__float_as_uint(xv[k]) ^ (((sn >> k) & 1u) << 31));
+    wht128<float>(y, lane);
+    // The codebook is symmetric (t_{6-k} = -t_k, t_3 = 0), so code_j =
+    // #{k : z > t_k} reads off |z| and the three positive thresholds:
+    // z > 0 -> 4 + #{|z| > t}, otherwise 3 - #{|z| >= t}.
+    uint32_t c[4];
+    bool near = false;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float yr = fmaf(mrow[r][3], y[3], fmaf(mrow[r][2], y[2], fmaf(mrow[r][1], y[1], mrow[r][0] * y[0])));
+      const float z = yr * inv;
+      const float a = fabsf(z);
+      const uint32_t gt = (a > t4 ? 1u : 0u) + (a > t5 ? 1u : 0u) + (a > t6 ? 1u : 0u);
+      const uint32_t ge = (a >= t4 ? 1u : 0u) + (a >= t5 ? 1u : 0u) + (a >= t6 ? 1u : 0u);
+      c[r] = z > 0.f ? 4u + gt : 3u - ge;
+      near |= (a < kRecheckBand) | (fabsf(a - t4) < kRecheckBand) | (fabsf(a - t5) < kRecheckBand) |
+              (fabsf(a - t6) < kRecheckBand);
+    }
+    if (__any_sync(0xffffffffu, near && ssf > 0.f)) {
+      double ss = static_cast<double>(xv[0]) * xv[0] + static_cast<double>(xv[1]) * xv[1] +
+                  static_cast<double>(xv[2]) * xv[2] + static_cast<double>(xv[3]) * xv[3];
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      const double n64 = sqrt(ss);
+      double y64[4];
+      rotate_f64(hp, lane, xv, y64);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const double z = n64 > 0.0 ? y64[k] / n64 : 0.0;
+        uint32_t code = 0;
+#pragma unroll
+        for (int q = 0; q < kLevels - 1; ++q) code += (z > cb.threshold64[q]) ? 1u : 0u;
+        c[k] = code;
+      }
+    }
+
+    // pack: word w holds codes 10w..10w+9, i.e. coordinates of lanes
+    // floor(10w/4) .. +2; an odd word starts two codes into its first lane.
+    const uint32_t c4 = c[0] | (c[1] << 3) | (c[2] << 6) | (c[3] << 9);
+    const int wd = lane;
+    const int a = (5 * wd) >> 1;
+    const uint32_t s0 = __shfl_sync(0xffffffffu, c4, a & 31);
+    const uint32_t s1 = __shfl_sync(0xffffffffu, c4, min(a + 1, 31));
+    const uint32_t s2 = __shfl_sync(0xffffffffu, c4, min(a + 2, 31));
+    const uint64_t comb = static_cast<uint64_t>(s0) | (static_cast<uint64_t>(s1) << 12) |
+                          (static_cast<uint64_t>(s2) << 24);
+    const uint32_t word =
+        static_cast<uint32_t>(comb >> ((wd & 1) ? 6 : 0)) & (wd == 12 ? 0x00FFFFFFu : 0x3FFFFFFFu);
+    const int64_t block = (page * 2 + kv) * H + h;
+    if (lane < kWords) codes[((block * kWords + wd) << ps_shift) + off] = word;
+    if (lane == 0) norms[(block << ps_shift) + off] = n16;
+  }
 }
 
 template <typename T>
@@ -159,14 +219,14 @@ __global__ void __launch_bounds__(256) k_rotate_q(const HeadParams *__restrict__
                                                   const T *__restrict__ q, int n_rows, int Hq, int G,
                                                   float *__restrict__ out) {
   const int lane = threadIdx.x & 31;
-  const int64_t vec = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (vec >= static_cast<int64_t>(n_rows) * Hq) return;
-  const int hq = static_cast<int>(vec % Hq);
+  const uint32_t vec = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (vec >= static_cast<uint32_t>(n_rows) * static_cast<uint32_t>(Hq)) return;
+  const int hq = static_cast<int>(vec % static_cast<uint32_t>(Hq));
   float x[4], y[4];
-  load4(q + vec * kD + 4 * lane, x);
+  load4(q + static_cast<int64_t>(vec) * kD + 4 * lane, x);
   rotate_f32(params[hq / G], lane, x, y);
   const float s = 0.08838834764831845f;  // 1/sqrt(128): the normalisation of Hn
-  *reinterpret_cast<float4 *>(out + vec * kD + 4 * lane) = make_float4(y[0] * s, y[1] * s, y[2] * s, y[3] * s);
+  *reinterpret_cast<float4 *>(out + static_cast<int64_t>(vec) * kD + 4 * lane) = make_float4(y[0] * s, y[1] * s, y[2] * s, y[3] * s);
 }
 
 }  // namespace
@@ -175,28 +235,31 @@ cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache
                             const void *v, int dtype, int n_tok, const int64_t *slot_mapping,
                             cudaStream_t stream) {
   const int H = ctx->num_kv_heads;
-  const int64_t warps = 2LL * n_tok * H;
-  const int64_t blocks = (warps * 32 + 255) / 256;
+  const int64_t warps = static_cast<int64_t>((n_tok + kVecPerWarp - 1) / kVecPerWarp) * H;
+  const int64_t blocks = (warps + 7) / 8;
   if (blocks == 0) return cudaSuccess;
-  dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  int ps_shift = 0;
+  while ((1 << ps_shift) < cache->page_size) ++ps_shift;
+  dim3 grid(static_cast<unsigned>(blocks), 2), block(256);
   switch (dtype) {
     case ISOQUANT_F32:
       k_compress<float><<<grid, block, 0, stream>>>(ctx->params, ctx->codebook, static_cast<const float *>(k),
                                                     static_cast<const float *>(v), n_tok, H, slot_mapping,
-                                                    cache->codes, cache->norms, cache->num_pages,
-                                                    cache->page_size, ctx->status);
+                                                    cache->codes, cache->norms, cache->num_pages, ps_shift,
+                                                    ctx->status);
       break;
     case ISOQUANT_BF16:
       k_compress<__nv_bfloat16><<<grid, block, 0, stream>>>(
           ctx->params, ctx->codebook, static_cast<const __nv_bfloat16 *>(k),
           static_cast<const __nv_bfloat16 *>(v), n_tok, H, slot_mapping, cache->codes, cache->norms,
-          cache->num_pages, cache->page_size, ctx->status);
+          cache->num_pages, ps_shift, ctx->status);
       break;
     default:
       k_compress<__half><<<grid, block, 0, stream>>>(ctx->params, ctx->codebook, static_cast<const __half *>(k),
                                                      static_cast<const __half *>(v), n_tok, H, slot_mapping,
-                                                     cache->codes, cache->norms, cache->num_pages,
-                                                     cache->page_size, ctx->status);
+                                                     cache->codes, cache->norms, cache->num_pages, ps_shift,
+                                                     ctx->status);
       break;
   }
   return cudaGetLastError();

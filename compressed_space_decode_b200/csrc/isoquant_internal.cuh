@@ -67,6 +67,7 @@ constexpr size_t kWsHeader = 256;
 constexpr size_t kRecordFloats = 8 * 2 + 8 * kD;  // (m,l) x 8 rows, o[8][128]
 
 size_t attend_workspace_bytes(const AttendShape &s);
+int attend_ctas_per_sm();
 cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache,
                                   const AttendShape &s, const float *q_rot, const int32_t *page_table,
                                   int max_pages, const int32_t *seq_lens, float scale, void *ws,
@@ -94,11 +95,12 @@ __device__ __forceinline__ void wht128(T (&v)[4], int lane) {
   v[0] = a0 + a2; v[1] = a1 + a3; v[2] = a0 - a2; v[3] = a1 - a3;
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) {
-    const bool upper = (lane & m) != 0;
+    // lower lane: v + p; upper lane: p - v; one fused op either way
+    const T sgn = (lane & m) ? T(-1) : T(1);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      T p = __shfl_xor_sync(0xffffffffu, v[i], m);
-      v[i] = upper ? (p - v[i]) : (v[i] + p);
+      const T p = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = fma(sgn, v[i], p);
     }
   }
 }
