@@ -54,9 +54,11 @@ def source_hash(*names):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_src):
+def profiled_traffic(kernel_src, bytes_per_launch):
     """Per-launch DRAM bytes of the attention kernel from the committed ncu
-    summary, or None when the kernel source changed since it was taken."""
+    summary, scaled from the captured launch to this one by the algorithmic
+    bytes (traffic grows in proportion to the pages streamed), or None when
+    the kernel source changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "attend_partial_traffic.json")
     try:
         with open(path) as f:
@@ -65,7 +67,7 @@ def profiled_traffic(kernel_src):
         return None
     if d.get("source_hash") != source_hash(*kernel_src):
         return None
-    return d.get("traffic_bytes_per_launch")
+    return d["traffic_bytes_per_launch"] * bytes_per_launch / d["algorithmic_bytes_per_launch"]
 
 
 class ClockSampler:
@@ -214,7 +216,7 @@ def run_ours(args):
     achieved = bytes_per_launch / (attn_avg_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
     traffic = profiled_traffic(["compressed_space_decode_b200/csrc/attend.cu",
-                                "compressed_space_decode_b200/csrc/isoquant_internal.cuh"])
+                                "compressed_space_decode_b200/csrc/isoquant_internal.cuh"], bytes_per_launch)
 
     # end to end through the public API from pinned host buffers
     attn_events = None
