@@ -48,8 +48,13 @@ constexpr int kMaxPage = 256;
 // are read as word rows {3t, 3t+1, 3t+2} by the four threads of a quad; a
 // stride = 24 (mod 32) puts those rows in distinct 16-byte bank groups.  V
 // rows are read as rows {2p, 2p+1}; a stride = 4 (mod 32) interleaves them.
+#ifdef ISOQUANT_DENSE_STAGE
+constexpr int kStrideK = kMaxPage;  // smem row stride = page_size at run time
+constexpr int kStrideV = kMaxPage;
+#else
 constexpr int kStrideK = kMaxPage + 24;
 constexpr int kStrideV = kMaxPage + 4;
+#endif
 constexpr int kStageKC = 0;
 constexpr int kStageVC = kStageKC + kWords * kStrideK * 4;
 constexpr int kStageKN = kStageVC + kWords * kStrideV * 4;
@@ -63,7 +68,12 @@ constexpr int kScratchM = kScratchO + kConsumerWarps * 8 * kD * 4;
 constexpr int kScratchL = kScratchM + kConsumerWarps * 8 * 4;
 constexpr int kScratchE = kScratchL + kConsumerWarps * 8 * 4;
 static_assert(kScratchE + 8 * 4 <= kStageBytes, "merge scratch must fit in one stage");
-constexpr int kBarriers = kStages * kStageBytes;
+// query A fragments of the current pair (hi/lo fp16, 8 k-chunks x 32 lanes x
+// 16 B) and the per-row power-of-two scale, shared by the consumer warps
+constexpr int kQFrag = kStages * kStageBytes;
+constexpr int kQScale = kQFrag + 8 * 32 * 16;
+constexpr int kBarriers = kQScale + 8 * 4;
+// abort flag (+0), CTA range and walk start (+8..+47)
 constexpr int kLocate = kBarriers + 2 * kStages * 8;
 constexpr int kSmemBytes = kLocate + 64;
 static_assert(kStageBytes % 16 == 0, "stage alignment");
@@ -277,6 +287,125 @@ __device__ __forceinline__ uint32_t k_pair(const uint4 (&kw)[4], int j, int k, u
   }
 }
 
+// ------------------------------------------------------------ merging
+// CTA that owns global page g when P pages are split as [c P / N, (c+1) P / N)
+__device__ __forceinline__ int64_t cta_of_page(int64_t g, int64_t N, int64_t P) {
+  return ((g + 1) * N + P - 1) / P - 1;
+}
+__device__ __forceinline__ bool cta_empty(int64_t c, int64_t N, int64_t P) {
+  return c * P / N == (c + 1) * P / N;
+}
+
+// Merge the records that CTAs c_lo..c_hi wrote for rows rr[0..NR) of
+// `pair`, divide by l and apply R^-1 = D Hn B^T of head parameters hp; the
+// warp stores row k's 128 outputs at dst[k] (lane holds dims 4 lane ..
+// 4 lane + 3), or skips row k when dst[k] is null.  CTAs with an empty page
+// range (possible only when there are fewer pages than CTAs) wrote no record
+// and are skipped.  Latency, not bandwidth, bounds this: lane i fetches the
+// (m, l) of record c_lo + i, and the o vectors are fetched 8 (record, row)
+// pairs at a time before any is used.  Records are read through L2
+// (ld.global.cg): in the fused path other CTAs of the running grid wrote
+// them.
+template <int NR>
+__device__ __forceinline__ void merge_rows(const float *records, int64_t pair, int64_t c_lo, int64_t c_hi, int64_t N,
+                                           int64_t total, const int (&rr)[NR], float *const (&dst)[NR],
+                                           const HeadParams &hp, int lane) {
+  // this lane's rows of B^T, fetched first so that their latency overlaps
+  const float4 *mb4 = reinterpret_cast<const float4 *>(hp.m32[lane]);
+  const float4 mb[4] = {mb4[0], mb4[1], mb4[2], mb4[3]};
+  const uint32_t sn = (hp.sign_bits[lane >> 3] >> (4 * (lane & 7))) & 0xFu;
+
+  // pass 1: running (max, sum) per lane over its records, then across lanes
+  float mr[NR], lr[NR], m0[NR];
+#pragma unroll
+  for (int k = 0; k < NR; ++k) { mr[k] = -INFINITY; lr[k] = 0.f; m0[k] = -INFINITY; }
+  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
+    const int64_t c = c0 + lane;
+    if (c <= c_hi && !cta_empty(c, N, total)) {
+      const float *rec = records + (c + pair) * kRecordFloats;
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(rec + 2 * rr[k]));
+        if (c0 == c_lo) m0[k] = ml.x;
+        if (ml.x > mr[k]) {
+          lr[k] = lr[k] * ex2(mr[k] - ml.x) + ml.y;
+          mr[k] = ml.x;
+        } else if (ml.x != -INFINITY) {
+          lr[k] += ml.y * ex2(ml.x - mr[k]);
+        }
+      }
+    }
+  }
+  float M[NR], l[NR], o[NR][4];
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    M[k] = mr[k];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M[k] = fmaxf(M[k], __shfl_xor_sync(0xffffffffu, M[k], off));
+    l[k] = (mr[k] == -INFINITY) ? 0.f : lr[k] * ex2(mr[k] - M[k]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) l[k] += __shfl_xor_sync(0xffffffffu, l[k], off);
+    o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
+  }
+  // pass 2: o = sum over records of 2^(m - M) o_c
+  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
+    const int64_t c = c0 + lane;
+    const bool mine = c <= c_hi && !cta_empty(c, N, total);
+    float sm[NR];
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      float mc = m0[k];
+      if (c0 != c_lo) mc = mine ? __ldcg(records + (c + pair) * kRecordFloats + 2 * rr[k]) : -INFINITY;
+      sm[k] = (!mine || M[k] == -INFINITY) ? 0.f : ex2(mc - M[k]);
+    }
+    const int n = static_cast<int>(c_hi - c0 + 1 < 32 ? c_hi - c0 + 1 : 32);
+    constexpr int kBatch = 8 / NR;
+    for (int i0 = 0; i0 < n; i0 += kBatch) {
+      float sv[kBatch][NR];
+      float4 v[kBatch][NR];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const float *rec = records + (c0 + i0 + u + pair) * kRecordFloats + 16 + 4 * lane;
+#pragma unroll
+        for (int k = 0; k < NR; ++k) {
+          sv[u][k] = __shfl_sync(0xffffffffu, sm[k], (i0 + u) & 31);
+          v[u][k] = (i0 + u < n && sv[u][k] != 0.f) ? __ldcg(reinterpret_cast<const float4 *>(rec + rr[k] * kD))
+                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+        for (int k = 0; k < NR; ++k) {
+          o[k][0] += sv[u][k] * v[u][k].x; o[k][1] += sv[u][k] * v[u][k].y;
+          o[k][2] += sv[u][k] * v[u][k].z; o[k][3] += sv[u][k] * v[u][k].w;
+        }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    if (dst[k] == nullptr) continue;
+    if (M[k] == -INFINITY || !(l[k] > 0.f)) {
+      *reinterpret_cast<float4 *>(dst[k]) = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    // o~ = sum p n C / (l sqrt(128)); then R^-1 = D Hn B^T, Hn = H / sqrt(128)
+    const float inv = 1.f / (l[k] * 128.f);
+    float y[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float *b0 = reinterpret_cast<const float *>(&mb[0]), *b1 = reinterpret_cast<const float *>(&mb[1]);
+      const float *b2 = reinterpret_cast<const float *>(&mb[2]), *b3 = reinterpret_cast<const float *>(&mb[3]);
+      y[c] = fmaf(b3[c], o[k][3], fmaf(b2[c], o[k][2], fmaf(b1[c], o[k][1], b0[c] * o[k][0])));
+    }
+    wht128<float>(y, lane);
+    float res[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) res[c] = __uint_as_float(__float_as_uint(y[c] * inv) ^ (((sn >> c) & 1u) << 31));
+    *reinterpret_cast<float4 *>(dst[k]) = make_float4(res[0], res[1], res[2], res[3]);
+  }
+}
+
 // ------------------------------------------------------------ partial kernel
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const PartialParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -300,6 +429,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // the set-up above touches only shared memory; global memory from here on
+  pdl_trigger();
+  pdl_wait();
   // CTA's page range [gs, ge) and where it starts
   if (warp == 0) {
     const int64_t pb = pages_before(p.seq_lens, p.B, ps, lane);
@@ -355,6 +487,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
       __syncwarp();
       const int64_t kblk = (static_cast<int64_t>(phys) * 2 + 0) * p.H + wk.h;
       const int64_t vblk = (static_cast<int64_t>(phys) * 2 + 1) * p.H + wk.h;
+#ifdef ISOQUANT_DENSE_STAGE
+      if (lane == 0) {
+        bulk_g2s(st + kStageKC, p.codes + kblk * kWords * ps, static_cast<uint32_t>(kWords * ps * 4), &full[stage]);
+      } else if (lane == 1) {
+        bulk_g2s(st + kStageVC, p.codes + vblk * kWords * ps, static_cast<uint32_t>(kWords * ps * 4), &full[stage]);
+      } else if (lane == 2 * kWords) {
+#else
       if (lane < kWords) {
         bulk_g2s(st + kStageKC + lane * kStrideK * 4, p.codes + (kblk * kWords + lane) * ps,
                  static_cast<uint32_t>(ps * 4), &full[stage]);
@@ -363,6 +502,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
         bulk_g2s(st + kStageVC + w * kStrideV * 4, p.codes + (vblk * kWords + w) * ps,
                  static_cast<uint32_t>(ps * 4), &full[stage]);
       } else if (lane == 2 * kWords) {
+#endif
         bulk_g2s(st + kStageKN, p.norms + kblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
       } else if (lane == 2 * kWords + 1) {
         bulk_g2s(st + kStageVN, p.norms + vblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
@@ -397,7 +537,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
     return 120 + gid;
   };
 
-  uint32_t qa[8][4];
+  uint4 *sq = reinterpret_cast<uint4 *>(smem + kQFrag);
+  float *sq_scale = reinterpret_cast<float *>(smem + kQScale);
   float acc[8][4];
   float m_run = -INFINITY, l_run = 0.f, inv2e = 1.f;
   int lim = 0, lim_min = 0, lim_max = 0;
@@ -408,44 +549,48 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
     const bool seg_start = (g == gs) || (wk.j == 0);
     const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
     if (seg_start) {
-      // load this pair's query rows as hi/lo fp16 A fragments
+      // every warp is done with the previous pair's query fragments
+      named_bar_sync(1, kConsumerWarps * 32);
       const int r = wk.rg * 8 + gid;
       const bool valid = r < p.R;
       const int qi = valid ? r / p.G : 0;
-      const int hq = wk.h * p.G + (valid ? r % p.G : 0);
-      const float *qp = p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD;
-      float qv[32];
-      float mx = 0.f;
+      if (warp == 0) {
+        // this pair's query rows as hi/lo fp16 A fragments, into shared memory
+        const int hq = wk.h * p.G + (valid ? r % p.G : 0);
+        const float *qp = p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD;
+        float qv[32];
+        float mx = 0.f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int d0 = kdim(k);
-        qv[2 * k] = valid ? qp[d0] * p.qfold : 0.f;
-        qv[2 * k + 1] = valid ? qp[d0 + 1] * p.qfold : 0.f;
-        mx = fmaxf(mx, fmaxf(fabsf(qv[2 * k]), fabsf(qv[2 * k + 1])));
-      }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      // power-of-two prescale: the largest |q| lands in [2^14, 2^15)
-      int ex = 0;
-      if (mx > 0.f) frexpf(mx, &ex);
-      ex = max(ex, -100);
-      const float up = ldexpf(1.f, 15 - ex);
-      inv2e = ldexpf(1.f, ex - 15);
-      uint32_t hi[16], lo[16];
+        for (int k = 0; k < 16; ++k) {
+          const int d0 = kdim(k);
+          qv[2 * k] = valid ? qp[d0] * p.qfold : 0.f;
+          qv[2 * k + 1] = valid ? qp[d0 + 1] * p.qfold : 0.f;
+          mx = fmaxf(mx, fmaxf(fabsf(qv[2 * k]), fabsf(qv[2 * k + 1])));
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        // power-of-two prescale: the largest |q| lands in [2^14, 2^15)
+        int ex = 0;
+        if (mx > 0.f) frexpf(mx, &ex);
+        ex = max(ex, -100);
+        const float up = ldexpf(1.f, 15 - ex);
+        if (tq == 0) sq_scale[gid] = ldexpf(1.f, ex - 15);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float a = qv[2 * k] * up, b = qv[2 * k + 1] * up;
-        const __half ah = __float2half_rn(a), bh = __float2half_rn(b);
-        hi[k] = pack_half2(__half2float(ah), __half2float(bh));
-        lo[k] = pack_half2(a - __half2float(ah), b - __half2float(bh));
-      }
+        for (int c = 0; c < 8; ++c) {
+          uint32_t hl[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        qa[c][0] = hi[2 * c];
-        qa[c][1] = lo[2 * c];
-        qa[c][2] = hi[2 * c + 1];
-        qa[c][3] = lo[2 * c + 1];
+          for (int e = 0; e < 2; ++e) {
+            const int k = 2 * c + e;
+            const float a = qv[2 * k] * up, b = qv[2 * k + 1] * up;
+            const __half ah = __float2half_rn(a), bh = __float2half_rn(b);
+            hl[2 * e] = pack_half2(__half2float(ah), __half2float(bh));
+            hl[2 * e + 1] = pack_half2(a - __half2float(ah), b - __half2float(bh));
+          }
+          sq[c * 32 + lane] = make_uint4(hl[0], hl[1], hl[2], hl[3]);
+        }
       }
+      named_bar_sync(1, kConsumerWarps * 32);
+      inv2e = sq_scale[gid];
       const int L = wk.L;
       lim = valid ? (p.causal ? L - p.nq + qi + 1 : L) : L;
       lim = max(lim, 0);
@@ -478,14 +623,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
 
       // ---- scores: tile t = 4h + j, column n = token t0 + 32h + 4n + j.  The
       // k-chunk loop is outermost so that the 8 tiles' mma chains interleave.
+#ifdef ISOQUANT_DENSE_STAGE
+      const int rsK = ps, rsV = ps;
+#else
+      constexpr int rsK = kStrideK, rsV = kStrideV;
+#endif
       uint4 kw[2][4];  // words 3tq, 3tq+1, 3tq+2 and 12 of tokens t0 + 32h + 4gid + {0..3}
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t *kb = kc + t0 + 32 * h + 4 * gid;
-        kw[h][0] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 0) * kStrideK);
-        kw[h][1] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 1) * kStrideK);
-        kw[h][2] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 2) * kStrideK);
-        kw[h][3] = *reinterpret_cast<const uint4 *>(kb + 12 * kStrideK);
+        kw[h][0] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 0) * rsK);
+        kw[h][1] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 1) * rsK);
+        kw[h][2] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 2) * rsK);
+        kw[h][3] = *reinterpret_cast<const uint4 *>(kb + 12 * rsK);
       }
       const uint32_t sh12 = 6 * tq;
       float d[8][4];
@@ -493,11 +643,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
       for (int t = 0; t < 8; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
+        const uint4 qa = sq[c * 32 + lane];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
           const uint32_t b0 = k_pair(kw[t >> 2], t & 3, 2 * c, sh12, lane4);
           const uint32_t b1 = k_pair(kw[t >> 2], t & 3, 2 * c + 1, sh12, lane4);
-          mma16816(d[t], qa[c][0], qa[c][1], qa[c][2], qa[c][3], b0, b1);
+          mma16816(d[t], qa.x, qa.y, qa.z, qa.w, b0, b1);
         }
       }
       float x[16];  // x[8h + i] = token t0 + 32h + 8tq + i
@@ -571,12 +722,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t *vb = vc + t0 + 32 * h + 8 * tq;
-        const uint4 va0 = *reinterpret_cast<const uint4 *>(vb + gid * kStrideV);
-        const uint4 va1 = *reinterpret_cast<const uint4 *>(vb + gid * kStrideV + 4);
-        const uint4 vb0 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * kStrideV);
-        const uint4 vb1 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * kStrideV + 4);
-        const uint4 vz0 = *reinterpret_cast<const uint4 *>(vb + 12 * kStrideV);
-        const uint4 vz1 = *reinterpret_cast<const uint4 *>(vb + 12 * kStrideV + 4);
+        const uint4 va0 = *reinterpret_cast<const uint4 *>(vb + gid * rsV);
+        const uint4 va1 = *reinterpret_cast<const uint4 *>(vb + gid * rsV + 4);
+        const uint4 vb0 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * rsV);
+        const uint4 vb1 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * rsV + 4);
+        const uint4 vz0 = *reinterpret_cast<const uint4 *>(vb + 12 * rsV);
+        const uint4 vz1 = *reinterpret_cast<const uint4 *>(vb + 12 * rsV + 4);
 #pragma unroll
         for (int kap = 0; kap < 2; ++kap) {
           uint32_t va[2][16];
@@ -610,6 +761,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
     }
     if (seg_end) {
       // ---- merge the consumer warps' states and write one record
+      const int64_t pair = (static_cast<int64_t>(wk.rg) * p.B + wk.b) * p.H + wk.h;
       // every warp is done reading this stage: reuse it as merge scratch
       named_bar_sync(1, kConsumerWarps * 32);
       uint8_t *scr = smem + static_cast<size_t>(stage) * kStageBytes;
@@ -634,7 +786,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
         if (warp == 0) sm_e[gid] = inv2e;
       }
       named_bar_sync(1, kConsumerWarps * 32);
-      const int64_t pair = (static_cast<int64_t>(wk.rg) * p.B + wk.b) * p.H + wk.h;
       float *rec = p.records + (blockIdx.x + pair) * static_cast<int64_t>(kRecordFloats);
       for (int e = tid; e < 8 * 32; e += kConsumerWarps * 32) {
         const int row = e >> 5, d0 = (e & 31) * 4;
@@ -677,15 +828,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
 }
 
 // ------------------------------------------------------------ combine kernel
-// CTA that owns global page g when P pages are split as [c P / N, (c+1) P / N)
-__device__ __forceinline__ int64_t cta_of_page(int64_t g, int64_t N, int64_t P) {
-  return ((g + 1) * N + P - 1) / P - 1;
-}
-__device__ __forceinline__ bool cta_empty(int64_t c, int64_t N, int64_t P) {
-  return c * P / N == (c + 1) * P / N;
-}
 
-__global__ void __launch_bounds__(256) k_attend_combine(const CombineParams p) {
+// Small blocks, so that they fit beside partial-kernel CTAs as soon as any
+// SM has room, and wait there for the partial kernel to complete.
+constexpr int kCombineThreads = 128;
+
+__global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const CombineParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const uint32_t row_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t n_rows = static_cast<uint32_t>(p.B) * p.nq * p.Hq;
@@ -711,58 +861,9 @@ __global__ void __launch_bounds__(256) k_attend_combine(const CombineParams p) {
   const int64_t N = p.n_cta;
   const int64_t c_lo = cta_of_page(g0, N, total), c_hi = cta_of_page(g0 + np - 1, N, total);
   const int64_t pair = (static_cast<int64_t>(rg) * p.B + b) * p.H + h;
-
-  // CTAs with an empty page range (possible when there are fewer pages than
-  // CTAs) wrote no record: skip them.  Lane i reads the (m, l) of record
-  // c_lo + i, so the records' maxima and weights come from one round trip.
-  float M = -INFINITY;
-  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
-    const int64_t c = c0 + lane;
-    if (c <= c_hi && !cta_empty(c, N, total)) M = fmaxf(M, p.records[(c + pair) * kRecordFloats + 2 * rr]);
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float o[4] = {0.f, 0.f, 0.f, 0.f};
-  float l = 0.f;
-  if (M != -INFINITY) {
-    for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
-      const int64_t c = c0 + lane;
-      float s_mine = 0.f;
-      if (c <= c_hi && !cta_empty(c, N, total)) {
-        const float *rec = p.records + (c + pair) * kRecordFloats;
-        s_mine = ex2(rec[2 * rr] - M);
-        l += s_mine * rec[2 * rr + 1];
-      }
-      const int n = static_cast<int>(c_hi - c0 + 1 < 32 ? c_hi - c0 + 1 : 32);
-      for (int i = 0; i < n; ++i) {
-        const float s = __shfl_sync(0xffffffffu, s_mine, i);
-        if (s == 0.f) continue;  // empty CTA, or a record with nothing visible
-        const float4 v =
-            *reinterpret_cast<const float4 *>(p.records + (c0 + i + pair) * kRecordFloats + 16 + rr * kD + 4 * lane);
-        o[0] += s * v.x; o[1] += s * v.y; o[2] += s * v.z; o[3] += s * v.w;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-  }
-  if (M == -INFINITY || !(l > 0.f)) {
-    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  // o~ = sum p n C / (l sqrt(128)); then R^-1 = D Hn B^T, Hn = H / sqrt(128)
-  const float inv = 1.f / (l * 128.f);
-  const HeadParams &hp = p.params[h];
-  const float *mb = hp.m32[lane];
-  float y[4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    y[c] = fmaf(mb[12 + c], o[3], fmaf(mb[8 + c], o[2], fmaf(mb[4 + c], o[1], mb[c] * o[0])));
-  wht128<float>(y, lane);
-  const uint32_t sn = (hp.sign_bits[lane >> 3] >> (4 * (lane & 7))) & 0xFu;
-  float res[4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) res[c] = __uint_as_float(__float_as_uint(y[c] * inv) ^ (((sn >> c) & 1u) << 31));
-  *reinterpret_cast<float4 *>(dst) = make_float4(res[0], res[1], res[2], res[3]);
+  const int rows[1] = {rr};
+  float *const dsts[1] = {dst};
+  merge_rows<1>(p.records, pair, c_lo, c_hi, N, total, rows, dsts, p.params[h], lane);
 }
 
 }  // namespace
@@ -807,8 +908,7 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
   p.records = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
   p.status = ctx->status;
   p.n_cta = s.n_cta;
-  k_attend_partial<<<s.n_cta, kThreads, kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(k_attend_partial, dim3(s.n_cta), dim3(kThreads), kSmemBytes, stream, p);
 }
 
 cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s, const int32_t *seq_lens,
@@ -827,10 +927,9 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
   p.page_size = s.page_size;
   p.n_cta = s.n_cta;
   const int64_t rows = static_cast<int64_t>(s.batch) * s.nq * s.q_heads;
-  const int64_t blocks = (rows * 32 + 255) / 256;
+  const int64_t blocks = (rows * 32 + kCombineThreads - 1) / kCombineThreads;
   if (blocks == 0) return cudaSuccess;
-  k_attend_combine<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(k_attend_combine, dim3(static_cast<unsigned>(blocks)), dim3(kCombineThreads), 0, stream, p);
 }
 
 }  // namespace isoquant

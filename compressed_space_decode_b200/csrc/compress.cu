@@ -82,6 +82,8 @@ __global__ void __launch_bounds__(256) k_compress(const HeadParams *__restrict__
                                                   uint32_t *__restrict__ codes,
                                                   uint16_t *__restrict__ norms, int num_pages,
                                                   int ps_shift, uint32_t *status) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int kv = blockIdx.y;
   const uint32_t w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -218,6 +220,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_rotate_q(const HeadParams *__restrict__ params,
                                                   const T *__restrict__ q, int n_rows, int Hq, int G,
                                                   float *__restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const uint32_t vec = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (vec >= static_cast<uint32_t>(n_rows) * static_cast<uint32_t>(Hq)) return;
@@ -244,25 +248,18 @@ cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache
   dim3 grid(static_cast<unsigned>(blocks), 2), block(256);
   switch (dtype) {
     case ISOQUANT_F32:
-      k_compress<float><<<grid, block, 0, stream>>>(ctx->params, ctx->codebook, static_cast<const float *>(k),
-                                                    static_cast<const float *>(v), n_tok, H, slot_mapping,
-                                                    cache->codes, cache->norms, cache->num_pages, ps_shift,
-                                                    ctx->status);
-      break;
+      return launch_pdl(k_compress<float>, grid, block, 0, stream, ctx->params, ctx->codebook,
+                        static_cast<const float *>(k), static_cast<const float *>(v), n_tok, H, slot_mapping,
+                        cache->codes, cache->norms, cache->num_pages, ps_shift, ctx->status);
     case ISOQUANT_BF16:
-      k_compress<__nv_bfloat16><<<grid, block, 0, stream>>>(
-          ctx->params, ctx->codebook, static_cast<const __nv_bfloat16 *>(k),
-          static_cast<const __nv_bfloat16 *>(v), n_tok, H, slot_mapping, cache->codes, cache->norms,
-          cache->num_pages, ps_shift, ctx->status);
-      break;
+      return launch_pdl(k_compress<__nv_bfloat16>, grid, block, 0, stream, ctx->params, ctx->codebook,
+                        static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), n_tok, H,
+                        slot_mapping, cache->codes, cache->norms, cache->num_pages, ps_shift, ctx->status);
     default:
-      k_compress<__half><<<grid, block, 0, stream>>>(ctx->params, ctx->codebook, static_cast<const __half *>(k),
-                                                     static_cast<const __half *>(v), n_tok, H, slot_mapping,
-                                                     cache->codes, cache->norms, cache->num_pages, ps_shift,
-                                                     ctx->status);
-      break;
+      return launch_pdl(k_compress<__half>, grid, block, 0, stream, ctx->params, ctx->codebook,
+                        static_cast<const __half *>(k), static_cast<const __half *>(v), n_tok, H, slot_mapping,
+                        cache->codes, cache->norms, cache->num_pages, ps_shift, ctx->status);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_rotate_q(const isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
@@ -274,19 +271,15 @@ cudaError_t launch_rotate_q(const isoquant_ctx *ctx, const void *q, int dtype, i
   dim3 grid(static_cast<unsigned>(blocks)), block(256);
   switch (dtype) {
     case ISOQUANT_F32:
-      k_rotate_q<float><<<grid, block, 0, stream>>>(ctx->params, static_cast<const float *>(q), n_rows,
-                                                    num_q_heads, G, q_rot);
-      break;
+      return launch_pdl(k_rotate_q<float>, grid, block, 0, stream, ctx->params, static_cast<const float *>(q),
+                        n_rows, num_q_heads, G, q_rot);
     case ISOQUANT_BF16:
-      k_rotate_q<__nv_bfloat16><<<grid, block, 0, stream>>>(
-          ctx->params, static_cast<const __nv_bfloat16 *>(q), n_rows, num_q_heads, G, q_rot);
-      break;
+      return launch_pdl(k_rotate_q<__nv_bfloat16>, grid, block, 0, stream, ctx->params,
+                        static_cast<const __nv_bfloat16 *>(q), n_rows, num_q_heads, G, q_rot);
     default:
-      k_rotate_q<__half><<<grid, block, 0, stream>>>(ctx->params, static_cast<const __half *>(q), n_rows,
-                                                     num_q_heads, G, q_rot);
-      break;
+      return launch_pdl(k_rotate_q<__half>, grid, block, 0, stream, ctx->params, static_cast<const __half *>(q),
+                        n_rows, num_q_heads, G, q_rot);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace isoquant

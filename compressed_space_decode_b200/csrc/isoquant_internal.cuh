@@ -76,6 +76,33 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
                                   const int32_t *seq_lens, const void *ws, float *out,
                                   cudaStream_t stream);
 
+// ------------------------------------------------------------ launch chain
+// Every kernel of the library is a programmatic dependent launch: it may be
+// scheduled while the kernel before it in the stream is still running, and
+// it calls pdl_wait() before it touches global memory, which returns once
+// that kernel has completed and its writes are visible.  pdl_trigger() at
+// the top of each CTA lets the next kernel's CTAs be scheduled as early as
+// resources allow, so a step's launch latencies overlap the running kernels.
+// After a kernel that never triggers (any other library's), the launch is
+// an ordinary stream-ordered one.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, A... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<P>(args)...);
+}
+
 // ------------------------------------------------------------ device helpers
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

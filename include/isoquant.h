@@ -131,12 +131,17 @@ int isoquant_compress_kv(isoquant_ctx *ctx, const isoquant_cache *cache,
 int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
                       int num_q_heads, float *q_rot, void *stream);
 
-/* Workspace bytes isoquant_attend_decode needs for this shape. */
+/* Workspace bytes isoquant_attend_decode (and the partial/combine pair)
+ * needs for this shape: a 256-byte header and one partial record of
+ * (16 + 8 * 128) floats per slot, a slot per CTA plus one per
+ * (row group, sequence, KV head) pair. */
 int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
                             int num_q_heads, size_t *bytes);
 
-/* Split-context decode attention over the packed cache, then the combine
- * step that merges the splits and applies R^-1 once.
+/* Split-context decode attention over the packed cache, then the merge of
+ * the splits with R^-1 applied once per output row (RotaryQuant, Abstract:
+ * attention on the packed codes in the rotated space).  Two kernel launches,
+ * the second a programmatic dependent launch that overlaps the first's tail.
  *   q_rot:      device float [batch][nq][num_q_heads][128] (from rotate_q)
  *   page_table: device int32 [batch][max_pages]
  *   seq_lens:   device int32 [batch]; tokens 0..seq_lens[b]-1 are in the
@@ -144,7 +149,9 @@ int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
  *   causal:     if nonzero, query position i sees tokens
  *               t <= seq_lens[b] - nq + i; otherwise all seq_lens[b] tokens
  *   scale:      softmax scale; 0 selects 1/sqrt(128)
- *   workspace:  device, >= isoquant_workspace_size bytes, 16-byte aligned
+ *   workspace:  device, >= isoquant_workspace_size bytes, 16-byte aligned;
+ *               its contents on entry do not matter; calls whose kernels
+ *               overlap on the GPU must not share one workspace
  *   out:        device float [batch][nq][num_q_heads][128]
  * A row that sees no token outputs zeros.  Rows of heads in one GQA group
  * share each KV tile.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE,
@@ -176,8 +183,9 @@ int isoquant_attend_decode_static(isoquant_ctx *ctx, const isoquant_cache *cache
                                   void *stream);
 
 /* The two halves of isoquant_attend_decode, for callers that schedule them
- * separately (same arguments; the partial half fills the workspace, the
- * combine half reads it and writes `out`). */
+ * separately (same arguments): the partial half writes the records to the
+ * workspace, the combine half (one warp per output row) merges them, applies
+ * R^-1 and writes `out`. */
 int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache,
                             const float *q_rot, int batch, int nq,
                             int num_q_heads, const int32_t *page_table,
