@@ -3,12 +3,13 @@
 Workload (default): GQA decode, batch 16, 32 query / 4 KV heads, d = 128,
 context 32768 (bf16 heavy-tailed K/V compressed into a paged 3-bit cache
 with 256-token pages and a shuffled page table).  One step = append one new
-token per sequence (isoquant_compress_kv), rotate the queries
-(isoquant_rotate_q), and split-context attention over the packed codes with
-the merge of the splits and the inverse rotation (isoquant_attend_decode:
-the partial and combine kernels): every row of the hot path.  All four
-kernels are programmatic dependent launches, so each one's launch overlaps
-the tail of the one before.
+token per sequence and rotate the queries (isoquant_decode_prep, one
+launch), then split-context attention over the packed codes with the merge
+of the splits and the inverse rotation (isoquant_attend_decode: the partial
+and combine kernels): every row of the hot path.  The kernels are
+programmatic dependent launches, so each one's launch overlaps the tail of
+the one before.  The end-to-end figure drives the same step through the
+one-call isoquant_decode_step.
 
 Metric: KV-token x KV-head pairs attended per second (sum over sequences of
 the context length times the KV heads, per step), and the achieved HBM
@@ -166,9 +167,10 @@ def run_ours(args):
     launches = [0]
 
     def step(s, k, v, q, slots, lens):
-        csd.isoquant_compress_kv(st.ctx, st.cache, k, v, slots, stream=stream)
-        launches[0] += csd.isoquant_last_launch_count(st.ctx)
-        csd.isoquant_rotate_q(st.ctx, q, q_rot.view(B * nq, Hq, 128), stream=stream)
+        # append + rotate q (one launch), then attention (partial + combine):
+        # the launches of isoquant_decode_step, issued as its two halves so
+        # that events can bracket the attention
+        csd.isoquant_decode_prep(st.ctx, st.cache, k, v, slots, q, q_rot.view(B * nq, Hq, 128), stream=stream)
         launches[0] += csd.isoquant_last_launch_count(st.ctx)
         ev = attn_events.get(s) if attn_events is not None else None
         if ev is not None:
@@ -239,6 +241,7 @@ def run_ours(args):
     qd, sd, ld = torch.empty_like(q_all[0]), torch.empty_like(slots_all[0]), torch.empty_like(lens_all[0])
     h2d = (kd.numel() * 2 + vd.numel() * 2 + qd.numel() * 2 + sd.numel() * 8 + ld.numel() * 4)
     d2h = out.numel() * 4
+    ws_step = csd.alloc_step_workspace(st.ctx, B, nq, Hq, device=dev)
     multi.barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -250,7 +253,9 @@ def run_ours(args):
         qd.copy_(qh[s], non_blocking=True)
         sd.copy_(slots_h[s], non_blocking=True)
         ld.copy_(lens_h[s], non_blocking=True)
-        step(0, kd, vd, qd, sd, ld)
+        # the one-call public API of a decode step
+        csd.isoquant_decode_step(st.ctx, st.cache, kd, vd, sd, qd.view(B, nq, Hq, 128), st.page_table, ld, ws_step,
+                                 out, causal=wl.causal, stream=stream)
         out_h[s].copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -274,7 +279,7 @@ def run_ours(args):
         "data": "synthetic (seeded bf16 Student-t(4) K/V, log-uniform channel scales, x20 outliers)",
         "config": {"workload": wl.name.split("@")[0], "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
                    "context_start": lens0[0], "page_size": st.ps, "page_table": "shuffled",
-                   "step": "append 1 token/seq + rotate_q + attend_decode (split-K attention + combine), programmatic launches",
+                   "step": "decode_prep (append 1 token/seq + rotate q, one launch) + attend_decode (split-K attention + combine); programmatic launches",
                    "l2": f"packed cache {bytes_per_launch / 1e6:.0f} MB > 126 MB L2; no flush",
                    "parallelism": f"dp{world} (independent shards)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -33,7 +33,8 @@ SYMBOLS = [
     "isoquant_init", "isoquant_destroy", "isoquant_strerror", "isoquant_codebook", "isoquant_cache_bytes",
     "isoquant_compress_kv", "isoquant_rotate_q", "isoquant_workspace_size", "isoquant_attend_decode",
     "isoquant_attend_partial", "isoquant_attend_combine", "isoquant_get_status", "isoquant_last_launch_count",
-    "isoquant_attend_decode_static",
+    "isoquant_attend_decode_static", "isoquant_decode_prep", "isoquant_step_workspace_size",
+    "isoquant_decode_step",
 ]
 
 
@@ -76,6 +77,10 @@ def lib():
             "isoquant_last_launch_count": ([vp], i32),
             "isoquant_attend_decode_static": ([vp, cp, vp, i32, i32, i32, vp, i32, vp, i32, ctypes.c_float, vp, vp],
                                               i32),
+            "isoquant_decode_prep": ([vp, cp, vp, vp, i32, vp, vp, i32, i32, i32, vp, vp], i32),
+            "isoquant_step_workspace_size": ([vp, i32, i32, i32, ctypes.POINTER(sz)], i32),
+            "isoquant_decode_step": ([vp, cp, vp, vp, i32, vp, vp, i32, i32, i32, i32, vp, i32, vp, i32,
+                                      ctypes.c_float, vp, sz, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -192,6 +197,48 @@ def isoquant_rotate_q(ctx, q, q_rot, stream=None):
     assert q.is_contiguous() and q_rot.is_contiguous() and q_rot.dtype == torch.float32
     _check(lib().isoquant_rotate_q(ctx.handle, _ptr(q), _dtype(q), q.shape[0], q.shape[1], _ptr(q_rot),
                                    _stream(stream)), "isoquant_rotate_q")
+
+
+def isoquant_decode_prep(ctx, cache, k, v, slot_mapping, q, q_rot, stream=None):
+    """Append k, v ([n_tok][H][128], device) at slot_mapping (int64 [n_tok])
+    and rotate q ([n_rows][Hq][128], same dtype) into q_rot (float32, same
+    shape), in one launch."""
+    assert k.is_contiguous() and v.is_contiguous() and slot_mapping.dtype == torch.int64
+    assert q.is_contiguous() and q_rot.is_contiguous() and q_rot.dtype == torch.float32
+    assert k.dtype == v.dtype == q.dtype
+    cs = cache.c_struct()
+    _check(lib().isoquant_decode_prep(ctx.handle, ctypes.byref(cs), _ptr(k), _ptr(v), k.shape[0], _ptr(slot_mapping),
+                                      _ptr(q), _dtype(q), q.shape[0], q.shape[1], _ptr(q_rot), _stream(stream)),
+           "isoquant_decode_prep")
+
+
+def isoquant_step_workspace_size(ctx, batch, nq, num_q_heads):
+    n = ctypes.c_size_t()
+    _check(lib().isoquant_step_workspace_size(ctx.handle, batch, nq, num_q_heads, ctypes.byref(n)),
+           "isoquant_step_workspace_size")
+    return n.value
+
+
+def alloc_step_workspace(ctx, batch, nq, num_q_heads, device="cuda"):
+    n = isoquant_step_workspace_size(ctx, batch, nq, num_q_heads)
+    return torch.empty(((n + 15) // 16) * 4, dtype=torch.int32, device=device)
+
+
+def isoquant_decode_step(ctx, cache, k, v, slot_mapping, q, page_table, seq_lens, workspace, out, causal=False,
+                         scale=0.0, stream=None):
+    """One decode step: append k, v (as isoquant_compress_kv), rotate q
+    ([B][nq][Hq][128], same dtype as k), attend over seq_lens tokens (which
+    count the appended ones) and write out (float32 [B][nq][Hq][128])."""
+    assert k.is_contiguous() and v.is_contiguous() and slot_mapping.dtype == torch.int64
+    assert q.is_contiguous() and q.dim() == 4 and k.dtype == v.dtype == q.dtype
+    assert page_table.dtype == torch.int32 and page_table.is_contiguous() and seq_lens.dtype == torch.int32
+    B, nq, Hq, _ = q.shape
+    cs = cache.c_struct()
+    _check(lib().isoquant_decode_step(ctx.handle, ctypes.byref(cs), _ptr(k), _ptr(v), k.shape[0], _ptr(slot_mapping),
+                                      _ptr(q), _dtype(q), B, nq, Hq, _ptr(page_table), page_table.shape[1],
+                                      _ptr(seq_lens), int(bool(causal)), float(scale), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
+           "isoquant_decode_step")
 
 
 def isoquant_workspace_size(ctx, batch, nq, num_q_heads):

@@ -253,6 +253,82 @@ int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows, i
   return ISOQUANT_OK;
 }
 
+int isoquant_decode_prep(isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v, int n_tok,
+                         const int64_t *slot_mapping, const void *q, int dtype, int n_rows, int num_q_heads,
+                         float *q_rot, void *stream) {
+  if (ctx == nullptr || n_tok < 0 || n_rows < 0 || num_q_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 0;
+  int st = check_cache(cache);
+  if (st != ISOQUANT_OK) return st;
+  if (num_q_heads % ctx->num_kv_heads != 0) return ISOQUANT_ERR_INVALID_ARG;
+  const int eb = dtype_bytes(dtype);
+  if (eb == 0) return ISOQUANT_ERR_UNSUPPORTED;
+  const uintptr_t need = eb == 4 ? 16 : 8;
+  if (n_tok > 0) {
+    if (k == nullptr || v == nullptr || slot_mapping == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+    if (!aligned(k, need) || !aligned(v, need) || !aligned(slot_mapping, 8)) return ISOQUANT_ERR_ALIGNMENT;
+  }
+  if (n_rows > 0) {
+    if (q == nullptr || q_rot == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+    if (!aligned(q, need) || !aligned(q_rot, 16)) return ISOQUANT_ERR_ALIGNMENT;
+  }
+  if (n_tok == 0 && n_rows == 0) return ISOQUANT_OK;
+  cudaError_t e = launch_decode_prep(ctx, cache, k, v, n_tok, slot_mapping, q, dtype, n_rows, num_q_heads, q_rot,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
+  ctx->last_launches = 1;
+  return ISOQUANT_OK;
+}
+
+namespace {
+size_t round_up_256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+}  // namespace
+
+int isoquant_step_workspace_size(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, size_t *bytes) {
+  if (ctx == nullptr || bytes == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  AttendShape s;
+  int st = make_shape(ctx, batch, nq, num_q_heads, 256, 0, &s);
+  if (st != ISOQUANT_OK) return st;
+  *bytes = round_up_256(attend_workspace_bytes(s)) +
+           static_cast<size_t>(batch) * nq * num_q_heads * kD * sizeof(float);
+  return ISOQUANT_OK;
+}
+
+int isoquant_decode_step(isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v, int n_tok,
+                         const int64_t *slot_mapping, const void *q, int dtype, int batch, int nq, int num_q_heads,
+                         const int32_t *page_table, int max_pages, const int32_t *seq_lens, int causal,
+                         float scale, void *workspace, size_t ws_bytes, float *out, void *stream) {
+  if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 0;
+  size_t need = 0;
+  int st = isoquant_step_workspace_size(ctx, batch, nq, num_q_heads, &need);
+  if (st != ISOQUANT_OK) return st;
+  int st_cache = check_cache(cache);
+  if (st_cache != ISOQUANT_OK) return st_cache;
+  if (batch == 0) {
+    // nothing to attend; the new tokens are still appended
+    return isoquant_compress_kv(ctx, cache, k, v, dtype, n_tok, slot_mapping, stream);
+  }
+  if (workspace == nullptr || out == nullptr || page_table == nullptr || seq_lens == nullptr || max_pages < 1)
+    return ISOQUANT_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16) || !aligned(out, 16) || !aligned(page_table, 4) || !aligned(seq_lens, 4))
+    return ISOQUANT_ERR_ALIGNMENT;
+  if (ws_bytes < need) return ISOQUANT_ERR_WORKSPACE;
+  if (!(scale >= 0.0f) || !std::isfinite(scale)) return ISOQUANT_ERR_INVALID_ARG;
+  AttendShape s;
+  st = make_shape(ctx, batch, nq, num_q_heads, cache->page_size, causal, &s);
+  if (st != ISOQUANT_OK) return st;
+  const size_t attend_bytes = round_up_256(attend_workspace_bytes(s));
+  float *q_rot = reinterpret_cast<float *>(static_cast<char *>(workspace) + attend_bytes);
+  st = isoquant_decode_prep(ctx, cache, k, v, n_tok, slot_mapping, q, dtype, batch * nq, num_q_heads, q_rot, stream);
+  if (st != ISOQUANT_OK) return st;
+  const int prep = ctx->last_launches;
+  st = isoquant_attend_decode(ctx, cache, q_rot, batch, nq, num_q_heads, page_table, max_pages, seq_lens, causal,
+                              scale, workspace, attend_bytes, out, stream);
+  ctx->last_launches += prep;
+  return st;
+}
+
 int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, size_t *bytes) {
   if (ctx == nullptr || bytes == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   AttendShape s;

@@ -75,18 +75,32 @@ __device__ __forceinline__ void rotate_f64(const HeadParams &hp, int lane, const
 // tokens' inputs are all requested before the first is rotated.
 constexpr int kVecPerWarp = 4;
 
+struct CompressArgs {
+  const HeadParams *params;
+  Codebook cb;
+  const void *kin, *vin;
+  int n_tok, H;
+  const int64_t *slots;
+  uint32_t *codes;
+  uint16_t *norms;
+  int num_pages, ps_shift;
+  uint32_t *status;
+};
+
+// Warp w of the K (kv = 0) or V (kv = 1) half: rotate, quantize and pack
+// tokens kVecPerWarp * (w / H) .. + kVecPerWarp - 1 of head w % H.
 template <typename T>
-__global__ void __launch_bounds__(256) k_compress(const HeadParams *__restrict__ params, Codebook cb,
-                                                  const T *__restrict__ kin, const T *__restrict__ vin,
-                                                  int n_tok, int H, const int64_t *__restrict__ slots,
-                                                  uint32_t *__restrict__ codes,
-                                                  uint16_t *__restrict__ norms, int num_pages,
-                                                  int ps_shift, uint32_t *status) {
-  pdl_trigger();
-  pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int kv = blockIdx.y;
-  const uint32_t w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+__device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uint32_t w, int lane) {
+  const HeadParams *__restrict__ params = g.params;
+  const Codebook &cb = g.cb;
+  const T *__restrict__ kin = static_cast<const T *>(g.kin);
+  const T *__restrict__ vin = static_cast<const T *>(g.vin);
+  const int n_tok = g.n_tok, H = g.H;
+  const int64_t *__restrict__ slots = g.slots;
+  uint32_t *__restrict__ codes = g.codes;
+  uint16_t *__restrict__ norms = g.norms;
+  const int num_pages = g.num_pages, ps_shift = g.ps_shift;
+  uint32_t *status = g.status;
   const uint32_t groups = (static_cast<uint32_t>(n_tok) + kVecPerWarp - 1) / kVecPerWarp;
   const uint32_t tg = w / static_cast<uint32_t>(H);
   if (tg >= groups) return;
@@ -216,14 +230,28 @@ __global__ void __launch_bounds__(256) k_compress(const HeadParams *__restrict__
   }
 }
 
+// warps per compress block; blockIdx.y selects K or V
 template <typename T>
-__global__ void __launch_bounds__(256) k_rotate_q(const HeadParams *__restrict__ params,
-                                                  const T *__restrict__ q, int n_rows, int Hq, int G,
-                                                  float *__restrict__ out) {
+__global__ void __launch_bounds__(256) k_compress(const CompressArgs g) {
   pdl_trigger();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const uint32_t vec = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  compress_warp<T>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), threadIdx.x & 31);
+}
+
+struct RotateArgs {
+  const HeadParams *params;
+  const void *q;
+  int n_rows, Hq, G;
+  float *out;
+};
+
+// q_rot = R q for query vector `vec` (row vec / Hq, head vec % Hq).
+template <typename T>
+__device__ __forceinline__ void rotate_warp(const RotateArgs &g, uint32_t vec, int lane) {
+  const HeadParams *__restrict__ params = g.params;
+  const T *__restrict__ q = static_cast<const T *>(g.q);
+  const int n_rows = g.n_rows, Hq = g.Hq, G = g.G;
+  float *__restrict__ out = g.out;
   if (vec >= static_cast<uint32_t>(n_rows) * static_cast<uint32_t>(Hq)) return;
   const int hq = static_cast<int>(vec % static_cast<uint32_t>(Hq));
   float x[4], y[4];
@@ -233,52 +261,122 @@ __global__ void __launch_bounds__(256) k_rotate_q(const HeadParams *__restrict__
   *reinterpret_cast<float4 *>(out + static_cast<int64_t>(vec) * kD + 4 * lane) = make_float4(y[0] * s, y[1] * s, y[2] * s, y[3] * s);
 }
 
+template <typename T>
+__global__ void __launch_bounds__(256) k_rotate_q(const RotateArgs g) {
+  pdl_trigger();
+  pdl_wait();
+  rotate_warp<T>(g, (blockIdx.x * blockDim.x + threadIdx.x) >> 5, threadIdx.x & 31);
+}
+
+// One launch for the two independent halves of a decode step's preparation:
+// blocks [0, 2 nbc) compress the new K (first nbc) and V tokens, the rest
+// rotate the queries.  Their latency chains overlap instead of adding up.
+template <typename T>
+__global__ void __launch_bounds__(256) k_decode_prep(const CompressArgs c, const RotateArgs r, int nbc) {
+  pdl_trigger();
+  pdl_wait();
+  const uint32_t warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bx = static_cast<int>(blockIdx.x);
+  if (bx < 2 * nbc) {
+    const int kv = bx >= nbc ? 1 : 0;
+    compress_warp<T>(c, kv, static_cast<uint32_t>(bx - kv * nbc) * (blockDim.x >> 5) + warp, lane);
+  } else {
+    rotate_warp<T>(r, static_cast<uint32_t>(bx - 2 * nbc) * (blockDim.x >> 5) + warp, lane);
+  }
+}
+
+}  // namespace
+
+namespace {
+
+CompressArgs compress_args(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v,
+                           int n_tok, const int64_t *slot_mapping) {
+  CompressArgs g{};
+  g.params = ctx->params;
+  g.cb = ctx->codebook;
+  g.kin = k;
+  g.vin = v;
+  g.n_tok = n_tok;
+  g.H = ctx->num_kv_heads;
+  g.slots = slot_mapping;
+  g.codes = cache->codes;
+  g.norms = cache->norms;
+  g.num_pages = cache->num_pages;
+  int ps_shift = 0;
+  while ((1 << ps_shift) < cache->page_size) ++ps_shift;
+  g.ps_shift = ps_shift;
+  g.status = ctx->status;
+  return g;
+}
+
+// compress blocks per K/V half (8 warps each)
+int64_t compress_blocks(const isoquant_ctx *ctx, int n_tok) {
+  const int64_t warps = static_cast<int64_t>((n_tok + kVecPerWarp - 1) / kVecPerWarp) * ctx->num_kv_heads;
+  return (warps + 7) / 8;
+}
+
+RotateArgs rotate_args(const isoquant_ctx *ctx, const void *q, int n_rows, int num_q_heads, float *q_rot) {
+  RotateArgs g{};
+  g.params = ctx->params;
+  g.q = q;
+  g.n_rows = n_rows;
+  g.Hq = num_q_heads;
+  g.G = num_q_heads / ctx->num_kv_heads;
+  g.out = q_rot;
+  return g;
+}
+
+int64_t rotate_blocks(int n_rows, int num_q_heads) {
+  return (static_cast<int64_t>(n_rows) * num_q_heads * 32 + 255) / 256;
+}
+
 }  // namespace
 
 cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k,
                             const void *v, int dtype, int n_tok, const int64_t *slot_mapping,
                             cudaStream_t stream) {
-  const int H = ctx->num_kv_heads;
-  const int64_t warps = static_cast<int64_t>((n_tok + kVecPerWarp - 1) / kVecPerWarp) * H;
-  const int64_t blocks = (warps + 7) / 8;
+  const int64_t blocks = compress_blocks(ctx, n_tok);
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  int ps_shift = 0;
-  while ((1 << ps_shift) < cache->page_size) ++ps_shift;
-  dim3 grid(static_cast<unsigned>(blocks), 2), block(256);
+  const CompressArgs g = compress_args(ctx, cache, k, v, n_tok, slot_mapping);
+  const dim3 grid(static_cast<unsigned>(blocks), 2), block(256);
   switch (dtype) {
-    case ISOQUANT_F32:
-      return launch_pdl(k_compress<float>, grid, block, 0, stream, ctx->params, ctx->codebook,
-                        static_cast<const float *>(k), static_cast<const float *>(v), n_tok, H, slot_mapping,
-                        cache->codes, cache->norms, cache->num_pages, ps_shift, ctx->status);
-    case ISOQUANT_BF16:
-      return launch_pdl(k_compress<__nv_bfloat16>, grid, block, 0, stream, ctx->params, ctx->codebook,
-                        static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), n_tok, H,
-                        slot_mapping, cache->codes, cache->norms, cache->num_pages, ps_shift, ctx->status);
-    default:
-      return launch_pdl(k_compress<__half>, grid, block, 0, stream, ctx->params, ctx->codebook,
-                        static_cast<const __half *>(k), static_cast<const __half *>(v), n_tok, H, slot_mapping,
-                        cache->codes, cache->norms, cache->num_pages, ps_shift, ctx->status);
+    case ISOQUANT_F32: return launch_pdl(k_compress<float>, grid, block, 0, stream, g);
+    case ISOQUANT_BF16: return launch_pdl(k_compress<__nv_bfloat16>, grid, block, 0, stream, g);
+    default: return launch_pdl(k_compress<__half>, grid, block, 0, stream, g);
   }
 }
 
 cudaError_t launch_rotate_q(const isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
                             int num_q_heads, float *q_rot, cudaStream_t stream) {
-  const int G = num_q_heads / ctx->num_kv_heads;
-  const int64_t warps = static_cast<int64_t>(n_rows) * num_q_heads;
-  const int64_t blocks = (warps * 32 + 255) / 256;
+  const int64_t blocks = rotate_blocks(n_rows, num_q_heads);
   if (blocks == 0) return cudaSuccess;
-  dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  const RotateArgs g = rotate_args(ctx, q, n_rows, num_q_heads, q_rot);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
   switch (dtype) {
-    case ISOQUANT_F32:
-      return launch_pdl(k_rotate_q<float>, grid, block, 0, stream, ctx->params, static_cast<const float *>(q),
-                        n_rows, num_q_heads, G, q_rot);
-    case ISOQUANT_BF16:
-      return launch_pdl(k_rotate_q<__nv_bfloat16>, grid, block, 0, stream, ctx->params,
-                        static_cast<const __nv_bfloat16 *>(q), n_rows, num_q_heads, G, q_rot);
-    default:
-      return launch_pdl(k_rotate_q<__half>, grid, block, 0, stream, ctx->params, static_cast<const __half *>(q),
-                        n_rows, num_q_heads, G, q_rot);
+    case ISOQUANT_F32: return launch_pdl(k_rotate_q<float>, grid, block, 0, stream, g);
+    case ISOQUANT_BF16: return launch_pdl(k_rotate_q<__nv_bfloat16>, grid, block, 0, stream, g);
+    default: return launch_pdl(k_rotate_q<__half>, grid, block, 0, stream, g);
+  }
+}
+
+cudaError_t launch_decode_prep(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v,
+                               int n_tok, const int64_t *slot_mapping, const void *q, int dtype, int n_rows,
+                               int num_q_heads, float *q_rot, cudaStream_t stream) {
+  const int64_t nbc = compress_blocks(ctx, n_tok);
+  const int64_t nbr = rotate_blocks(n_rows, num_q_heads);
+  const int64_t blocks = 2 * nbc + nbr;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  const CompressArgs c = compress_args(ctx, cache, k, v, n_tok, slot_mapping);
+  const RotateArgs r = rotate_args(ctx, q, n_rows, num_q_heads, q_rot);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  const int nb = static_cast<int>(nbc);
+  switch (dtype) {
+    case ISOQUANT_F32: return launch_pdl(k_decode_prep<float>, grid, block, 0, stream, c, r, nb);
+    case ISOQUANT_BF16: return launch_pdl(k_decode_prep<__nv_bfloat16>, grid, block, 0, stream, c, r, nb);
+    default: return launch_pdl(k_decode_prep<__half>, grid, block, 0, stream, c, r, nb);
   }
 }
 

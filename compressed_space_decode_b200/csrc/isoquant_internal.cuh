@@ -57,6 +57,9 @@ cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache
                             cudaStream_t stream);
 cudaError_t launch_rotate_q(const isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
                             int num_q_heads, float *q_rot, cudaStream_t stream);
+cudaError_t launch_decode_prep(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k,
+                               const void *v, int n_tok, const int64_t *slot_mapping, const void *q,
+                               int dtype, int n_rows, int num_q_heads, float *q_rot, cudaStream_t stream);
 
 struct AttendShape {
   int batch, nq, q_heads, kv_heads, group, rows, row_groups, page_size, causal;

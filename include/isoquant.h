@@ -163,6 +163,42 @@ int isoquant_attend_decode(isoquant_ctx *ctx, const isoquant_cache *cache,
                            float scale, void *workspace, size_t ws_bytes,
                            float *out, void *stream);
 
+/* The preparation half of a decode step in one launch: append the step's new
+ * K/V tokens to the cache (as isoquant_compress_kv: k, v device
+ * [n_tok][num_kv_heads][128], slot_mapping device int64 [n_tok]) and rotate
+ * the queries (as isoquant_rotate_q: q device [n_rows][num_q_heads][128],
+ * q_rot device float, same shape).  The two are independent, so one grid
+ * does both and their latencies overlap.  k, v and q share `dtype`.  Either
+ * half may be empty (n_tok = 0 or n_rows = 0).  Errors: as the two calls. */
+int isoquant_decode_prep(isoquant_ctx *ctx, const isoquant_cache *cache,
+                         const void *k, const void *v, int n_tok,
+                         const int64_t *slot_mapping, const void *q, int dtype,
+                         int n_rows, int num_q_heads, float *q_rot,
+                         void *stream);
+
+/* Workspace bytes isoquant_decode_step needs: the attention workspace
+ * rounded up to 256 bytes, then the rotated queries
+ * (batch * nq * num_q_heads * 128 floats). */
+int isoquant_step_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
+                                 int num_q_heads, size_t *bytes);
+
+/* One whole decode step (RotaryQuant, Abstract: compress the new KV, then
+ * attend on the packed codes): isoquant_decode_prep (append + rotate q) and
+ * isoquant_attend_decode, three kernel launches chained by programmatic
+ * dependent launch.  Arguments as those calls; q is
+ * [batch][nq][num_q_heads][128] of `dtype`, seq_lens must already count the
+ * appended tokens, and the rotated queries live in the workspace
+ * (>= isoquant_step_workspace_size bytes, 16-byte aligned, contents on entry
+ * irrelevant).  With batch = 0 it only appends.  Errors: as those calls. */
+int isoquant_decode_step(isoquant_ctx *ctx, const isoquant_cache *cache,
+                         const void *k, const void *v, int n_tok,
+                         const int64_t *slot_mapping, const void *q, int dtype,
+                         int batch, int nq, int num_q_heads,
+                         const int32_t *page_table, int max_pages,
+                         const int32_t *seq_lens, int causal, float scale,
+                         void *workspace, size_t ws_bytes, float *out,
+                         void *stream);
+
 /* isoquant_attend_decode without a workspace argument, for callers that can
  * neither allocate device memory nor lend the library a buffer (a serving
  * process whose memory pool owns all device memory, or a decode loop that

@@ -313,3 +313,72 @@ def test_decode_step_graph_replay(cuda_lib):
         assert torch.equal(got, ref), step
     assert csd.isoquant_get_status(st.ctx) == 0
     del g
+
+
+def test_decode_prep_equals_separate_calls(cuda_lib):
+    """isoquant_decode_prep (append + rotate q in one launch) writes the same
+    cache bytes as isoquant_compress_kv and the same q_rot as
+    isoquant_rotate_q, bit for bit, for every input dtype."""
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    wl = csd.synthetic.workloads(small=True)["gqa_b16_q32_kv4_L32768_paged"]
+    for dt in (torch.bfloat16, torch.float16, torch.float32):
+        sa, sb = DecodeState(wl, growth=8), DecodeState(wl, growth=8)
+        k = torch.stack([sa.kv_tokens(b, sa.seq_lens[b], sa.seq_lens[b] + 3)[0] for b in range(sa.B)], 1)
+        v = torch.stack([sa.kv_tokens(b, sa.seq_lens[b], sa.seq_lens[b] + 3)[1] for b in range(sa.B)], 1)
+        k = k.reshape(-1, sa.H, D).to(dt).contiguous()
+        v = v.reshape(-1, sa.H, D).to(dt).contiguous()
+        slots = sa.slot_matrix(sa.seq_lens, 3).reshape(-1).contiguous()
+        q = sa.queries(0).reshape(-1, sa.Hq, D).to(dt).contiguous()
+        qa = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+        qb = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+        csd.isoquant_compress_kv(sa.ctx, sa.cache, k, v, slots)
+        csd.isoquant_rotate_q(sa.ctx, q, qa)
+        csd.isoquant_decode_prep(sb.ctx, sb.cache, k, v, slots, q, qb)
+        assert csd.isoquant_last_launch_count(sb.ctx) == 1
+        torch.cuda.synchronize()
+        assert csd.isoquant_get_status(sb.ctx) == 0
+        assert torch.equal(qa, qb), dt
+        assert torch.equal(sa.cache.codes, sb.cache.codes), dt
+        assert torch.equal(sa.cache.norms.view(torch.int16), sb.cache.norms.view(torch.int16)), dt
+
+
+def test_decode_step_matches_separate_calls_and_oracle(cuda_lib):
+    """isoquant_decode_step over several steps: the same outputs and cache as
+    compress_kv + rotate_q + attend_decode, and the oracle's attention."""
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    for name in ("gqa_b16_q32_kv4_L32768_paged", "verify_b8_nq16_q32_kv8_L16384"):
+        wl = csd.synthetic.workloads(small=True)[name]
+        nq = wl.nq
+        sa, sb = DecodeState(wl, growth=3 * nq), DecodeState(wl, growth=3 * nq)
+        ws_a = _ws(csd, sa)
+        ws_b = csd.alloc_step_workspace(sb.ctx, sb.B, nq, sb.Hq).fill_(0x7FC00000)
+        for step in range(3):
+            k = torch.stack([sa.kv_tokens(b, sa.seq_lens[b], sa.seq_lens[b] + nq)[0] for b in range(sa.B)], 1)
+            v = torch.stack([sa.kv_tokens(b, sa.seq_lens[b], sa.seq_lens[b] + nq)[1] for b in range(sa.B)], 1)
+            k = k.reshape(-1, sa.H, D).contiguous()
+            v = v.reshape(-1, sa.H, D).contiguous()
+            slots = sa.slot_matrix(sa.seq_lens, nq).reshape(-1).contiguous()
+            for st in (sa, sb):
+                st.seq_lens = [L + nq for L in st.seq_lens]
+                st.seq_lens_dev += nq
+            q = sa.queries(step)
+            # separate calls
+            q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+            out_a = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+            csd.isoquant_compress_kv(sa.ctx, sa.cache, k, v, slots)
+            csd.isoquant_rotate_q(sa.ctx, q.reshape(-1, sa.Hq, D), q_rot.view(-1, sa.Hq, D))
+            csd.isoquant_attend_decode(sa.ctx, sa.cache, q_rot, sa.page_table, sa.seq_lens_dev, ws_a, out_a,
+                                       causal=wl.causal)
+            # one call
+            out_b = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+            csd.isoquant_decode_step(sb.ctx, sb.cache, k, v, slots, q.contiguous(), sb.page_table, sb.seq_lens_dev,
+                                     ws_b, out_b, causal=wl.causal)
+            assert csd.isoquant_last_launch_count(sb.ctx) == 3
+            torch.cuda.synchronize()
+            assert csd.isoquant_get_status(sa.ctx) == 0 and csd.isoquant_get_status(sb.ctx) == 0
+            assert torch.equal(out_a, out_b), (name, step)
+        assert torch.equal(sa.cache.codes, sb.cache.codes)
+        b = sb.B - 1
+        check_pair(sb, b, sb.H - 1, q.float().cpu(), out_b.cpu())
