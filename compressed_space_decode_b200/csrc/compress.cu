@@ -70,11 +70,6 @@ __device__ __forceinline__ void rotate_f64(const HeadParams &hp, int lane, const
     out[r] = fma(m[4 * r + 3], y[3], fma(m[4 * r + 2], y[2], fma(m[4 * r + 1], y[1], m[4 * r] * y[0])));
 }
 
-// One warp handles kVecPerWarp consecutive tokens of one (head, K/V): the
-// head's block matrices and sign bits are loaded once into registers and the
-// tokens' inputs are all requested before the first is rotated.
-constexpr int kVecPerWarp = 4;
-
 struct CompressArgs {
   const HeadParams *params;
   Codebook cb;
@@ -84,155 +79,277 @@ struct CompressArgs {
   uint32_t *codes;
   uint16_t *norms;
   int num_pages, ps_shift;
+  int strip;  // tokens per warp strip (a multiple of 4)
   uint32_t *status;
 };
 
-// Warp w of the K (kv = 0) or V (kv = 1) half: rotate, quantize and pack
-// tokens kVecPerWarp * (w / H) .. + kVecPerWarp - 1 of head w % H.
-template <typename T>
-__device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uint32_t w, int lane) {
-  const HeadParams *__restrict__ params = g.params;
-  const Codebook &cb = g.cb;
-  const T *__restrict__ kin = static_cast<const T *>(g.kin);
-  const T *__restrict__ vin = static_cast<const T *>(g.vin);
-  const int n_tok = g.n_tok, H = g.H;
-  const int64_t *__restrict__ slots = g.slots;
-  uint32_t *__restrict__ codes = g.codes;
-  uint16_t *__restrict__ norms = g.norms;
-  const int num_pages = g.num_pages, ps_shift = g.ps_shift;
-  uint32_t *status = g.status;
-  const uint32_t groups = (static_cast<uint32_t>(n_tok) + kVecPerWarp - 1) / kVecPerWarp;
-  const uint32_t tg = w / static_cast<uint32_t>(H);
-  if (tg >= groups) return;
-  const int h = static_cast<int>(w - tg * static_cast<uint32_t>(H));
-  const int page_size = 1 << ps_shift;
-  const HeadParams &hp = params[h];
-  const T *src = kv ? vin : kin;
+// ------------------------------------------------------------ wide layout
+// A warp compresses four vectors of one head at a time: lane group
+// g = lane / 8 holds one vector, its lane q = lane % 8 holding coordinates
+// 16q..16q+15.  Four WHT strides (1..8) stay inside the lane and three
+// (16, 32, 64) cross lanes of the group, the lane's four SO(4) blocks
+// 4q..4q+3 stay in registers for the warp's whole strip of tokens, and the
+// per-vector work (norm rounding, packing) is shared by 8 lanes instead of
+// 32.
 
-  // this warp's tokens: inputs first, so their loads overlap
-  float x[kVecPerWarp][4];
-  int64_t slot[kVecPerWarp];
+__device__ __forceinline__ void load16(const float *p, float (&x)[16]) {
 #pragma unroll
-  for (int i = 0; i < kVecPerWarp; ++i) {
-    const int t = static_cast<int>(tg) * kVecPerWarp + i;
-    slot[i] = -1;
-    if (t < n_tok) {
-      slot[i] = slots[t];
-      load4(src + (static_cast<int64_t>(t) * H + h) * kD + 4 * lane, x[i]);
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = reinterpret_cast<const float4 *>(p)[i];
+    x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+  }
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16 *p, float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint4 u = reinterpret_cast<const uint4 *>(p)[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+      x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
     }
   }
-  const uint32_t sn = lane_sign_nibble(hp, lane);
-  float mrow[4][4];
+}
+__device__ __forceinline__ void load16(const __half *p, float (&x)[16]) {
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const float4 row = reinterpret_cast<const float4 *>(hp.m32[lane])[r];
-    mrow[r][0] = row.x; mrow[r][1] = row.y; mrow[r][2] = row.z; mrow[r][3] = row.w;
+  for (int i = 0; i < 2; ++i) {
+    const uint4 u = reinterpret_cast<const uint4 *>(p)[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
+      x[8 * i + 2 * k] = f.x;
+      x[8 * i + 2 * k + 1] = f.y;
+    }
+  }
+}
+
+// Sylvester WHT (unnormalised) of 128 values held 16 per lane by the 8 lanes
+// of a group, lane q holding elements 16q..16q+15 (q = lane & 7).  The lower
+// index of each butterfly keeps a+b, the upper one a-b.
+__device__ __forceinline__ void wht128_wide(float (&v)[16], int q) {
+#pragma unroll
+  for (int s = 1; s < 16; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i & s) continue;
+      const float a = v[i], b = v[i + s];
+      v[i] = a + b;
+      v[i + s] = a - b;
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < 8; m <<= 1) {
+    // lower lane: v + p; upper lane: p - v
+    const float sgn = (q & m) ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = fmaf(sgn, v[i], p);
+    }
+  }
+}
+
+// Pack the 128 codes of a lane group (lane q holding codes 16q..16q+15 at
+// bits 3e of cbits) into the 13 canonical words (word w: codes 10w..10w+9 at
+// bits 3(j - 10w)) and, if `store`, write the words that start in this lane
+// to codes[(row0 + w) << ps_shift].  A word that straddles two lanes gets
+// the second lane's part by one shuffle, which every lane executes.
+__device__ __forceinline__ void pack_store_wide(uint64_t cbits, int q, bool store, uint32_t *codes, int64_t row0,
+                                                int ps_shift) {
+  const int d0 = 16 * q;
+  const int wlo = d0 / 10, whi = (d0 + 15) / 10;
+  uint32_t part[3];
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    const int w = wlo + r;
+    const int j0 = max(10 * w, d0), j1 = min(10 * w + 10, d0 + 16);
+    part[r] = 0u;
+    if (w <= whi && j1 > j0) {
+      const uint64_t bits = (cbits >> (3 * (j0 - d0))) & ((1ull << (3 * (j1 - j0))) - 1ull);
+      part[r] = static_cast<uint32_t>(bits) << (3 * (j0 - 10 * w));
+    }
+  }
+  // the next lane's share of its first word (when that word began here)
+  const uint32_t nxt = __shfl_down_sync(0xffffffffu, part[0], 1);
+  const bool spans = q < 7 && (d0 + 16) % 10 != 0;  // word whi continues in lane q + 1
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    const int w = wlo + r;
+    if (w > whi) continue;
+    uint32_t word = part[r];
+    if (spans && w == whi) word |= nxt;
+    if (store && 10 * w >= d0) codes[(row0 + w) << ps_shift] = word;
+  }
+}
+
+// The fp64 path for one vector, by the whole warp (lane l: coordinates
+// 4l..4l+3): norm, rotation and codes all in fp64.  Used for the few vectors
+// whose fp16 norm rounding or codes the fp32 fast path cannot decide.
+template <typename T>
+__device__ void compress_one_fp64(const HeadParams &hp, const Codebook &cb, const T *src, uint32_t *codes,
+                                  uint16_t *norms, int64_t block, int off, int ps_shift, int lane) {
+  float xv[4];
+  load4(src + 4 * lane, xv);
+  double ss = static_cast<double>(xv[0]) * xv[0] + static_cast<double>(xv[1]) * xv[1] +
+              static_cast<double>(xv[2]) * xv[2] + static_cast<double>(xv[3]) * xv[3];
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  const double n = sqrt(ss);
+  const uint16_t n16 = __half_as_ushort(__double2half(fmin(n, 65504.0)));
+  double y64[4];
+  rotate_f64(hp, lane, xv, y64);
+  uint32_t c[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const double z = n > 0.0 ? y64[k] / n : 0.0;
+    uint32_t code = 0;
+#pragma unroll
+    for (int t = 0; t < kLevels - 1; ++t) code += (z > cb.threshold64[t]) ? 1u : 0u;
+    c[k] = code;
+  }
+  // word w holds codes 10w..10w+9, i.e. coordinates of lanes
+  // floor(10w/4) .. +2; an odd word starts two codes into its first lane.
+  const uint32_t c4 = c[0] | (c[1] << 3) | (c[2] << 6) | (c[3] << 9);
+  const int wd = lane;
+  const int a = (5 * wd) >> 1;
+  const uint32_t s0 = __shfl_sync(0xffffffffu, c4, a & 31);
+  const uint32_t s1 = __shfl_sync(0xffffffffu, c4, min(a + 1, 31));
+  const uint32_t s2 = __shfl_sync(0xffffffffu, c4, min(a + 2, 31));
+  const uint64_t comb = static_cast<uint64_t>(s0) | (static_cast<uint64_t>(s1) << 12) |
+                        (static_cast<uint64_t>(s2) << 24);
+  const uint32_t word =
+      static_cast<uint32_t>(comb >> ((wd & 1) ? 6 : 0)) & (wd == 12 ? 0x00FFFFFFu : 0x3FFFFFFFu);
+  if (lane < kWords) codes[((block * kWords + wd) << ps_shift) + off] = word;
+  if (lane == 0) norms[(block << ps_shift) + off] = n16;
+}
+
+// Warp w of the K (kv = 0) or V (kv = 1) half: rotate, quantize and pack
+// tokens strip * (w / H) .. + strip - 1 of head w % H, four at a time.
+template <typename T>
+__device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uint32_t w, int lane) {
+  const int H = g.H, n_tok = g.n_tok, ps_shift = g.ps_shift;
+  const uint32_t strips = (static_cast<uint32_t>(n_tok) + g.strip - 1) / g.strip;
+  const uint32_t sidx = w / static_cast<uint32_t>(H);
+  if (sidx >= strips) return;
+  const int h = static_cast<int>(w - sidx * static_cast<uint32_t>(H));
+  const HeadParams &hp = g.params[h];
+  const Codebook &cb = g.cb;
+  const T *__restrict__ src = static_cast<const T *>(kv ? g.vin : g.kin);
+  const int grp = lane >> 3, q = lane & 7;
+
+  // this lane's sign bits and SO(4) blocks 4q..4q+3, for the whole strip
+  const uint32_t sbits = (hp.sign_bits[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+  float mrow[4][16];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 row = reinterpret_cast<const float4 *>(hp.m32[4 * q + k])[r];
+      mrow[k][4 * r] = row.x; mrow[k][4 * r + 1] = row.y; mrow[k][4 * r + 2] = row.z; mrow[k][4 * r + 3] = row.w;
+    }
   }
   const float t4 = cb.threshold[4], t5 = cb.threshold[5], t6 = cb.threshold[6];
 
+  const int t_begin = static_cast<int>(sidx) * g.strip;
+  const int t_end = min(t_begin + g.strip, n_tok);
+  for (int tb = t_begin; tb < t_end; tb += 4) {
+    const int t = tb + grp;
+    const bool live = t < t_end;
+    float x[16];
+    int64_t slot = -1;
+    if (live) {
+      slot = g.slots[t];
+      load16(src + (static_cast<int64_t>(t) * H + h) * kD + 16 * q, x);
+    } else {
 #pragma unroll
-  for (int i = 0; i < kVecPerWarp; ++i) {
-    if (slot[i] < 0) continue;  // past the end, or a skipped token (uniform)
-    const int64_t page = slot[i] >> ps_shift;
-    const int off = static_cast<int>(slot[i] & (page_size - 1));
-    if (page >= num_pages) {
-      if (lane == 0) set_status(status, ISOQUANT_DEVERR_SLOT_RANGE);
-      continue;
+      for (int i = 0; i < 16; ++i) x[i] = 0.f;
     }
-    const float(&xv)[4] = x[i];
-    // ||x||^2 in fp32 (squares of bf16/fp16 inputs are exact; the tree sum is
-    // within 7 * 2^-24 relative).  The fp64 norm is only formed for the few
-    // vectors whose fp16 rounding the fp32 value cannot decide (below).
-    float ssf = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
+    const int64_t page = slot >> ps_shift;
+    const bool valid = live && slot >= 0 && page < g.num_pages;
+    if (live && slot >= 0 && page >= g.num_pages && q == 0) set_status(g.status, ISOQUANT_DEVERR_SLOT_RANGE);
+
+    // ||x||^2 in fp32: squares of bf16/fp16 inputs are exact and the tree
+    // (4 levels in the lane, 3 across the group) is within 7 * 2^-24
+    // relative; the fp16 norm is decided in fp32 unless n lies within 1e-6
+    // (relative) of a rounding midpoint, or is huge, tiny or not finite
+    float sq[16];
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) ssf += __shfl_xor_sync(0xffffffffu, ssf, m);
+    for (int i = 0; i < 16; ++i) sq[i] = x[i] * x[i];
+#pragma unroll
+    for (int s = 8; s >= 1; s >>= 1)
+#pragma unroll
+      for (int i = 0; i < s; ++i) sq[i] += sq[i + s];
+    float ssf = sq[0];
+    ssf += __shfl_xor_sync(0xffffffffu, ssf, 1);
+    ssf += __shfl_xor_sync(0xffffffffu, ssf, 2);
+    ssf += __shfl_xor_sync(0xffffffffu, ssf, 4);
     const float n32 = sqrtf(ssf);
-    // fp16 norm, round to nearest even: decided in fp32 unless n lies within
-    // 1e-6 (relative) of a rounding midpoint, or is huge, tiny or not finite
     const __half h32 = __float2half_rn(fminf(n32, 65504.f));
     const float hv = __half2float(h32);
     const uint16_t hb = __half_as_ushort(h32);
     const float up = __half2float(__ushort_as_half(static_cast<uint16_t>(hb + 1)));
     const float dn = hb > 0 ? __half2float(__ushort_as_half(static_cast<uint16_t>(hb - 1))) : 0.f;
     const float mid = n32 >= hv ? 0.5f * (hv + up) : 0.5f * (hv + dn);
-    const bool exact_f32 = ssf > 1e-30f && n32 < 65000.f && fabsf(n32 - mid) > 1e-6f * n32;
-    uint16_t n16 = hb;
-    float inv;
-    if (__all_sync(0xffffffffu, exact_f32)) {
-      // 1/n: hardware reciprocal square root plus one Newton step (~1e-7)
-      const float r = rsqrtf(ssf);
-      inv = r * (1.5f - 0.5f * ssf * r * r);
-    } else {
-      double ss = static_cast<double>(xv[0]) * xv[0] + static_cast<double>(xv[1]) * xv[1] +
-                  static_cast<double>(xv[2]) * xv[2] + static_cast<double>(xv[3]) * xv[3];
-#pragma unroll
-      for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-      const double n = sqrt(ss);
-      n16 = __half_as_ushort(__double2half(fmin(n, 65504.0)));
-      inv = n > 0.0 ? static_cast<float>(1.0 / n) : 0.0f;
-    }
+    bool slow = !(ssf > 1e-30f && n32 < 65000.f && fabsf(n32 - mid) > 1e-6f * n32);
+    // 1/n: hardware reciprocal square root plus one Newton step (~1e-7)
+    const float rs = rsqrtf(ssf);
+    const float inv = rs * (1.5f - 0.5f * ssf * rs * rs);
 
     // z = (B H D x) / n; sqrt(128) of the normalised Hn cancels against the
     // sqrt(128) of z = sqrt(128) * y / n.
-    float y[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) y[k] = __uint_as_float(__float_as_uint(xv[k]) ^ (((sn >> k) & 1u) << 31));
-    wht128<float>(y, lane);
-    // The codebook is symmetric (t_{6-k} = -t_k, t_3 = 0), so code_j =
-    // #{k : z > t_k} reads off |z| and the three positive thresholds:
-    // z > 0 -> 4 + #{|z| > t}, otherwise 3 - #{|z| >= t}.
-    uint32_t c[4];
+    for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(__float_as_uint(x[i]) ^ (((sbits >> i) & 1u) << 31));
+    wht128_wide(x, q);
+    // codes from |z| and the three positive thresholds (the codebook is
+    // symmetric): z > 0 -> 4 + #{|z| > t}, otherwise 3 - #{|z| >= t}
+    uint64_t cbits = 0;
     bool near = false;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float yr = fmaf(mrow[r][3], y[3], fmaf(mrow[r][2], y[2], fmaf(mrow[r][1], y[1], mrow[r][0] * y[0])));
-      const float z = yr * inv;
-      const float a = fabsf(z);
-      const uint32_t gt = (a > t4 ? 1u : 0u) + (a > t5 ? 1u : 0u) + (a > t6 ? 1u : 0u);
-      const uint32_t ge = (a >= t4 ? 1u : 0u) + (a >= t5 ? 1u : 0u) + (a >= t6 ? 1u : 0u);
-      c[r] = z > 0.f ? 4u + gt : 3u - ge;
-      near |= (a < kRecheckBand) | (fabsf(a - t4) < kRecheckBand) | (fabsf(a - t5) < kRecheckBand) |
-              (fabsf(a - t6) < kRecheckBand);
-    }
-    if (__any_sync(0xffffffffu, near && ssf > 0.f)) {
-      double ss = static_cast<double>(xv[0]) * xv[0] + static_cast<double>(xv[1]) * xv[1] +
-                  static_cast<double>(xv[2]) * xv[2] + static_cast<double>(xv[3]) * xv[3];
+    for (int k = 0; k < 4; ++k) {
 #pragma unroll
-      for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-      const double n64 = sqrt(ss);
-      double y64[4];
-      rotate_f64(hp, lane, xv, y64);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const double z = n64 > 0.0 ? y64[k] / n64 : 0.0;
-        uint32_t code = 0;
-#pragma unroll
-        for (int q = 0; q < kLevels - 1; ++q) code += (z > cb.threshold64[q]) ? 1u : 0u;
-        c[k] = code;
+      for (int r = 0; r < 4; ++r) {
+        const float yr = fmaf(mrow[k][4 * r + 3], x[4 * k + 3],
+                              fmaf(mrow[k][4 * r + 2], x[4 * k + 2],
+                                   fmaf(mrow[k][4 * r + 1], x[4 * k + 1], mrow[k][4 * r] * x[4 * k])));
+        const float z = yr * inv;
+        const float a = fabsf(z);
+        const uint32_t gt = (a > t4 ? 1u : 0u) + (a > t5 ? 1u : 0u) + (a > t6 ? 1u : 0u);
+        const uint32_t ge = (a >= t4 ? 1u : 0u) + (a >= t5 ? 1u : 0u) + (a >= t6 ? 1u : 0u);
+        const uint32_t c = z > 0.f ? 4u + gt : 3u - ge;
+        cbits |= static_cast<uint64_t>(c) << (3 * (4 * k + r));
+        near |= (a < kRecheckBand) | (fabsf(a - t4) < kRecheckBand) | (fabsf(a - t5) < kRecheckBand) |
+                (fabsf(a - t6) < kRecheckBand);
       }
     }
-
-    // pack: word w holds codes 10w..10w+9, i.e. coordinates of lanes
-    // floor(10w/4) .. +2; an odd word starts two codes into its first lane.
-    const uint32_t c4 = c[0] | (c[1] << 3) | (c[2] << 6) | (c[3] << 9);
-    const int wd = lane;
-    const int a = (5 * wd) >> 1;
-    const uint32_t s0 = __shfl_sync(0xffffffffu, c4, a & 31);
-    const uint32_t s1 = __shfl_sync(0xffffffffu, c4, min(a + 1, 31));
-    const uint32_t s2 = __shfl_sync(0xffffffffu, c4, min(a + 2, 31));
-    const uint64_t comb = static_cast<uint64_t>(s0) | (static_cast<uint64_t>(s1) << 12) |
-                          (static_cast<uint64_t>(s2) << 24);
-    const uint32_t word =
-        static_cast<uint32_t>(comb >> ((wd & 1) ? 6 : 0)) & (wd == 12 ? 0x00FFFFFFu : 0x3FFFFFFFu);
+    // the group's verdict: any lane near a threshold sends the vector to
+    // the fp64 path
+    const uint32_t gmask = 0xFFu << (8 * grp);
+    slow = (__ballot_sync(0xffffffffu, (near || slow) && valid) & gmask) != 0;
+    const int off = static_cast<int>(slot & ((1 << ps_shift) - 1));
     const int64_t block = (page * 2 + kv) * H + h;
-    if (lane < kWords) codes[((block * kWords + wd) << ps_shift) + off] = word;
-    if (lane == 0) norms[(block << ps_shift) + off] = n16;
+    const bool fast = valid && !slow;
+    pack_store_wide(cbits, q, fast, g.codes + off, block * kWords, ps_shift);
+    if (fast && q == 0) g.norms[(block << ps_shift) + off] = hb;
+    // vectors for the fp64 path, one at a time by the whole warp
+    uint32_t todo = __ballot_sync(0xffffffffu, valid && slow && q == 0);
+    while (todo) {
+      const int src_lane = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int gv = src_lane >> 3;
+      const int tv = tb + gv;
+      const int64_t sl = __shfl_sync(0xffffffffu, slot, src_lane);
+      const int64_t pg = sl >> ps_shift;
+      compress_one_fp64<T>(hp, cb, src + (static_cast<int64_t>(tv) * H + h) * kD, g.codes, g.norms,
+                           (pg * 2 + kv) * H + h, static_cast<int>(sl & ((1 << ps_shift) - 1)), ps_shift, lane);
+    }
   }
 }
 
 // warps per compress block; blockIdx.y selects K or V
 template <typename T>
-__global__ void __launch_bounds__(256) k_compress(const CompressArgs g) {
+__global__ void __launch_bounds__(256, 2) k_compress(const CompressArgs g) {
   pdl_trigger();
   pdl_wait();
   compress_warp<T>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), threadIdx.x & 31);
@@ -290,6 +407,11 @@ __global__ void __launch_bounds__(256) k_decode_prep(const CompressArgs c, const
 
 namespace {
 
+// Tokens per warp strip: long strips amortise loading a head's SO(4) blocks
+// in bulk compression; short ones spread a decode step's few tokens over
+// more warps.
+int strip_tokens(int n_tok) { return n_tok >= 4096 ? 16 : 4; }
+
 CompressArgs compress_args(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v,
                            int n_tok, const int64_t *slot_mapping) {
   CompressArgs g{};
@@ -306,13 +428,15 @@ CompressArgs compress_args(const isoquant_ctx *ctx, const isoquant_cache *cache,
   int ps_shift = 0;
   while ((1 << ps_shift) < cache->page_size) ++ps_shift;
   g.ps_shift = ps_shift;
+  g.strip = strip_tokens(n_tok);
   g.status = ctx->status;
   return g;
 }
 
-// compress blocks per K/V half (8 warps each)
+// compress blocks per K/V half (8 warps each, one strip per warp)
 int64_t compress_blocks(const isoquant_ctx *ctx, int n_tok) {
-  const int64_t warps = static_cast<int64_t>((n_tok + kVecPerWarp - 1) / kVecPerWarp) * ctx->num_kv_heads;
+  const int strip = strip_tokens(n_tok);
+  const int64_t warps = static_cast<int64_t>((n_tok + strip - 1) / strip) * ctx->num_kv_heads;
   return (warps + 7) / 8;
 }
 
