@@ -124,6 +124,18 @@ int make_shape(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, int 
   return ISOQUANT_OK;
 }
 
+}  // namespace
+
+int attend_workspace_min(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, size_t *bytes) {
+  AttendShape s;
+  int st = make_shape(ctx, batch, nq, num_q_heads, 256, 0, &s);
+  if (st != ISOQUANT_OK) return st;
+  *bytes = attend_workspace_min_bytes(s);
+  return ISOQUANT_OK;
+}
+
+namespace {
+
 int check_cache(const isoquant_cache *cache) {
   if (cache == nullptr || cache->codes == nullptr || cache->norms == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   if (cache->num_pages < 1) return ISOQUANT_ERR_INVALID_ARG;
@@ -355,9 +367,9 @@ int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache, cons
     return ISOQUANT_ERR_INVALID_ARG;
   if (!aligned(workspace, 16) || !aligned(q_rot, 4) || !aligned(page_table, 4) || !aligned(seq_lens, 4))
     return ISOQUANT_ERR_ALIGNMENT;
-  if (ws_bytes < attend_workspace_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
+  if (ws_bytes < attend_workspace_min_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
   cudaError_t e = launch_attend_partial(ctx, cache, s, q_rot, page_table, max_pages, seq_lens, scale, workspace,
-                                        static_cast<cudaStream_t>(stream));
+                                        ws_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
   ctx->last_launches = 1;
   return ISOQUANT_OK;
@@ -374,8 +386,8 @@ int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq, int num_q_head
   if (batch == 0) return ISOQUANT_OK;
   if (seq_lens == nullptr || workspace == nullptr || out == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   if (!aligned(workspace, 16) || !aligned(out, 16) || !aligned(seq_lens, 4)) return ISOQUANT_ERR_ALIGNMENT;
-  if (ws_bytes < attend_workspace_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
-  cudaError_t e = launch_attend_combine(ctx, s, seq_lens, workspace, out, static_cast<cudaStream_t>(stream));
+  if (ws_bytes < attend_workspace_min_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
+  cudaError_t e = launch_attend_combine(ctx, s, seq_lens, workspace, ws_bytes, out, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
   ctx->last_launches = 1;
   return ISOQUANT_OK;

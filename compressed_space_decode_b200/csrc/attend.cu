@@ -102,6 +102,7 @@ struct CombineParams {
   const int32_t *seq_lens;
   float *out;
   int B, nq, Hq, H, G, RG, page_size, n_cta;
+  int rps;  // query rows per stream: 8 (mma.sync kernel) or 64 (tcgen05 kernel)
 };
 
 // ------------------------------------------------------------------ PTX
@@ -306,10 +307,11 @@ __device__ __forceinline__ bool cta_empty(int64_t c, int64_t N, int64_t P) {
 // pairs at a time before any is used.  Records are read through L2
 // (ld.global.cg): in the fused path other CTAs of the running grid wrote
 // them.
+// Record of CTA c for the stream: slot (c + stream) * per + sub.
 template <int NR>
-__device__ __forceinline__ void merge_rows(const float *records, int64_t pair, int64_t c_lo, int64_t c_hi, int64_t N,
-                                           int64_t total, const int (&rr)[NR], float *const (&dst)[NR],
-                                           const HeadParams &hp, int lane) {
+__device__ __forceinline__ void merge_rows(const float *records, int64_t pair, int per, int sub, int64_t c_lo,
+                                           int64_t c_hi, int64_t N, int64_t total, const int (&rr)[NR],
+                                           float *const (&dst)[NR], const HeadParams &hp, int lane) {
   // this lane's rows of B^T, fetched first so that their latency overlaps
   const float4 *mb4 = reinterpret_cast<const float4 *>(hp.m32[lane]);
   const float4 mb[4] = {mb4[0], mb4[1], mb4[2], mb4[3]};
@@ -322,7 +324,7 @@ __device__ __forceinline__ void merge_rows(const float *records, int64_t pair, i
   for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
     const int64_t c = c0 + lane;
     if (c <= c_hi && !cta_empty(c, N, total)) {
-      const float *rec = records + (c + pair) * kRecordFloats;
+      const float *rec = records + ((c + pair) * per + sub) * kRecordFloats;
 #pragma unroll
       for (int k = 0; k < NR; ++k) {
         const float2 ml = __ldcg(reinterpret_cast<const float2 *>(rec + 2 * rr[k]));
@@ -355,7 +357,7 @@ __device__ __forceinline__ void merge_rows(const float *records, int64_t pair, i
 #pragma unroll
     for (int k = 0; k < NR; ++k) {
       float mc = m0[k];
-      if (c0 != c_lo) mc = mine ? __ldcg(records + (c + pair) * kRecordFloats + 2 * rr[k]) : -INFINITY;
+      if (c0 != c_lo) mc = mine ? __ldcg(records + ((c + pair) * per + sub) * kRecordFloats + 2 * rr[k]) : -INFINITY;
       sm[k] = (!mine || M[k] == -INFINITY) ? 0.f : ex2(mc - M[k]);
     }
     const int n = static_cast<int>(c_hi - c0 + 1 < 32 ? c_hi - c0 + 1 : 32);
@@ -365,7 +367,7 @@ __device__ __forceinline__ void merge_rows(const float *records, int64_t pair, i
       float4 v[kBatch][NR];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        const float *rec = records + (c0 + i0 + u + pair) * kRecordFloats + 16 + 4 * lane;
+        const float *rec = records + ((c0 + i0 + u + pair) * per + sub) * kRecordFloats + 16 + 4 * lane;
 #pragma unroll
         for (int k = 0; k < NR; ++k) {
           sv[u][k] = __shfl_sync(0xffffffffu, sm[k], (i0 + u) & 31);
@@ -827,6 +829,480 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
   }
 }
 
+// ------------------------------------------------------------ tcgen05 kernel
+// Many query rows per KV head (speculative verification: nq positions x G
+// heads, 64 rows and more).  The mma.sync kernel above decodes every KV
+// tile once per group of 8 rows; this one decodes it once for 64 rows and
+// runs both products on the fifth-generation tensor cores with the
+// accumulators in tensor memory.
+//
+// Work = pages of (stream, sequence, KV head), a stream being 64 query rows;
+// CTA c (two per SM) takes pages [c P / N, (c + 1) P / N) as above.  Per
+// 64-token tile of a page, the CTA's 4 warps (128 threads):
+//   1. decode the tile's K codes (threads 0..63, one token each, read from
+//      global memory word by word: 32 tokens' word w are 128 contiguous
+//      bytes) and V codes (threads 64..127) into fp16 centroid tiles in
+//      shared memory, both in
+//      the no-swizzle canonical layout: core matrix = 8 tokens x 8 dims
+//      (16 B per token row), dim chunks 128 B apart, token groups 2 KB
+//      apart.  K is read as a K-major B operand (N = tokens), V as an
+//      MN-major B operand (N = dims, K = tokens);
+//   2. S[128 x 64] = Q~ K^T with one tcgen05.mma per 16 dims: A = Q~, the
+//      64 rows' fp16 high parts in rows 0..63 and low parts in rows 64..127,
+//      so S's lanes 64..127 hold the low-part scores;
+//   3. thread r < 64 (row r) adds its two score halves (the low half through
+//      shared memory), applies the K norms, the row's prescale and the
+//      limits and runs the online softmax; p * n_v goes to the A operand of
+//      the next product as fp16 high part (row r) and low part (row r + 64),
+//      so the weights keep ~22 bits at no extra tensor work; when the running
+//      maximum moved, rows r and r + 64 of O in tensor memory are rescaled;
+//   4. O[128 x 128] += P' V with one tcgen05.mma per 16 tokens.
+// At the end of a stream's pages in this CTA, row r of the result is O's
+// rows r + (r + 64), written with (m, l) as 8-row records for the combine.
+constexpr int kTRows = 64;    // query rows per stream
+constexpr int kTTok = 64;     // tokens per tile
+constexpr int kTThreads = 4 * 32;
+constexpr int kTCtasPerSm = 2;
+constexpr int kTCols = 256;   // tensor memory per CTA: S at column 0, O at column 128
+constexpr int kTQ = 0;                               // Q~ tile: 128 rows x 128 dims fp16
+constexpr int kTK = kTQ + 128 * kD * 2;              // K tile: 64 tokens x 128 dims
+constexpr int kTV = kTK + kTTok * kD * 2;            // V tile (right after K: the two hold O's low rows at the end)
+constexpr int kTP = kTV + kTTok * kD * 2;            // P' tile: 128 rows x 64 tokens
+constexpr int kTX = kTP + 128 * kTTok * 2;           // low-part scores: 64 rows x 64 tokens fp32
+constexpr int kTKN = kTX + kTRows * kTTok * 4;       // K norms of the tile (fp32)
+constexpr int kTVN = kTKN + kTTok * 4;               // V norms
+constexpr int kTScale = kTVN + kTTok * 4;            // per-row prescale
+constexpr int kTRed = kTScale + kTRows * 4;          // row maxima and sums of the two token halves
+constexpr int kTBar = kTRed + 4 * kTRows * 4;        // s_done, pv_done
+constexpr int kTMisc = kTBar + 2 * 8;                // tensor-memory base, abort flag
+constexpr int kTSmemBytes = kTMisc + 16;
+static_assert(kTK % 128 == 0 && kTV % 128 == 0 && kTP % 128 == 0, "UMMA tile alignment");
+
+// shared-memory matrix descriptor, no swizzle (16-byte units)
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo16, uint32_t sbo16) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(lbo16 & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>(sbo16 & 0x3FFFu) << 32) | (1ull << 46);
+}
+// instruction descriptor: f16 A/B, f32 accumulator, M x N, B K- or MN-major
+__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, int b_mn_major) {
+  return (1u << 4) | (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// byte offset of element (row, col) in a no-swizzle canonical tile whose
+// 8-row groups are `group_bytes` apart and whose 8-column chunks are 128 B
+// apart (row = M/N index, col = K index for K-major tiles)
+__device__ __forceinline__ uint32_t canon_off(int row, int col, int group_bytes) {
+  return static_cast<uint32_t>((row >> 3) * group_bytes + (col >> 3) * 128 + (row & 7) * 16 + (col & 7) * 2);
+}
+
+__global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const PartialParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + kTBar);
+  uint64_t *bar_pv = bar_s + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kTMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kTMisc + 4);
+  const int ps = p.page_size;
+
+  for (int e = tid; e < 64 * 32; e += kTThreads) {
+    const int idx = e >> 5;
+    s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kTCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    tc_fence_before();
+  }
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_pv, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int64_t tloc[5];
+  if (warp == 0) {
+    const int64_t pb = pages_before(p.seq_lens, p.B, ps, lane);
+    const int64_t p_rg = static_cast<int64_t>(p.H) * pb;
+    const int64_t total = p_rg * p.RG;
+    const int64_t gs = total * blockIdx.x / p.n_cta;
+    const int64_t ge = total * (blockIdx.x + 1) / p.n_cta;
+    int b = 0;
+    int64_t before = 0, rem = 0, rg = 0;
+    if (gs < ge) {
+      rg = gs / p_rg;
+      rem = gs - rg * p_rg;
+      locate_batch(p.seq_lens, p.B, p.H, ps, rem, lane, b, before);
+    }
+    if (lane == 0) {
+      tloc[0] = gs;
+      tloc[1] = ge;
+      tloc[2] = rg;
+      tloc[3] = b;
+      tloc[4] = rem - before;
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t gs = tloc[0], ge = tloc[1];
+  Walk wk;
+  if (gs < ge) {
+    wk.rg = static_cast<int>(tloc[2]);
+    wk.b = static_cast<int>(tloc[3]);
+    wk.L = p.seq_lens[wk.b];
+    wk.np = pages_of(wk.L, ps);
+    wk.h = static_cast<int>(tloc[4] / wk.np);
+    wk.j = static_cast<int>(tloc[4] - static_cast<int64_t>(wk.h) * wk.np);
+  }
+
+  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+  const int r = tid & 63;        // row (softmax) or token (decode) of this thread
+  const bool lo_half = tid >= 64;
+  float *xchg = reinterpret_cast<float *>(smem + kTX);
+  float *row_scale = reinterpret_cast<float *>(smem + kTScale);
+  float *red_max = reinterpret_cast<float *>(smem + kTRed);  // [2][64]
+  float *red_sum = red_max + 2 * kTRows;                      // [2][64]
+  const uint32_t sQ = smem_addr(smem + kTQ), sK = smem_addr(smem + kTK), sV = smem_addr(smem + kTV),
+                 sP = smem_addr(smem + kTP);
+  constexpr uint32_t kIdescS = umma_idesc(128, kTTok, 0);
+  constexpr uint32_t kIdescPV = umma_idesc(128, kD, 1);
+  float m_run = -INFINITY, l_run = 0.f;
+  int lim = 0;
+  bool row_valid = false, first_pv = true, any_pv = false;
+  uint32_t ph_s = 0, ph_pv = 0;
+  bool ok = true;
+  // Control flow depends on the page walk only, so the four warps meet at
+  // every named barrier even after a bounded wait has given up (`ok` false:
+  // the work is skipped, the barriers are not).
+  for (int64_t g = gs; g < ge; ++g) {
+    const bool seg_start = (g == gs) || (wk.j == 0);
+    const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
+    const int L = wk.L;
+    if (seg_start) {
+      // this stream's 64 rows as Q~: high parts in rows 0..63, low parts in
+      // rows 64..127, each row prescaled by a power of two so that its
+      // largest |q| lands in [2^14, 2^15).  The previous stream's products
+      // have completed (its record was written).
+      const int row = wk.rg * kTRows + r;
+      row_valid = row < p.R;
+      const int qi = row_valid ? row / p.G : 0;
+      const int hq = wk.h * p.G + (row_valid ? row % p.G : 0);
+      const float *qp = p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD;
+      float mx = 0.f;
+      for (int d = 0; d < kD; d += 4) {
+        const float4 v = row_valid ? *reinterpret_cast<const float4 *>(qp + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
+      mx *= p.qfold;
+      int ex = 0;
+      if (mx > 0.f) frexpf(mx, &ex);
+      ex = max(ex, -100);
+      const float up = ldexpf(1.f, 15 - ex) * p.qfold;
+      if (!lo_half) row_scale[r] = ldexpf(1.f, ex - 15);
+      for (int c = 0; c < kD / 8; ++c) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = row_valid ? qp[8 * c + 2 * e] * up : 0.f;
+          const float bb = row_valid ? qp[8 * c + 2 * e + 1] * up : 0.f;
+          const __half ah = __float2half_rn(a), bh = __float2half_rn(bb);
+          w4[e] = lo_half ? pack_half2(a - __half2float(ah), bb - __half2float(bh))
+                          : pack_half2(__half2float(ah), __half2float(bh));
+        }
+        *reinterpret_cast<uint4 *>(smem + kTQ + canon_off(r + (lo_half ? 64 : 0), 8 * c, 2048)) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      lim = row_valid ? (p.causal ? L - p.nq + qi + 1 : L) : 0;
+      m_run = -INFINITY;
+      l_run = 0.f;
+      first_pv = true;
+    }
+    // this page's K (threads 0..63) or V (64..127) codes and norms in global
+    // memory: word w of token t at cw[w * ps + t]
+    int phys = -1;
+    if (wk.j < p.max_pages) phys = p.page_table[static_cast<int64_t>(wk.b) * p.max_pages + wk.j];
+    if (phys < 0 || phys >= p.num_pages) {
+      if (tid == 0) set_status(p.status, ISOQUANT_DEVERR_PAGE_RANGE);
+      phys = 0;
+    }
+    const int64_t blk = (static_cast<int64_t>(phys) * 2 + (lo_half ? 1 : 0)) * p.H + wk.h;
+    const uint32_t *cw = p.codes + blk * kWords * ps;
+    const __half *nw = reinterpret_cast<const __half *>(p.norms) + blk * ps;
+
+    const int ntile = ps / kTTok;
+    for (int ti = 0; ti < ntile; ++ti) {
+      const int t0 = ti * kTTok;
+      if (wk.j * ps + t0 >= L) break;  // past the sequence (uniform)
+      // the previous tile's P.V reads the V and P' tiles and O: the V warps
+      // wait for it here, the K warps before they write P'
+      bool pv_pending = any_pv;
+      if (lo_half && pv_pending) {
+        ok = mbar_wait(bar_pv, ph_pv, p.status, abort_flag) && ok;
+        ok = __all_sync(0xffffffffu, ok);
+        pv_pending = false;
+        tc_fence_after();
+      }
+      if (any_pv) ph_pv ^= 1u;
+      any_pv = false;
+      // ---- 1. decode token t0 + r of K (threads 0..63) or V (64..127)
+      {
+        const int t = t0 + r;
+        uint32_t x[kWords];
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) x[w] = __ldg(cw + w * ps + t);
+        const float nrm = __half2float(nw[t]);
+        uint32_t out[64];
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) {
+#pragma unroll
+          for (int k = 0; k < 5; ++k)
+            if (w < 12 || k < 4) out[5 * w + k] = lut_at((((x[w] >> (6 * k)) & 63u) << 7) | lane4);
+        }
+        uint8_t *tile = smem + (lo_half ? kTV : kTK);
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          *reinterpret_cast<uint4 *>(tile + canon_off(r, 8 * c, 2048)) =
+              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+        reinterpret_cast<float *>(smem + (lo_half ? kTVN : kTKN))[r] = nrm;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      named_bar_sync(1, kTThreads);
+      // ---- 2. S = Q~ K^T
+      if (tid == 0 && ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kc2 = 0; kc2 < kD / 16; ++kc2)
+          umma_f16(tmem, umma_desc(sQ + kc2 * 256, 8, 128), umma_desc(sK + kc2 * 256, 8, 128), kIdescS,
+                   kc2 > 0 ? 1u : 0u);
+        umma_commit(bar_s);
+      }
+      ok = mbar_wait(bar_s, ph_s, p.status, abort_flag) && ok;
+      ok = __all_sync(0xffffffffu, ok);
+      ph_s ^= 1u;
+      tc_fence_after();
+      // ---- 3. softmax: row r's tokens 0..31 by thread r (which holds the
+      // high-part scores, lanes 0..63), tokens 32..63 by thread r + 64 (low
+      // parts, lanes 64..127); each half sends the other the half it needs
+      float sv[64];
+      {
+        const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+        float tmp[32];
+        tmem_ld32(ta, tmp);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[i] = tmp[i];
+        tmem_ld32(ta + 32, tmp);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[32 + i] = tmp[i];
+      }
+      // xchg: [half][4-column group][row][4]; half 0 = high parts of tokens
+      // 32..63 (for the low warps), half 1 = low parts of tokens 0..31
+      const int own = lo_half ? 32 : 0;    // tokens this thread finishes
+      {
+        float *dst = xchg + (lo_half ? 1 : 0) * (32 * kTRows);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4 *>(dst + (i * kTRows + 4 * r)) =
+              lo_half ? make_float4(sv[i], sv[i + 1], sv[i + 2], sv[i + 3])
+                      : make_float4(sv[32 + i], sv[33 + i], sv[34 + i], sv[35 + i]);
+      }
+      tc_fence_before();
+      named_bar_sync(1, kTThreads);
+      float mx = -INFINITY;
+      {
+        const float *kn_t = reinterpret_cast<const float *>(smem + kTKN) + own;
+        const float *src = xchg + (lo_half ? 0 : 1) * (32 * kTRows);
+        const float rs = row_scale[r];
+        const int pos0 = wk.j * ps + t0 + own;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 o4 = *reinterpret_cast<const float4 *>(src + (i * kTRows + 4 * r));
+          const float4 kn4 = *reinterpret_cast<const float4 *>(kn_t + i);
+          const float x4[4] = {o4.x, o4.y, o4.z, o4.w}, k4[4] = {kn4.x, kn4.y, kn4.z, kn4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float sc = ((lo_half ? sv[32 + i + e] : sv[i + e]) + x4[e]) * rs * k4[e];
+            if (!row_valid || pos0 + i + e >= lim) sc = -INFINITY;
+            sv[i + e] = sc;  // compacted into sv[0..31]
+            mx = fmaxf(mx, sc);
+          }
+        }
+      }
+      red_max[(lo_half ? kTRows : 0) + r] = mx;
+      named_bar_sync(1, kTThreads);
+      // P' and O may still be read by the previous tile's P.V
+      if (!lo_half && pv_pending) {
+        ok = mbar_wait(bar_pv, ph_pv ^ 1u, p.status, abort_flag) && ok;
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+      }
+      const float m_new = fmaxf(m_run, fmaxf(red_max[r], red_max[kTRows + r]));
+      const float corr = (m_run == -INFINITY || m_new == m_run) ? 1.f : ex2(m_run - m_new);
+      {
+        const float *vn_t = reinterpret_cast<const float *>(smem + kTVN) + own;
+        const float mm = m_new == -INFINITY ? 0.f : m_new;
+        float psum = 0.f;
+        uint32_t pk[16], pl[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ex2(sv[i] - mm), p1 = ex2(sv[i + 1] - mm);
+          psum += p0 + p1;
+          // masked slots may hold stale norms: select, do not multiply
+          const float w0 = p0 > 0.f ? p0 * vn_t[i] : 0.f, w1 = p1 > 0.f ? p1 * vn_t[i + 1] : 0.f;
+          const __half h0 = __float2half_rn(w0), h1 = __float2half_rn(w1);
+          pk[i >> 1] = pack_half2(__half2float(h0), __half2float(h1));
+          pl[i >> 1] = pack_half2(w0 - __half2float(h0), w1 - __half2float(h1));
+        }
+        // p n_v: high part in row r, low part in row r + 64 of the A tile
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          *reinterpret_cast<uint4 *>(smem + kTP + canon_off(r, own + 8 * c, 1024)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          *reinterpret_cast<uint4 *>(smem + kTP + canon_off(r + 64, own + 8 * c, 1024)) =
+              make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+        }
+        red_sum[(lo_half ? kTRows : 0) + r] = psum;
+      }
+      named_bar_sync(1, kTThreads);
+      // both threads of a row keep the same (m, l)
+      l_run = l_run * corr + red_sum[r] + red_sum[kTRows + r];
+      m_run = m_new;
+      // rescale rows r (warps 0-1) and r + 64 (warps 2-3) of O when the row's
+      // maximum moved (each warp loads and stores together)
+      if (!first_pv && __any_sync(0xffffffffu, corr != 1.f)) {
+        const uint32_t to = tmem + 128 + (static_cast<uint32_t>(32 * warp) << 16);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float ov[32];
+          tmem_ld32(to + 32 * c, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= corr;
+          tmem_st32(to + 32 * c, ov);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      named_bar_sync(1, kTThreads);
+      // ---- 4. O += P' V
+      if (tid == 0 && ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kc2 = 0; kc2 < kTTok / 16; ++kc2)
+          umma_f16(tmem + 128, umma_desc(sP + kc2 * 256, 8, 64), umma_desc(sV + kc2 * 4096, 128, 8), kIdescPV,
+                   (first_pv && kc2 == 0) ? 0u : 1u);
+        umma_commit(bar_pv);
+      }
+      first_pv = false;
+      any_pv = true;
+    }
+    if (seg_end) {
+      // ---- the stream's record: wait for the last P.V, then row r of the
+      // result is O's rows r + (r + 64); the low rows go through the K and V
+      // tiles (every product has completed)
+      if (any_pv) {
+        ok = mbar_wait(bar_pv, ph_pv, p.status, abort_flag) && ok;
+        ok = __all_sync(0xffffffffu, ok);
+        ph_pv ^= 1u;
+        any_pv = false;
+      }
+      tc_fence_after();
+      float *olo = reinterpret_cast<float *>(smem + kTK);
+      const uint32_t to = tmem + 128 + (static_cast<uint32_t>(32 * warp) << 16);
+      if (lo_half) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float ov[32];
+          tmem_ld32(to + 32 * c, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) olo[(32 * c + i) * kTRows + r] = ov[i];
+        }
+      }
+      named_bar_sync(1, kTThreads);
+      if (!lo_half) {
+        const int row = wk.rg * kTRows + r;
+        const int64_t stream = (static_cast<int64_t>(wk.rg) * p.B + wk.b) * p.H + wk.h;
+        float *rec =
+            p.records + ((blockIdx.x + stream) * (kTRows / 8) + (r >> 3)) * static_cast<int64_t>(kRecordFloats);
+        const int rr = r & 7;
+        const bool have = !first_pv;
+        if (row < p.R) {
+          rec[2 * rr] = have ? m_run : -INFINITY;
+          rec[2 * rr + 1] = have ? l_run : 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float ov[32];
+          tmem_ld32(to + 32 * c, ov);
+          if (row < p.R && have) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4 *>(rec + 16 + rr * kD + 32 * c + i) =
+                  make_float4(ov[i] + olo[(32 * c + i) * kTRows + r], ov[i + 1] + olo[(32 * c + i + 1) * kTRows + r],
+                              ov[i + 2] + olo[(32 * c + i + 2) * kTRows + r], ov[i + 3] + olo[(32 * c + i + 3) * kTRows + r]);
+          }
+        }
+      }
+      tc_fence_before();
+      named_bar_sync(1, kTThreads);
+    }
+    if (g + 1 < ge) wk.advance(p.seq_lens, p.B, p.H, ps);
+  }
+  // the last P.V must finish before tensor memory is released
+  if (any_pv) mbar_wait(bar_pv, ph_pv, p.status, nullptr);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTCols));
+  }
+}
+
 // ------------------------------------------------------------ combine kernel
 
 // Small blocks, so that they fit beside partial-kernel CTAs as soon as any
@@ -845,7 +1321,8 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
   const int i = static_cast<int>(bi % static_cast<uint32_t>(p.nq));
   const int b = static_cast<int>(bi / static_cast<uint32_t>(p.nq));
   const int h = hq / p.G, g = hq % p.G;
-  const int r = i * p.G + g, rg = r >> 3, rr = r & 7;
+  // stream rg holds rows rg * rps .. ; record `sub` of a CTA holds 8 of them
+  const int r = i * p.G + g, rg = r / p.rps, sub = (r % p.rps) >> 3, rr = r & 7;
   const int ps = p.page_size;
   float *dst = p.out + static_cast<int64_t>(row_id) * kD + 4 * lane;
 
@@ -863,25 +1340,52 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
   const int64_t pair = (static_cast<int64_t>(rg) * p.B + b) * p.H + h;
   const int rows[1] = {rr};
   float *const dsts[1] = {dst};
-  merge_rows<1>(p.records, pair, c_lo, c_hi, N, total, rows, dsts, p.params[h], lane);
+  merge_rows<1>(p.records, pair, p.rps >> 3, sub, c_lo, c_hi, N, total, rows, dsts, p.params[h], lane);
 }
 
 }  // namespace
 
 int attend_ctas_per_sm() { return kCtasPerSm; }
 
-size_t attend_workspace_bytes(const AttendShape &s) {
+namespace {
+// The tcgen05 kernel serves 64 or more query rows per KV head (pages of at
+// least 64 tokens); it keeps 8 records per (CTA, stream of 64 rows).
+int tile_streams(const AttendShape &s) { return (s.rows + kTRows - 1) / kTRows; }
+size_t tile_slots(const AttendShape &s, int n_cta) {
+  return (static_cast<size_t>(n_cta) +
+          static_cast<size_t>(tile_streams(s)) * static_cast<size_t>(s.batch) * s.kv_heads) *
+         (kTRows / 8);
+}
+bool use_tiles(const isoquant_ctx *ctx, const AttendShape &s, size_t ws_bytes) {
+  return s.rows >= kTRows && s.page_size >= kTTok &&
+         kWsHeader + tile_slots(s, ctx->num_sms * kTCtasPerSm) * kRecordFloats * sizeof(float) <= ws_bytes;
+}
+}  // namespace
+
+size_t attend_workspace_min_bytes(const AttendShape &s) {
   return kWsHeader + s.slots * kRecordFloats * sizeof(float);
+}
+
+size_t attend_workspace_bytes(const AttendShape &s) {
+  // room for the tcgen05 kernel's records too, when the shape can use it
+  const size_t tiles = s.rows >= kTRows ? tile_slots(s, s.n_cta / kCtasPerSm * kTCtasPerSm) : 0;
+  return kWsHeader + (s.slots > tiles ? s.slots : tiles) * kRecordFloats * sizeof(float);
 }
 
 cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache, const AttendShape &s,
                                   const float *q_rot, const int32_t *page_table, int max_pages,
-                                  const int32_t *seq_lens, float scale, void *ws, cudaStream_t stream) {
+                                  const int32_t *seq_lens, float scale, void *ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
   static int configured_device = -1;
   if (configured_device != ctx->device) {
     cudaError_t e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_attend_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_attend_tiles, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured_device = ctx->device;
@@ -908,11 +1412,16 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
   p.records = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
   p.status = ctx->status;
   p.n_cta = s.n_cta;
+  if (use_tiles(ctx, s, ws_bytes)) {
+    p.RG = tile_streams(s);
+    p.n_cta = ctx->num_sms * kTCtasPerSm;
+    return launch_pdl(k_attend_tiles, dim3(p.n_cta), dim3(kTThreads), kTSmemBytes, stream, p);
+  }
   return launch_pdl(k_attend_partial, dim3(s.n_cta), dim3(kThreads), kSmemBytes, stream, p);
 }
 
 cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s, const int32_t *seq_lens,
-                                  const void *ws, float *out, cudaStream_t stream) {
+                                  const void *ws, size_t ws_bytes, float *out, cudaStream_t stream) {
   CombineParams p{};
   p.records = reinterpret_cast<const float *>(static_cast<const char *>(ws) + kWsHeader);
   p.params = ctx->params;
@@ -926,6 +1435,12 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
   p.RG = s.row_groups;
   p.page_size = s.page_size;
   p.n_cta = s.n_cta;
+  p.rps = 8;
+  if (use_tiles(ctx, s, ws_bytes)) {
+    p.RG = tile_streams(s);
+    p.n_cta = ctx->num_sms * kTCtasPerSm;
+    p.rps = kTRows;
+  }
   const int64_t rows = static_cast<int64_t>(s.batch) * s.nq * s.q_heads;
   const int64_t blocks = (rows * 32 + kCombineThreads - 1) / kCombineThreads;
   if (blocks == 0) return cudaSuccess;

@@ -9,7 +9,7 @@
 // partial records of the split-context attention live in a fixed array
 // compiled into the library.
 //
-// The array is a file-scope __device__ variable of kScratchBytes (4 MiB):
+// The array is a file-scope __device__ variable of kScratchBytes (8 MiB):
 // every GPU that loads the library holds it until the process exits.  In
 // host code its name is only a host-side stand-in, so the device address is
 // looked up with cudaGetSymbolAddress, once per device, with that device
@@ -28,7 +28,7 @@
 namespace isoquant {
 namespace {
 
-constexpr size_t kScratchBytes = size_t(4) << 20;
+constexpr size_t kScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -61,9 +61,10 @@ extern "C" int isoquant_attend_decode_static(isoquant_ctx *ctx, const isoquant_c
   ctx->last_launches = 0;
   if (num_q_heads < 1 || nq < 1 || batch < 0 || num_q_heads % ctx->num_kv_heads != 0)
     return ISOQUANT_ERR_INVALID_ARG;
-  // the shape's record count must fit the fixed array
+  // the shape's records must fit the fixed array (the mma.sync kernel's at
+  // least; the tcgen05 kernel is used when its records fit too)
   size_t need = 0;
-  int st = isoquant_workspace_size(ctx, batch, nq, num_q_heads, &need);
+  int st = attend_workspace_min(ctx, batch, nq, num_q_heads, &need);
   if (st != ISOQUANT_OK) return st;
   if (need > kScratchBytes) return ISOQUANT_ERR_WORKSPACE;
   if (batch == 0) return ISOQUANT_OK;

@@ -69,14 +69,18 @@ struct AttendShape {
 constexpr size_t kWsHeader = 256;
 constexpr size_t kRecordFloats = 8 * 2 + 8 * kD;  // (m,l) x 8 rows, o[8][128]
 
+// Workspace sizes: the full size (room for either attention kernel's
+// records) and the minimum any call accepts (the mma.sync kernel's).
 size_t attend_workspace_bytes(const AttendShape &s);
+size_t attend_workspace_min_bytes(const AttendShape &s);
+int attend_workspace_min(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, size_t *bytes);
 int attend_ctas_per_sm();
 cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache,
                                   const AttendShape &s, const float *q_rot, const int32_t *page_table,
                                   int max_pages, const int32_t *seq_lens, float scale, void *ws,
-                                  cudaStream_t stream);
+                                  size_t ws_bytes, cudaStream_t stream);
 cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
-                                  const int32_t *seq_lens, const void *ws, float *out,
+                                  const int32_t *seq_lens, const void *ws, size_t ws_bytes, float *out,
                                   cudaStream_t stream);
 
 // ------------------------------------------------------------ launch chain

@@ -382,3 +382,49 @@ def test_decode_step_matches_separate_calls_and_oracle(cuda_lib):
         assert torch.equal(sa.cache.codes, sb.cache.codes)
         b = sb.B - 1
         check_pair(sb, b, sb.H - 1, q.float().cpu(), out_b.cpu())
+
+
+@pytest.mark.parametrize("case", ["verify", "ragged_ps64", "rows96_ps128", "short"])
+def test_tcgen05_rows_kernel_matches_mma_path(cuda_lib, case):
+    """64 or more query rows per KV head run on the tcgen05 kernel (one
+    decode of each KV tile for 64 rows, products in tensor memory) when the
+    workspace has its records; a workspace of the minimum size runs the
+    mma.sync kernel.  Both match the oracle and each other."""
+    from compressed_space_decode_b200.synthetic import Workload
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    if case == "verify":
+        wl = csd.synthetic.workloads(small=True)["verify_b8_nq16_q32_kv8_L16384"]
+    elif case == "ragged_ps64":
+        # 16 positions x 4 heads = 64 rows, causal, ragged lengths, 64-token pages
+        wl = Workload(case, 5, 16, 4, [3000, 1, 700, 64, 1234], nq=16, page_size=64, causal=True, seed=31)
+    elif case == "rows96_ps128":
+        # 3 positions x 32 heads = 96 rows: a full stream and one of 32 rows
+        wl = Workload(case, 3, 32, 1, [2000, 517, 130], nq=3, page_size=128, causal=True, seed=32)
+    else:
+        wl = Workload(case, 4, 16, 2, [17, 64, 65, 200], nq=16, page_size=256, causal=True, seed=33)
+    st = DecodeState(wl)
+    q = st.queries(0)
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    csd.isoquant_rotate_q(st.ctx, q.reshape(-1, st.Hq, D), q_rot.view(-1, st.Hq, D))
+    outs = []
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pairs = ((wl.nq * st.G + 7) // 8) * st.B * st.H
+    ws_min = (256 + (2 * n_sms + pairs) * 4160) // 4
+    for ws in (_ws(csd, st), torch.empty(ws_min, dtype=torch.int32, device="cuda").fill_(0x7FC00000)):
+        out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+        csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, ws, out,
+                                   causal=wl.causal)
+        torch.cuda.synchronize()
+        assert csd.isoquant_get_status(st.ctx) == 0
+        outs.append(out.cpu())
+    tiles, mma = outs
+    assert torch.isfinite(tiles).all()
+    err = rowwise_rel_err(tiles.numpy(), mma.numpy())
+    # each path is within ATTN_TOL of the exact result
+    assert err.max() <= 2 * ATTN_TOL, err.max()
+    qc = q.float().cpu()
+    for b in range(st.B):
+        if st.seq_lens[b] == 0:
+            continue
+        check_pair(st, b, (b * 3) % st.H, qc, tiles)
