@@ -94,6 +94,7 @@ struct PartialParams {
   float *records;
   uint32_t *status;
   int n_cta;
+  int64_t *prefix;  // tcgen05 kernels: pages before each (stream, sequence) unit
 };
 
 struct CombineParams {
@@ -102,7 +103,8 @@ struct CombineParams {
   const int32_t *seq_lens;
   float *out;
   int B, nq, Hq, H, G, RG, page_size, n_cta;
-  int rps;  // query rows per stream: 8 (mma.sync kernel) or 64 (tcgen05 kernel)
+  int rps;  // query rows per stream: 8 (mma.sync kernel), 64 or 128 (tcgen05 kernels)
+  const int64_t *prefix;  // null for the mma.sync kernel
 };
 
 // ------------------------------------------------------------------ PTX
@@ -126,12 +128,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: gives up after kSpinLimit polls, raising the timeout bit.
+// It spins (try_wait itself suspends briefly) for the first kSpin polls and
+// then backs off with __nanosleep.  A sleeping waiter wakes late, which costs
+// a hand-off between warp-specialised roles hundreds of cycles (those spin
+// long); where many threads of a CTA wait together, spinning takes issue
+// slots from the CTA beside it (those back off early).
+template <uint32_t kSpin = 64>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
                                           volatile int *abort_flag) {
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort_flag != nullptr && *abort_flag) return false;
-    if (i > 64) __nanosleep(64);
+    if (i > kSpin) __nanosleep(64);
   }
   set_status(status, ISOQUANT_DEVERR_WAIT_TIMEOUT);
   if (abort_flag != nullptr) *abort_flag = 1;
@@ -227,6 +235,109 @@ struct Walk {
     } while (np == 0);
   }
 };
+
+// ------------------------------------------------------------ unit walk
+// The tcgen05 kernels split pages of (stream, sequence, KV head), a stream
+// being `rps` consecutive query rows of a KV head.  Under causal masking
+// stream rg of sequence b sees only the first L - nq + q_last + 1 tokens
+// (q_last = its last query position), so it walks only the pages holding
+// them: unit u = rg * B + b carries H * pages_of(horizon) pages.  Causal
+// prefill thus costs the triangle, not the square.
+__device__ __forceinline__ int unit_horizon(const PartialParams &p, int rps, int rg, int b) {
+  const int L = p.seq_lens[b];
+  if (!p.causal) return max(L, 0);
+  const int q_last = min(p.nq - 1, (rg * rps + rps - 1) / p.G);
+  return max(0, min(L, L - p.nq + q_last + 1));
+}
+// (units and the pages of one unit are counted in 32 bits: the host keeps
+// streams * batch and max_pages * kv_heads below 2^31)
+__device__ __forceinline__ int64_t unit_pages(const PartialParams &p, int rps, int u) {
+  const int rg = u / p.B, b = u - rg * p.B;
+  return static_cast<int64_t>(p.H) * pages_of(unit_horizon(p, rps, rg, b), p.page_size);
+}
+
+struct UWalk {
+  int u, rg, b, h, j, np, hz;
+  __device__ void set(const PartialParams &p, int rps, int u_) {
+    u = u_;
+    rg = u / p.B;
+    b = u - rg * p.B;
+    hz = unit_horizon(p, rps, rg, b);
+    np = pages_of(hz, p.page_size);
+  }
+  __device__ void start(const PartialParams &p, int rps, int u_, int off) {
+    set(p, rps, u_);
+    h = off / np;
+    j = off - h * np;
+  }
+  __device__ void advance(const PartialParams &p, int rps) {
+    if (++j < np) return;
+    j = 0;
+    if (++h < p.H) return;
+    h = 0;
+    do set(p, rps, u + 1); while (np == 0);
+  }
+  // tokens of the current page this stream sees, and its 64-token tiles
+  __device__ int page_tokens(int ps) const { return min(ps, hz - j * ps); }
+};
+
+// Every thread of the CTA: sum the pages of all units (each thread a slice
+// of units, then a scan over the slices), take this CTA's range [gs, ge) of
+// the total and find the unit and page offset where it starts:
+// loc = {gs, ge, unit, offset}.  CTA 0 also writes prefix[u] (pages before
+// unit u) and prefix[U] = total for the combine kernel.  Ends with
+// __syncthreads.
+template <int NT>
+__device__ void tile_locate(const PartialParams &p, int rps, int64_t *scratch, int64_t *loc) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int U = p.RG * p.B;
+  const int u0 = static_cast<int>(static_cast<int64_t>(U) * tid / NT),
+            u1 = static_cast<int>(static_cast<int64_t>(U) * (tid + 1) / NT);
+  int64_t mine = 0;
+  for (int u = u0; u < u1; ++u) mine += unit_pages(p, rps, u);
+  int64_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int64_t before = 0, total = 0;
+  for (int w = 0; w < NT / 32; ++w) {
+    if (w < warp) before += scratch[w];
+    total += scratch[w];
+  }
+  const int64_t excl = before + incl - mine;
+  const int64_t gs = total * blockIdx.x / p.n_cta, ge = total * (blockIdx.x + 1) / p.n_cta;
+  if (blockIdx.x == 0 && p.prefix != nullptr) {
+    int64_t run = excl;
+    for (int u = u0; u < u1; ++u) {
+      p.prefix[u] = run;
+      run += unit_pages(p, rps, u);
+    }
+    if (tid == NT - 1) p.prefix[U] = total;
+  }
+  if (gs < ge && excl <= gs && gs < excl + mine) {
+    int64_t run = excl;
+    for (int u = u0; u < u1; ++u) {
+      const int64_t n = unit_pages(p, rps, u);
+      if (gs < run + n) {
+        loc[0] = gs;
+        loc[1] = ge;
+        loc[2] = u;
+        loc[3] = gs - run;
+        break;
+      }
+      run += n;
+    }
+  }
+  if (tid == 0 && !(gs < ge)) {
+    loc[0] = gs;
+    loc[1] = ge;
+  }
+  __syncthreads();
+}
 
 // ------------------------------------------------------------ pair table
 // s_lut[idx * 32 + lane] = half2(C[idx & 7], C[idx >> 3]): one copy per lane
@@ -888,16 +999,42 @@ __host__ __device__ constexpr uint32_t umma_idesc(int m, int n, int b_mn_major) 
   return (1u << 4) | (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
 }
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// One tensor-core product D (+)= A B (kind::f16, fp32 accumulator in tensor
+// memory, A and B in shared memory), issued by the threads with `issue` set
+// (one thread per CTA)
+__device__ __forceinline__ void umma_f16_by(bool issue, uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%6, %7, %8, %9}, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(static_cast<uint32_t>(issue)), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
       : "memory");
 }
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
-               : "memory");
+// the same with A in tensor memory (row m = lane m, column c = the packed
+// fp16 pair k = 2c, 2c + 1 of the 16-wide K slice starting at a_tmem)
+__device__ __forceinline__ void umma_ts_by(bool issue, uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                           uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%6, %7, %8, %9}, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(static_cast<uint32_t>(issue)), "r"(0u), "r"(0u), "r"(0u),
+      "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_by(bool issue, uint64_t *bar) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+      "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(smem_addr(bar)),
+      "r"(static_cast<uint32_t>(issue))
+      : "memory");
 }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -965,41 +1102,13 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
   }
   pdl_trigger();
   pdl_wait();
-  __shared__ int64_t tloc[5];
-  if (warp == 0) {
-    const int64_t pb = pages_before(p.seq_lens, p.B, ps, lane);
-    const int64_t p_rg = static_cast<int64_t>(p.H) * pb;
-    const int64_t total = p_rg * p.RG;
-    const int64_t gs = total * blockIdx.x / p.n_cta;
-    const int64_t ge = total * (blockIdx.x + 1) / p.n_cta;
-    int b = 0;
-    int64_t before = 0, rem = 0, rg = 0;
-    if (gs < ge) {
-      rg = gs / p_rg;
-      rem = gs - rg * p_rg;
-      locate_batch(p.seq_lens, p.B, p.H, ps, rem, lane, b, before);
-    }
-    if (lane == 0) {
-      tloc[0] = gs;
-      tloc[1] = ge;
-      tloc[2] = rg;
-      tloc[3] = b;
-      tloc[4] = rem - before;
-    }
-  }
-  __syncthreads();
+  __shared__ int64_t tloc[4 + kTThreads / 32];
+  tile_locate<kTThreads>(p, kTRows, tloc + 4, tloc);
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t gs = tloc[0], ge = tloc[1];
-  Walk wk;
-  if (gs < ge) {
-    wk.rg = static_cast<int>(tloc[2]);
-    wk.b = static_cast<int>(tloc[3]);
-    wk.L = p.seq_lens[wk.b];
-    wk.np = pages_of(wk.L, ps);
-    wk.h = static_cast<int>(tloc[4] / wk.np);
-    wk.j = static_cast<int>(tloc[4] - static_cast<int64_t>(wk.h) * wk.np);
-  }
+  UWalk wk;
+  if (gs < ge) wk.start(p, kTRows, static_cast<int>(tloc[2]), static_cast<int>(tloc[3]));
 
   const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
   const int r = tid & 63;        // row (softmax) or token (decode) of this thread
@@ -1008,8 +1117,9 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
   float *row_scale = reinterpret_cast<float *>(smem + kTScale);
   float *red_max = reinterpret_cast<float *>(smem + kTRed);  // [2][64]
   float *red_sum = red_max + 2 * kTRows;                      // [2][64]
-  const uint32_t sQ = smem_addr(smem + kTQ), sK = smem_addr(smem + kTK), sV = smem_addr(smem + kTV),
-                 sP = smem_addr(smem + kTP);
+  // descriptors built once (per product only constant start offsets are added)
+  const uint64_t dQ = umma_desc(smem_addr(smem + kTQ), 8, 128), dK = umma_desc(smem_addr(smem + kTK), 8, 128),
+                 dV = umma_desc(smem_addr(smem + kTV), 128, 8), dP = umma_desc(smem_addr(smem + kTP), 8, 64);
   constexpr uint32_t kIdescS = umma_idesc(128, kTTok, 0);
   constexpr uint32_t kIdescPV = umma_idesc(128, kD, 1);
   float m_run = -INFINITY, l_run = 0.f;
@@ -1023,7 +1133,7 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
   for (int64_t g = gs; g < ge; ++g) {
     const bool seg_start = (g == gs) || (wk.j == 0);
     const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
-    const int L = wk.L;
+    const int L = p.seq_lens[wk.b];
     if (seg_start) {
       // this stream's 64 rows as Q~: high parts in rows 0..63, low parts in
       // rows 64..127, each row prescaled by a power of two so that its
@@ -1075,10 +1185,9 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
     const uint32_t *cw = p.codes + blk * kWords * ps;
     const __half *nw = reinterpret_cast<const __half *>(p.norms) + blk * ps;
 
-    const int ntile = ps / kTTok;
+    const int ntile = (wk.page_tokens(ps) + kTTok - 1) / kTTok;  // tiles within the stream's horizon
     for (int ti = 0; ti < ntile; ++ti) {
       const int t0 = ti * kTTok;
-      if (wk.j * ps + t0 >= L) break;  // past the sequence (uniform)
       // the previous tile's P.V reads the V and P' tiles and O: the V warps
       // wait for it here, the K warps before they write P'
       bool pv_pending = any_pv;
@@ -1118,10 +1227,8 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
       if (tid == 0 && ok) {
         tc_fence_after();
 #pragma unroll
-        for (int kc2 = 0; kc2 < kD / 16; ++kc2)
-          umma_f16(tmem, umma_desc(sQ + kc2 * 256, 8, 128), umma_desc(sK + kc2 * 256, 8, 128), kIdescS,
-                   kc2 > 0 ? 1u : 0u);
-        umma_commit(bar_s);
+        for (int kc2 = 0; kc2 < kD / 16; ++kc2) umma_f16_by(true, tmem, dQ + kc2 * 16, dK + kc2 * 16, kIdescS, kc2 > 0 ? 1u : 0u);
+        umma_commit_by(true, bar_s);
       }
       ok = mbar_wait(bar_s, ph_s, p.status, abort_flag) && ok;
       ok = __all_sync(0xffffffffu, ok);
@@ -1234,9 +1341,8 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
         tc_fence_after();
 #pragma unroll
         for (int kc2 = 0; kc2 < kTTok / 16; ++kc2)
-          umma_f16(tmem + 128, umma_desc(sP + kc2 * 256, 8, 64), umma_desc(sV + kc2 * 4096, 128, 8), kIdescPV,
-                   (first_pv && kc2 == 0) ? 0u : 1u);
-        umma_commit(bar_pv);
+          umma_f16_by(true, tmem + 128, dP + kc2 * 16, dV + kc2 * 256, kIdescPV, (first_pv && kc2 == 0) ? 0u : 1u);
+        umma_commit_by(true, bar_pv);
       }
       first_pv = false;
       any_pv = true;
@@ -1291,7 +1397,7 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
       tc_fence_before();
       named_bar_sync(1, kTThreads);
     }
-    if (g + 1 < ge) wk.advance(p.seq_lens, p.B, p.H, ps);
+    if (g + 1 < ge) wk.advance(p, kTRows);
   }
   // the last P.V must finish before tensor memory is released
   if (any_pv) mbar_wait(bar_pv, ph_pv, p.status, nullptr);
@@ -1300,6 +1406,453 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTCols));
+  }
+}
+
+// ------------------------------------------------------------ tcgen05 kernel, 128-row streams
+// k_attend_wide: 128 or more query rows per KV head (causal prefill, long
+// verification chunks).  One CTA per SM, warp-specialised, streams of 128
+// query rows, 64-token tiles, the same unit walk as above:
+//   * the decoder warps (groups of 4 after the softmax warps) take the
+//     CTA's tiles in turn into stage T % 2, each thread one token of K
+//     (threads 0..63 of the group) or V (64..127), as in k_attend_tiles.
+//     Two groups in flight hide the load latency of the code words;
+//   * the last warp, one thread, issues the tensor-core products: S_T = Q~ K_T^T
+//     into one of two score buffers in tensor memory (16 MMAs: the queries'
+//     fp16 high parts, then their low parts, accumulated), and, once the
+//     softmax of tile T - 1 is in shared memory, O += P'_{T-1} V_{T-1}
+//     (8 MMAs: the weights' high parts, then their low parts).  S_{T+1} is
+//     issued before P.V_T, so the tensor pipe computes the next scores while
+//     the softmax warps work;
+//   * warps 0..7 run the online softmax: two threads per row r (tensor-
+//     memory lane r of S and O), one per half of the tile's tokens, which
+//     exchange their maxima through shared memory (one warp per row would
+//     leave each SM sub-partition a single latency-bound softmax warp):
+//     scores times the K norms and the row's prescale, causal and length
+//     limits, running max and per-half sums, p * n_v split into fp16
+//     high and low parts (the A operands of P.V, double-buffered so that
+//     they are written while the previous P.V runs), and the rescale of its
+//     O row when the row's maximum moved (after the previous P.V completed).
+//     At a stream's last tile in this CTA it writes the row's (m, l, o)
+//     record for the combine.
+// Hand-offs are mbarriers: kv_full[s] (decoders -> MMA), kv_free[s] (P.V of
+// the tile that used stage s completed -> decoders), s_full[b] (S in
+// buffer b -> softmax), s_free[b] (softmax has read it -> MMA), p_full
+// (P' written -> MMA), pv_done (P.V completed -> softmax) and q_full (the
+// stream's Q~ written -> MMA).  Every wait is bounded; after one expires all
+// roles skip their work and fall through to the end.
+constexpr int kWRows = 128;
+constexpr int kWTok = 64;
+constexpr int kWSoftWarps = 8;  // two warpgroups: each row's tokens split in halves
+#ifndef ISOQUANT_WIDE_DEC_GROUPS
+#define ISOQUANT_WIDE_DEC_GROUPS 1
+#endif
+constexpr int kWDecGroups = ISOQUANT_WIDE_DEC_GROUPS;  // decoder groups of 4 warps, taking tiles in turn
+constexpr int kWDecWarps = 4 * kWDecGroups;
+constexpr int kWMmaWarp = kWSoftWarps + kWDecWarps;
+constexpr int kWThreads = (kWMmaWarp + 1) * 32;
+// Tensor memory (512 columns, one CTA per SM): S buffers 0 and 1, O, then
+// the A operands of both products, fp16 pairs packed per 32-bit column
+// (row = lane): Q~ high and low parts (64 columns each) and two buffers of
+// P' high and low parts (32 columns each).  With the A operands there, the
+// products read only K and V from shared memory: fed from shared memory,
+// an M = 128 product with N <= 128 is bound by shared-memory bandwidth.
+constexpr int kWCols = 512;
+constexpr uint32_t kWColS = 0, kWColO = 128, kWColQh = 256, kWColQl = 320, kWColP = 384;  // P buffer b: +64 b, low +32
+#ifndef ISOQUANT_WIDE_STAGES
+#define ISOQUANT_WIDE_STAGES 4
+#endif
+constexpr int kWStages = ISOQUANT_WIDE_STAGES;        // K/V tile ring
+static_assert((kWStages & (kWStages - 1)) == 0 && kWStages >= 2, "power-of-two ring");
+constexpr int kWStageBytes = kWTok * kD * 2;          // one 64-token tile of K or V, fp16
+constexpr int kWK = 0;                                // kWStages K tiles
+constexpr int kWV = kWK + kWStages * kWStageBytes;    // kWStages V tiles
+constexpr int kWKN = kWV + kWStages * kWStageBytes;   // K norms, kWStages x 64 fp32
+constexpr int kWVN = kWKN + kWStages * kWTok * 4;     // V norms
+constexpr int kWRed = kWVN + kWStages * kWTok * 4;    // row maxima [2][2][128] and sums [2][128]
+constexpr int kWBar = kWRed + 6 * kWRows * 4;         // 2 kWStages + 8 mbarriers
+constexpr int kWMisc = kWBar + (2 * kWStages + 8) * 8;  // tensor-memory base, abort flag, MMA-issued flag
+constexpr int kWLoc = kWMisc + 16;                    // walk start + scan scratch
+constexpr int kWSmemBytes = kWLoc + (4 + kWThreads / 32) * 8;
+static_assert(kWK % 128 == 0 && kWV % 128 == 0, "UMMA tile alignment");
+static_assert(kWBar % 8 == 0 && kWLoc % 8 == 0, "barrier alignment");
+
+// the walk's tiles: for each page of [gs, ge), its 64-token tiles within the
+// stream's horizon; f(wk, t0, first, last) with first / last = the stream's
+// first / last tile in this CTA.  Every role runs the same sequence.
+template <typename F>
+__device__ __forceinline__ void for_each_tile(const PartialParams &p, int64_t gs, int64_t ge, int u0, int off0,
+                                              F &&f) {
+  if (!(gs < ge)) return;
+  const int ps = p.page_size;
+  UWalk wk;
+  wk.start(p, kWRows, u0, off0);
+  for (int64_t g = gs; g < ge; ++g) {
+    const bool seg_start = (g == gs) || (wk.j == 0);
+    const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
+    const int nt = (wk.page_tokens(ps) + kWTok - 1) / kWTok;
+    for (int ti = 0; ti < nt; ++ti) f(wk, ti * kWTok, seg_start && ti == 0, seg_end && ti == nt - 1);
+    if (g + 1 < ge) wk.advance(p, kWRows);
+  }
+}
+
+__global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kWBar);
+  uint64_t *kv_full = bars, *kv_free = bars + kWStages, *s_full = bars + 2 * kWStages, *s_free = s_full + 2;
+  uint64_t *p_full = s_full + 4, *pv_done = s_full + 5, *q_full = s_full + 6, *mma_done = s_full + 7;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kWMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kWMisc + 4);
+  volatile int *mma_issued = reinterpret_cast<volatile int *>(smem + kWMisc + 8);
+  int64_t *loc = reinterpret_cast<int64_t *>(smem + kWLoc);
+  const int ps = p.page_size;
+
+  for (int e = tid; e < 64 * 32; e += kWThreads) {
+    const int idx = e >> 5;
+    s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kWCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    tc_fence_before();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(&kv_full[s], 4);
+      mbar_init(&kv_free[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], kWSoftWarps);
+    }
+    mbar_init(p_full, kWSoftWarps);
+    mbar_init(pv_done, 1);
+    mbar_init(q_full, kWSoftWarps);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    *mma_issued = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  pdl_trigger();
+  pdl_wait();
+  tile_locate<kWThreads>(p, kWRows, loc + 4, loc);
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t gs = loc[0], ge = loc[1];
+  const int u0 = static_cast<int>(loc[2]), off0 = static_cast<int>(loc[3]);
+
+  if (warp == kWMmaWarp) {
+    // ---------------------------------------------------------------- MMA
+    // the whole warp runs this role in step (waits included); lane 0 issues
+    const bool leader = lane == 0;
+    if (gs < ge) {
+      // B descriptors built once; per product only the start address moves,
+      // by whole 16-byte units that never carry out of its 14-bit field
+      const uint64_t dK = umma_desc(smem_addr(smem + kWK), 8, 128), dV = umma_desc(smem_addr(smem + kWV), 128, 8);
+      constexpr uint32_t kIdescS = umma_idesc(128, kWTok, 0);
+      constexpr uint32_t kIdescPV = umma_idesc(128, kD, 1);
+      bool ok = true;
+      uint32_t T = 0, seg = 0, prev_T = 0;
+      bool have_prev = false, prev_first = false;
+      auto issue_pv = [&](uint32_t t, bool first) {
+        ok = mbar_wait<4096>(p_full, t & 1u, p.status, abort_flag) && ok;
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        if (!ok) return;
+        const uint64_t so = (t % kWStages) * static_cast<uint32_t>(kWStageBytes >> 4);
+        const uint32_t pa = tmem + kWColP + (t & 1u) * 64;
+#pragma unroll
+        for (int kc = 0; kc < kWTok / 16; ++kc)
+          umma_ts_by(leader, tmem + kWColO, pa + kc * 8, dV + so + kc * 256, kIdescPV, (first && kc == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kc = 0; kc < kWTok / 16; ++kc)
+          umma_ts_by(leader, tmem + kWColO, pa + 32 + kc * 8, dV + so + kc * 256, kIdescPV, 1u);
+        umma_commit_by(leader, pv_done);
+        umma_commit_by(leader, &kv_free[t % kWStages]);
+      };
+      for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &, int, bool first, bool last) {
+        const uint32_t st = T % kWStages, sb = T & 1u;
+        if (first) ok = mbar_wait<4096>(q_full, seg & 1u, p.status, abort_flag) && ok;
+        ok = mbar_wait<4096>(&kv_full[st], (T / kWStages) & 1u, p.status, abort_flag) && ok;
+        if (T >= 2) ok = mbar_wait<4096>(&s_free[sb], ((T >> 1) + 1u) & 1u, p.status, abort_flag) && ok;
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        if (ok) {
+          const uint64_t so = st * static_cast<uint32_t>(kWStageBytes >> 4);
+          const uint32_t d = tmem + kWColS + 64 * sb;
+#pragma unroll
+          for (int kc = 0; kc < kD / 16; ++kc)
+            umma_ts_by(leader, d, tmem + kWColQh + kc * 8, dK + so + kc * 16, kIdescS, kc > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kc = 0; kc < kD / 16; ++kc)
+            umma_ts_by(leader, d, tmem + kWColQl + kc * 8, dK + so + kc * 16, kIdescS, 1u);
+          umma_commit_by(leader, &s_full[sb]);
+          *mma_issued = 1;
+        }
+        // the previous tile's P.V (same stream) after this tile's scores
+        if (have_prev) issue_pv(prev_T, prev_first);
+        have_prev = false;
+        if (last) {
+          issue_pv(T, first);
+          ++seg;
+        } else {
+          have_prev = true;
+          prev_T = T;
+          prev_first = first;
+        }
+        ++T;
+      });
+      __syncwarp();
+      if (*mma_issued) umma_commit_by(leader, mma_done);
+    }
+  } else if (warp >= kWSoftWarps) {
+    // ------------------------------------------------------------ decoders
+    const int grp = (warp - kWSoftWarps) >> 2;
+    const int i = tid - (kWSoftWarps + 4 * grp) * 32;
+    const int r = i & 63;
+    const bool is_v = i >= 64;
+    const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+    uint8_t *tile0 = smem + (is_v ? kWV : kWK);
+    float *nrm0 = reinterpret_cast<float *>(smem + (is_v ? kWVN : kWKN));
+    bool ok = true;
+    uint32_t T = 0;
+    int cur_page = -1, cur_h = -1, cur_u = -1;
+    const uint32_t *cw = nullptr;
+    const __half *nw = nullptr;
+    for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &wk, int t0, bool, bool) {
+      if (T % kWDecGroups == static_cast<uint32_t>(grp)) {
+        const uint32_t st = T % kWStages;
+        uint8_t *tile = tile0 + st * kWStageBytes;
+        float *nrm_out = nrm0 + st * kWTok;
+        if (wk.j != cur_page || wk.h != cur_h || wk.u != cur_u) {
+          cur_page = wk.j;
+          cur_h = wk.h;
+          cur_u = wk.u;
+          int phys = -1;
+          if (wk.j < p.max_pages) phys = p.page_table[static_cast<int64_t>(wk.b) * p.max_pages + wk.j];
+          if (phys < 0 || phys >= p.num_pages) {
+            if (i == 0) set_status(p.status, ISOQUANT_DEVERR_PAGE_RANGE);
+            phys = 0;
+          }
+          const int64_t blk = (static_cast<int64_t>(phys) * 2 + (is_v ? 1 : 0)) * p.H + wk.h;
+          cw = p.codes + blk * kWords * ps;
+          nw = reinterpret_cast<const __half *>(p.norms) + blk * ps;
+        }
+        // the code words are loaded first: their latency overlaps the wait
+        // for stage st, free once the P.V of tile T - kWStages has completed
+        const int t = t0 + r;
+        uint32_t x[kWords];
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) x[w] = __ldg(cw + w * ps + t);
+        const __half nh = nw[t];
+        if (T >= kWStages)
+          ok = mbar_wait<4096>(&kv_free[st], ((T / kWStages) + 1u) & 1u, p.status, abort_flag) && ok;
+        if (ok) {
+          const float nrm = __half2float(nh);
+          uint32_t out[64];
+#pragma unroll
+          for (int w = 0; w < kWords; ++w) {
+#pragma unroll
+            for (int k = 0; k < 5; ++k)
+              if (w < 12 || k < 4) out[5 * w + k] = lut_at((((x[w] >> (6 * k)) & 63u) << 7) | lane4);
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<uint4 *>(tile + canon_off(r, 8 * c, 2048)) =
+                make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+          nrm_out[r] = nrm;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&kv_full[st]);
+      }
+      ++T;
+    });
+  } else {
+    // ------------------------------------------------------------- softmax
+    // thread (r, hf): row r of the stream (tensor-memory lane r), tokens
+    // 32 hf .. 32 hf + 31 of each tile, Q~ dims and O columns 64 hf ..
+    // 64 hf + 63
+    const int r = tid & (kWRows - 1), hf = tid >> 7;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);  // this warp's lanes
+    float *red = reinterpret_cast<float *>(smem + kWRed);  // [2 tiles][2 halves][128 rows]
+    bool ok = true;
+    uint32_t T = 0;
+    float m_run = -INFINITY, l_half = 0.f, rs = 1.f;
+    int lim = 0;
+    bool row_valid = false;
+    for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &wk, int t0, bool first, bool last) {
+      const uint32_t st = T % kWStages, sb = T & 1u;
+      const int row = wk.rg * kWRows + r;
+      if (first) {
+        // the stream's rows as Q~ in tensor memory (high parts, low parts),
+        // each row prescaled by a power of two so that its largest |q|
+        // lands in [2^14, 2^15).  Every S of the previous stream has been
+        // read.
+        row_valid = row < p.R;
+        const int qi = row_valid ? row / p.G : 0;
+        const int hq = wk.h * p.G + (row_valid ? row % p.G : 0);
+        const float *qp = p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD;
+        float mx = 0.f;
+        for (int d = 0; d < kD; d += 4) {
+          const float4 v = row_valid ? *reinterpret_cast<const float4 *>(qp + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+        mx *= p.qfold;
+        int ex = 0;
+        if (mx > 0.f) frexpf(mx, &ex);
+        ex = max(ex, -100);
+        const float up = ldexpf(1.f, 15 - ex) * p.qfold;
+        rs = ldexpf(1.f, ex - 15);
+        for (int c16 = 0; c16 < 2; ++c16) {
+          // dims 64 hf + 32 c16 .. + 31: 16 packed columns of each part
+          uint32_t wh[16], wl[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int d = 64 * hf + 32 * c16 + 2 * e;
+            const float a = row_valid ? qp[d] * up : 0.f;
+            const float bb = row_valid ? qp[d + 1] * up : 0.f;
+            const __half2 h = __floats2half2_rn(a, bb);
+            const float2 hf2 = __half22float2(h);
+            wh[e] = *reinterpret_cast<const uint32_t *>(&h);
+            wl[e] = pack_half2(a - hf2.x, bb - hf2.y);
+          }
+          tmem_st16u(tl + kWColQh + 32 * hf + 16 * c16, wh);
+          tmem_st16u(tl + kWColQl + 32 * hf + 16 * c16, wl);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        const int L = p.seq_lens[wk.b];
+        lim = row_valid ? (p.causal ? L - p.nq + qi + 1 : L) : 0;
+        m_run = -INFINITY;
+        l_half = 0.f;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full);
+      }
+      // ---- scores of tile T, this thread's 32 tokens
+      ok = mbar_wait<4096>(&s_full[sb], (T >> 1) & 1u, p.status, abort_flag) && ok;
+      tc_fence_after();
+      float sv[32];
+      tmem_ld32(tl + kWColS + 64 * sb + 32 * hf, sv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
+      const float *kn = reinterpret_cast<const float *>(smem + kWKN) + st * kWTok + 32 * hf;
+      const float *vn = reinterpret_cast<const float *>(smem + kWVN) + st * kWTok + 32 * hf;
+      const int pos0 = wk.j * ps + t0 + 32 * hf;
+      const bool masked = __any_sync(0xffffffffu, pos0 + 32 > lim);
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four chains, not one
+#pragma unroll
+      for (int t = 0; t < 32; t += 4) {
+        const float4 k4 = *reinterpret_cast<const float4 *>(kn + t);
+        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x = sv[t + e] * kk[e];
+          if (masked && pos0 + t + e >= lim) x = -INFINITY;
+          sv[t + e] = x;
+          mx4[e] = fmaxf(mx4[e], x);
+        }
+      }
+      // the row's maximum over both halves (exchange buffer alternates by tile)
+      float *rt = red + sb * (2 * kWRows);
+      rt[hf * kWRows + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      named_bar_sync(1, 2 * kWRows);
+      const float m_new = fmaxf(m_run, fmaxf(rt[r], rt[kWRows + r]) * rs);
+      const float corr = (m_run == -INFINITY || m_new == m_run) ? 1.f : ex2(m_run - m_new);
+      const float mm = m_new == -INFINITY ? 0.f : m_new;
+      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+      // P' into tensor-memory buffer sb (its last reader, the P.V of tile
+      // T - 2, has completed: this thread waited for it at tile T - 1 or at
+      // the end of the previous stream)
+      uint32_t ph[16], pl[16];
+#pragma unroll
+      for (int t = 0; t < 32; t += 8) {
+        const float4 va = *reinterpret_cast<const float4 *>(vn + t);
+        const float4 vb = *reinterpret_cast<const float4 *>(vn + t + 4);
+        const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float pe = ex2(fmaf(sv[t + e], rs, -mm));
+          ps4[e & 3] += pe;
+          // masked slots may hold stale norms: select, do not multiply
+          w[e] = masked ? (pe > 0.f ? pe * vv[e] : 0.f) : pe * vv[e];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          // high part: the pair rounded to fp16; low part: what rounding lost
+          const __half2 h = __floats2half2_rn(w[e], w[e + 1]);
+          const float2 hf2 = __half22float2(h);
+          ph[(t + e) >> 1] = *reinterpret_cast<const uint32_t *>(&h);
+          pl[(t + e) >> 1] = pack_half2(w[e] - hf2.x, w[e + 1] - hf2.y);
+        }
+      }
+      tmem_st16u(tl + kWColP + 64 * sb + 16 * hf, ph);
+      tmem_st16u(tl + kWColP + 64 * sb + 32 + 16 * hf, pl);
+      // O is still accumulated by the previous tile's P.V; this thread
+      // rescales O columns 64 hf .. 64 hf + 63 of its row
+      if (!first) {
+        ok = mbar_wait<4096>(pv_done, (T - 1u) & 1u, p.status, abort_flag) && ok;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+          const uint32_t to = tl + kWColO + 64 * hf;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float ov[32];
+            tmem_ld32(to + 32 * c, ov);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] *= corr;
+            tmem_st32(to + 32 * c, ov);
+          }
+        }
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      l_half = l_half * corr + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
+      m_run = m_new;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      if (last) {
+        // ---- the stream's record: (m, l) and the row's O after the last P.V
+        ok = mbar_wait<4096>(pv_done, T & 1u, p.status, abort_flag) && ok;
+        tc_fence_after();
+        float *rl = red + 4 * kWRows;  // [2 halves][128 rows]
+        rl[hf * kWRows + r] = l_half;
+        named_bar_sync(1, 2 * kWRows);
+        const int64_t stream = static_cast<int64_t>(wk.u) * p.H + wk.h;
+        float *rec = p.records + ((blockIdx.x + stream) * (kWRows / 8) + (r >> 3)) * static_cast<int64_t>(kRecordFloats);
+        const int rr = r & 7;
+        if (row_valid && hf == 0) {
+          rec[2 * rr] = m_run;
+          rec[2 * rr + 1] = rl[r] + rl[kWRows + r];
+        }
+        const uint32_t to = tl + kWColO + 64 * hf;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float ov[32];
+          tmem_ld32(to + 32 * c, ov);
+          if (row_valid) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+              *reinterpret_cast<float4 *>(rec + 16 + rr * kD + 64 * hf + 32 * c + k) =
+                  make_float4(ov[k], ov[k + 1], ov[k + 2], ov[k + 3]);
+          }
+        }
+        tc_fence_before();
+      }
+      ++T;
+    });
+  }
+  // the products must complete before tensor memory is released
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    if (*mma_issued) mbar_wait<4096>(mma_done, 0, p.status, nullptr);
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kWCols));
   }
 }
 
@@ -1326,15 +1879,25 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
   const int ps = p.page_size;
   float *dst = p.out + static_cast<int64_t>(row_id) * kD + 4 * lane;
 
-  const int np = pages_of(p.seq_lens[b], ps);
-  const int64_t p_rg = static_cast<int64_t>(p.H) * pages_before(p.seq_lens, p.B, ps, lane);
+  int np;
+  int64_t g0, total;
+  if (p.prefix != nullptr) {
+    // tcgen05 kernels: the partial kernel wrote the pages before each unit
+    const int64_t u = static_cast<int64_t>(rg) * p.B + b;
+    const int64_t a0 = __ldcg(p.prefix + u), a1 = __ldcg(p.prefix + u + 1);
+    np = static_cast<int>(a1 - a0) / p.H;
+    g0 = a0 + h * np;
+    total = __ldcg(p.prefix + static_cast<int64_t>(p.RG) * p.B);
+  } else {
+    np = pages_of(p.seq_lens[b], ps);
+    const int64_t p_rg = static_cast<int64_t>(p.H) * pages_before(p.seq_lens, p.B, ps, lane);
+    total = p_rg * p.RG;
+    g0 = rg * p_rg + static_cast<int64_t>(p.H) * pages_before(p.seq_lens, b, ps, lane) + static_cast<int64_t>(h) * np;
+  }
   if (np == 0) {
     *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
-  const int64_t total = p_rg * p.RG;
-  const int64_t g0 = rg * p_rg + static_cast<int64_t>(p.H) * pages_before(p.seq_lens, b, ps, lane) +
-                     static_cast<int64_t>(h) * np;
   const int64_t N = p.n_cta;
   const int64_t c_lo = cta_of_page(g0, N, total), c_hi = cta_of_page(g0 + np - 1, N, total);
   const int64_t pair = (static_cast<int64_t>(rg) * p.B + b) * p.H + h;
@@ -1348,17 +1911,39 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
 int attend_ctas_per_sm() { return kCtasPerSm; }
 
 namespace {
-// The tcgen05 kernel serves 64 or more query rows per KV head (pages of at
-// least 64 tokens); it keeps 8 records per (CTA, stream of 64 rows).
-int tile_streams(const AttendShape &s) { return (s.rows + kTRows - 1) / kTRows; }
-size_t tile_slots(const AttendShape &s, int n_cta) {
-  return (static_cast<size_t>(n_cta) +
-          static_cast<size_t>(tile_streams(s)) * static_cast<size_t>(s.batch) * s.kv_heads) *
-         (kTRows / 8);
+// The tcgen05 kernels serve 64 or more query rows per KV head (pages of at
+// least 64 tokens): k_attend_tiles (streams of 64 rows, two CTAs per SM)
+// below kWideMinRows rows, k_attend_wide (streams of 128 rows, one CTA per
+// SM) from there.  Their workspace: rps / 8 records per (CTA, stream) slot,
+// then the unit prefix (streams * batch + 1 int64).
+#ifndef ISOQUANT_WIDE_MIN_ROWS
+#define ISOQUANT_WIDE_MIN_ROWS 128
+#endif
+constexpr int kWideMinRows = ISOQUANT_WIDE_MIN_ROWS;
+static_assert(kWideMinRows >= kTRows, "the 128-row kernel serves shapes of 64+ rows");
+struct TilePlan {
+  int kind;  // 0: mma.sync kernel, 1: k_attend_tiles, 2: k_attend_wide
+  int rps, streams, n_cta;
+  size_t prefix_off, bytes;
+};
+TilePlan tile_plan(const AttendShape &s, int num_sms) {
+  TilePlan t{};
+  if (s.rows < kTRows || s.page_size < kTTok) return t;
+  t.kind = s.rows >= kWideMinRows ? 2 : 1;
+  t.rps = t.kind == 2 ? kWRows : kTRows;
+  t.n_cta = t.kind == 2 ? num_sms : num_sms * kTCtasPerSm;
+  t.streams = (s.rows + t.rps - 1) / t.rps;
+  const size_t slots = (static_cast<size_t>(t.n_cta) +
+                        static_cast<size_t>(t.streams) * static_cast<size_t>(s.batch) * s.kv_heads) *
+                       static_cast<size_t>(t.rps / 8);
+  t.prefix_off = kWsHeader + slots * kRecordFloats * sizeof(float);
+  t.bytes = t.prefix_off + (static_cast<size_t>(t.streams) * s.batch + 1) * sizeof(int64_t);
+  return t;
 }
-bool use_tiles(const isoquant_ctx *ctx, const AttendShape &s, size_t ws_bytes) {
-  return s.rows >= kTRows && s.page_size >= kTTok &&
-         kWsHeader + tile_slots(s, ctx->num_sms * kTCtasPerSm) * kRecordFloats * sizeof(float) <= ws_bytes;
+TilePlan use_tiles(const isoquant_ctx *ctx, const AttendShape &s, size_t ws_bytes) {
+  TilePlan t = tile_plan(s, ctx->num_sms);
+  if (t.kind != 0 && t.bytes > ws_bytes) t.kind = 0;
+  return t;
 }
 }  // namespace
 
@@ -1367,9 +1952,11 @@ size_t attend_workspace_min_bytes(const AttendShape &s) {
 }
 
 size_t attend_workspace_bytes(const AttendShape &s) {
-  // room for the tcgen05 kernel's records too, when the shape can use it
-  const size_t tiles = s.rows >= kTRows ? tile_slots(s, s.n_cta / kCtasPerSm * kTCtasPerSm) : 0;
-  return kWsHeader + (s.slots > tiles ? s.slots : tiles) * kRecordFloats * sizeof(float);
+  // room for the tcgen05 kernels' records and unit prefix too, when the
+  // shape can use them
+  const size_t mma = attend_workspace_min_bytes(s);
+  const TilePlan t = tile_plan(s, s.n_cta / kCtasPerSm);
+  return t.kind != 0 && t.bytes > mma ? t.bytes : mma;
 }
 
 cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache, const AttendShape &s,
@@ -1386,6 +1973,11 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
     e = cudaFuncSetAttribute(k_attend_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k_attend_tiles, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_attend_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_attend_wide, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured_device = ctx->device;
@@ -1412,9 +2004,13 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
   p.records = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
   p.status = ctx->status;
   p.n_cta = s.n_cta;
-  if (use_tiles(ctx, s, ws_bytes)) {
-    p.RG = tile_streams(s);
-    p.n_cta = ctx->num_sms * kTCtasPerSm;
+  p.prefix = nullptr;
+  const TilePlan t = use_tiles(ctx, s, ws_bytes);
+  if (t.kind != 0) {
+    p.RG = t.streams;
+    p.n_cta = t.n_cta;
+    p.prefix = reinterpret_cast<int64_t *>(static_cast<char *>(ws) + t.prefix_off);
+    if (t.kind == 2) return launch_pdl(k_attend_wide, dim3(p.n_cta), dim3(kWThreads), kWSmemBytes, stream, p);
     return launch_pdl(k_attend_tiles, dim3(p.n_cta), dim3(kTThreads), kTSmemBytes, stream, p);
   }
   return launch_pdl(k_attend_partial, dim3(s.n_cta), dim3(kThreads), kSmemBytes, stream, p);
@@ -1436,10 +2032,13 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
   p.page_size = s.page_size;
   p.n_cta = s.n_cta;
   p.rps = 8;
-  if (use_tiles(ctx, s, ws_bytes)) {
-    p.RG = tile_streams(s);
-    p.n_cta = ctx->num_sms * kTCtasPerSm;
-    p.rps = kTRows;
+  p.prefix = nullptr;
+  const TilePlan t = use_tiles(ctx, s, ws_bytes);
+  if (t.kind != 0) {
+    p.RG = t.streams;
+    p.n_cta = t.n_cta;
+    p.rps = t.rps;
+    p.prefix = reinterpret_cast<const int64_t *>(static_cast<const char *>(ws) + t.prefix_off);
   }
   const int64_t rows = static_cast<int64_t>(s.batch) * s.nq * s.q_heads;
   const int64_t blocks = (rows * 32 + kCombineThreads - 1) / kCombineThreads;

@@ -384,6 +384,63 @@ def test_decode_step_matches_separate_calls_and_oracle(cuda_lib):
         check_pair(sb, b, sb.H - 1, q.float().cpu(), out_b.cpu())
 
 
+@pytest.mark.parametrize("case", ["prefill_b1_L600", "chunk_b2", "rows128_noncausal", "rows200_ragged_ps64",
+                                  "prefill_nq_gt_L"])
+def test_tcgen05_wide_kernel_matches_mma_path_and_oracle(cuda_lib, case):
+    """128 or more query rows per KV head (causal prefill, long chunks) run
+    on the warp-specialised 128-row tcgen05 kernel, each stream walking only
+    the pages inside its causal horizon.  It matches the oracle on every
+    query row of sampled (sequence, head) pairs and the mma.sync kernel (the
+    minimum workspace) on all rows."""
+    from compressed_space_decode_b200.synthetic import Workload
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    if case == "prefill_b1_L600":
+        # a 600-token prompt attends to itself: 2400 rows per KV head, 19
+        # streams (the last of 96 rows), 64-token pages
+        wl = Workload(case, 1, 8, 2, [600], nq=600, page_size=64, causal=True, seed=41)
+    elif case == "chunk_b2":
+        # chunked prefill: the last 200 positions of two ragged contexts
+        wl = Workload(case, 2, 16, 4, [1500, 900], nq=200, page_size=128, causal=True, seed=42)
+    elif case == "rows128_noncausal":
+        wl = Workload(case, 3, 32, 1, [2000, 517, 130], nq=4, page_size=256, causal=False, seed=43)
+    elif case == "rows200_ragged_ps64":
+        wl = Workload(case, 5, 16, 2, [3000, 1, 700, 64, 1234], nq=25, page_size=64, causal=True, seed=44)
+    else:
+        # more query positions than tokens: the first positions see nothing
+        wl = Workload(case, 2, 8, 2, [40, 300], nq=100, page_size=64, causal=True, seed=45)
+    st = DecodeState(wl)
+    q = st.queries(0)
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    csd.isoquant_rotate_q(st.ctx, q.reshape(-1, st.Hq, D), q_rot.view(-1, st.Hq, D))
+    outs = []
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pairs = ((wl.nq * st.G + 7) // 8) * st.B * st.H
+    ws_min = (256 + (2 * n_sms + pairs) * 4160) // 4
+    for ws in (_ws(csd, st), torch.empty(ws_min, dtype=torch.int32, device="cuda").fill_(0x7FC00000)):
+        out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+        csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, ws, out,
+                                   causal=wl.causal)
+        torch.cuda.synchronize()
+        assert csd.isoquant_get_status(st.ctx) == 0
+        outs.append(out.cpu())
+    wide, mma = outs
+    assert torch.isfinite(wide).all()
+    err = rowwise_rel_err(wide.numpy(), mma.numpy())
+    assert err.max() <= 2 * ATTN_TOL, err.max()
+    if wl.causal:
+        # rows that see no token are zero
+        for b in range(st.B):
+            for i in range(wl.nq):
+                if st.seq_lens[b] - wl.nq + i + 1 <= 0:
+                    assert not wide[b, i].any()
+    qc = q.float().cpu()
+    for b in range(st.B):
+        if st.seq_lens[b] == 0:
+            continue
+        check_pair(st, b, (b * 3 + 1) % st.H, qc, wide)
+
+
 @pytest.mark.parametrize("case", ["verify", "ragged_ps64", "rows96_ps128", "short"])
 def test_tcgen05_rows_kernel_matches_mma_path(cuda_lib, case):
     """64 or more query rows per KV head run on the tcgen05 kernel (one
