@@ -49,6 +49,19 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Measured sustained dense bf16 tensor throughput (TFLOP/s): the fp16
+    products run at the same rate, in a step that keeps them busy for
+    seconds."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            mp = json.load(f)
+        return float(mp["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        return 1400.0, "fallback (sustained)"
+
+
 def source_hash(*names):
     h = hashlib.sha256()
     for n in names:
@@ -358,6 +371,26 @@ def run_reference(args):
     from compressed_space_decode_b200 import synthetic
     torch.cuda.set_device(local_rank)
     wl = synthetic.workloads()[args.workload]
+    if args.workload.startswith("prefill_attend"):
+        ostep, oflops, text = prefill_oracle_sample(wl)
+        for _ in range(args.warmup):
+            ostep()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            ostep()
+        dt = time.perf_counter() - t0
+        value = args.steps * oflops / dt / 1e12
+        print(json.dumps({
+            "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.q_heads, "kv_heads": wl.kv_heads,
+                       "head_dim": 128, "prompt": wl.seq_lens[0], "query_positions": wl.nq, "causal": True},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {text}"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
     o = oracle_sample(wl, 0, 0)
     for _ in range(args.warmup):
         oracle_step(o)
@@ -378,6 +411,176 @@ def run_reference(args):
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
+
+
+# ------------------------------------------------ causal prefill attention
+PREFILL_METRIC = "causal prefill attention TFLOP/s over packed 3-bit KV (4*128 flop per visible query-key pair per q head)"
+
+
+def causal_pairs(wl):
+    """Visible (query position, key) pairs per q head: query i of a sequence
+    of L tokens with nq query positions sees min(L, max(0, L - nq + i + 1))."""
+    import numpy as np
+    i = np.arange(wl.nq, dtype=np.int64)
+    return int(sum(np.clip(L - wl.nq + i + 1, 0, L).sum() for L in wl.seq_lens))
+
+
+def prefill_oracle_sample(wl, rows=32):
+    """The oracle on a bounded sample of the prefill attention: KV head 0 of
+    sequence 0, its own codes of the whole prompt, and the last rows / G
+    query positions of its G query heads.  Returns (step, flops, text)."""
+    import numpy as np
+
+    import oracle
+    from compressed_space_decode_b200 import synthetic
+    L, G, nq = wl.seq_lens[0], wl.group, wl.nq
+    k, v = synthetic.workload_kv_tokens(wl, 0, 0, L, device="cuda")
+    signs, quats = synthetic.rotation_params(wl.seed, wl.kv_heads)
+    s, qt = signs[0].numpy(), quats[0].numpy()
+    kc, kn, _, _ = oracle.compress(s, qt, k[:, 0].double().cpu().numpy())
+    vc, vn, _, _ = oracle.compress(s, qt, v[:, 0].double().cpu().numpy())
+    npos = max(1, rows // G)
+    q = synthetic.workload_queries(wl, 0, device="cuda")[0, nq - npos:, 0:G].double().cpu().numpy()
+    q = q.reshape(npos * G, 128)
+    lim = [max(0, min(L, L - nq + i + 1)) for i in range(nq - npos, nq) for _ in range(G)]
+    flops = 4 * 128 * sum(lim)
+
+    def step():
+        return oracle.attend(s, qt, q, kc, kn, vc, vn, lim)
+    text = (f"sequence 0, KV head 0 of {wl.name}: the last {npos} query positions x {G} q heads "
+            f"({npos * G} rows over up to {L} tokens)")
+    return step, flops, text
+
+
+def run_prefill_attend(args):
+    """Causal prefill attention over the packed cache: every step compresses
+    the prompt's K/V into the paged cache and rotates its queries
+    (isoquant_decode_prep, one launch), then runs the split attention with
+    its combine and inverse rotation (isoquant_attend_decode).  With 128 or
+    more query rows per KV head the partial kernel is the warp-specialised
+    tcgen05 one, each 128-row stream walking only the pages inside its
+    causal horizon.  Reported as useful TFLOP/s (4*128 flop per visible
+    query-key pair per q head); the tensor cores issue twice that (fp16 high
+    and low parts of the queries and of the softmax weights)."""
+    import torch
+
+    import compressed_space_decode_b200 as csd
+    from compressed_space_decode_b200 import synthetic
+    from compressed_space_decode_b200.workload import DecodeState
+
+    wl = synthetic.workloads()[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    st = DecodeState(wl, device=dev, fill=False)
+    B, H, Hq, nq = st.B, st.H, st.Hq, wl.nq
+    kv = [st.kv_tokens(b, 0, wl.seq_lens[b]) for b in range(B)]
+    ks = torch.cat([k for k, _ in kv]).contiguous()
+    vs = torch.cat([v for _, v in kv]).contiguous()
+    slots = torch.cat([st.slots(b, 0, wl.seq_lens[b]) for b in range(B)]).contiguous()
+    qs = [st.queries(i) for i in range(2)]  # two query sets of 268 MB, alternating (> L2)
+    q_rot = torch.empty((B, nq, Hq, 128), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q_rot)
+    ws = csd.alloc_workspace(st.ctx, B, nq, Hq, device=dev)
+    launches = [0]
+    ev = {}
+
+    def step(i, timed):
+        csd.isoquant_decode_prep(st.ctx, st.cache, ks, vs, slots, qs[i % 2].view(B * nq, Hq, 128),
+                                 q_rot.view(B * nq, Hq, 128), stream=stream)
+        launches[0] += csd.isoquant_last_launch_count(st.ctx)
+        if timed:
+            ev[i] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[i][0].record(stream)
+        csd.isoquant_attend_partial(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, ws, causal=True,
+                                    stream=stream)
+        launches[0] += csd.isoquant_last_launch_count(st.ctx)
+        if timed:
+            ev[i][1].record(stream)
+        csd.isoquant_attend_combine(st.ctx, B, nq, Hq, st.seq_lens_dev, st.ps, ws, out, stream=stream)
+        launches[0] += csd.isoquant_last_launch_count(st.ctx)
+
+    for i in range(args.warmup):
+        step(i, False)
+    torch.cuda.synchronize(dev)
+    assert csd.isoquant_get_status(st.ctx) == 0
+    launches[0] = 0
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    part_ms = sum(a.elapsed_time(b) for a, b in ev.values()) / len(ev)
+    flops = 4 * 128 * Hq * causal_pairs(wl)
+    value = flops / (ms / 1e3) / 1e12
+    achieved = flops / (part_ms / 1e3) / 1e12
+    peak, peak_kind = tensor_peak()
+
+    # end to end: the one-call step from pinned host buffers (prompt K/V,
+    # queries, slots, lengths in; the attention output back)
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    kh, vh = ks.cpu().pin_memory(), vs.cpu().pin_memory()
+    qh = qs[0].cpu().pin_memory()
+    sh = slots.cpu().pin_memory()
+    lh = st.seq_lens_dev.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    kd, vd, qd, sd, ld = (torch.empty_like(ks), torch.empty_like(vs), torch.empty_like(qs[0]),
+                          torch.empty_like(slots), torch.empty_like(st.seq_lens_dev))
+    ws_step = csd.alloc_step_workspace(st.ctx, B, nq, Hq, device=dev)
+    h2d = (kd.numel() + vd.numel() + qd.numel()) * 2 + sd.numel() * 8 + ld.numel() * 4
+    d2h = out.numel() * 4
+    del ws
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        qd.copy_(qh, non_blocking=True)
+        sd.copy_(sh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        csd.isoquant_decode_step(st.ctx, st.cache, kd, vd, sd, qd, st.page_table, ld, ws_step, out, causal=True,
+                                 stream=stream)
+        oh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    assert csd.isoquant_get_status(st.ctx) == 0
+
+    line = {
+        "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 accumulate (fp16 high + low parts of queries and softmax weights on tcgen05)",
+        "data": "synthetic (seeded bf16 Student-t(4) K/V, log-uniform channel scales, x20 outliers; N(0,1) queries)",
+        "config": {"workload": wl.name, "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
+                   "prompt": wl.seq_lens[0], "query_positions": nq, "causal": True, "page_size": st.ps,
+                   "step": "decode_prep (compress the prompt's K/V + rotate its queries, one launch) + "
+                           "attend_partial (tcgen05, causal horizon per 128-row stream) + attend_combine",
+                   "l2": "two query sets of 268 MB alternate; no flush"},
+        "e2e": {"value": flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "roofline": {"bound": "tensor", "kernel": "isoquant_attend_partial (k_attend_wide)", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": None, "avg_launch_ms": part_ms, "flops_per_launch": flops,
+                     "tensor_issued_tflops": 2 * achieved},
+        "gpu_launches": launches[0], "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        ostep, oflops, text = prefill_oracle_sample(wl)
+        n, c0 = 0, time.perf_counter()
+        while time.perf_counter() - c0 < args.cpu_seconds:
+            ostep()
+            n += 1
+        dt = time.perf_counter() - c0
+        line["cpu_baseline"] = {"value": n * oflops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{text}, repeated {n}x in {dt:.1f} s"}
+    print(json.dumps(line))
 
 
 def run_prefill(args):
@@ -458,6 +661,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload.startswith("prefill_attend"):
+        run_prefill_attend(args)
     elif args.workload.startswith("prefill"):
         run_prefill(args)
     else:

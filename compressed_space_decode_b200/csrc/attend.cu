@@ -95,6 +95,7 @@ struct PartialParams {
   uint32_t *status;
   int n_cta;
   int64_t *prefix;  // tcgen05 kernels: pages before each (stream, sequence) unit
+  int vpages;       // tcgen05 kernels: work-free pages that follow each (unit, head) block
 };
 
 struct CombineParams {
@@ -105,6 +106,7 @@ struct CombineParams {
   int B, nq, Hq, H, G, RG, page_size, n_cta;
   int rps;  // query rows per stream: 8 (mma.sync kernel), 64 or 128 (tcgen05 kernels)
   const int64_t *prefix;  // null for the mma.sync kernel
+  int vpages;             // as in PartialParams
 };
 
 // ------------------------------------------------------------------ PTX
@@ -168,6 +170,15 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// High part of w >= 0 for an fp16 high/low split: w with its 13 low
+// mantissa bits cleared (exact in fp16 for 2^-14 <= w < 65520), or 0 below
+// 2^-14, where all of w goes to the low part; w - high is exact in fp32 and
+// below 2^-10 w, so the two fp16 parts keep ~21 bits.  Bit operations
+// instead of a round trip through fp16 conversions.
+__device__ __forceinline__ float hi_part(float w) {
+  const float h = __uint_as_float(__float_as_uint(w) & 0xFFFFE000u);
+  return w >= 6.103515625e-05f ? h : 0.f;
 }
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
@@ -249,34 +260,47 @@ __device__ __forceinline__ int unit_horizon(const PartialParams &p, int rps, int
   const int q_last = min(p.nq - 1, (rg * rps + rps - 1) / p.G);
   return max(0, min(L, L - p.nq + q_last + 1));
 }
-// (units and the pages of one unit are counted in 32 bits: the host keeps
-// streams * batch and max_pages * kv_heads below 2^31)
+// The CTAs split pages evenly; where a stream's switch in a CTA costs as
+// much as a few pages of work (k_attend_wide: its queries are loaded, its
+// record written, the pipeline drains), each (unit, head) block of np real
+// pages is followed by vpages work-free ones, so that the split balances
+// work rather than pages (a causal prefill's early streams are one or two
+// tiles long).  (Units and the pages of one unit are counted in 32 bits:
+// the host keeps streams * batch and max_pages * kv_heads below 2^31.)
 __device__ __forceinline__ int64_t unit_pages(const PartialParams &p, int rps, int u) {
   const int rg = u / p.B, b = u - rg * p.B;
-  return static_cast<int64_t>(p.H) * pages_of(unit_horizon(p, rps, rg, b), p.page_size);
+  const int np = pages_of(unit_horizon(p, rps, rg, b), p.page_size);
+  return np > 0 ? static_cast<int64_t>(p.H) * (np + p.vpages) : 0;
 }
 
 struct UWalk {
-  int u, rg, b, h, j, np, hz;
+  int u, rg, b, h, j, np, nb, hz;  // j < nb = np + vpages; pages j >= np carry no work
   __device__ void set(const PartialParams &p, int rps, int u_) {
     u = u_;
     rg = u / p.B;
     b = u - rg * p.B;
     hz = unit_horizon(p, rps, rg, b);
     np = pages_of(hz, p.page_size);
+    nb = np + p.vpages;
   }
   __device__ void start(const PartialParams &p, int rps, int u_, int off) {
     set(p, rps, u_);
-    h = off / np;
-    j = off - h * np;
+    h = off / nb;
+    j = off - h * nb;
   }
   __device__ void advance(const PartialParams &p, int rps) {
-    if (++j < np) return;
+    if (++j < nb) return;
     j = 0;
     if (++h < p.H) return;
     h = 0;
     do set(p, rps, u + 1); while (np == 0);
   }
+  // to page 0 of the next (unit, head) block that has pages
+  __device__ void next_block(const PartialParams &p, int rps) {
+    j = nb - 1;
+    advance(p, rps);
+  }
+  __device__ bool real() const { return j < np; }
   // tokens of the current page this stream sees, and its 64-token tiles
   __device__ int page_tokens(int ps) const { return min(ps, hz - j * ps); }
 };
@@ -1000,18 +1024,22 @@ __host__ __device__ constexpr uint32_t umma_idesc(int m, int n, int b_mn_major) 
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 // One tensor-core product D (+)= A B (kind::f16, fp32 accumulator in tensor
-// memory, A and B in shared memory), issued by the threads with `issue` set
-// (one thread per CTA)
-__device__ __forceinline__ void umma_f16_by(bool issue, uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                            uint32_t acc) {
+// memory, A and B in shared memory), issued by the calling thread
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%6, %7, %8, %9}, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(static_cast<uint32_t>(issue)), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
       : "memory");
 }
-// the same with A in tensor memory (row m = lane m, column c = the packed
-// fp16 pair k = 2c, 2c + 1 of the 16-wide K slice starting at a_tmem)
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+// A in tensor memory (row m = lane m, column c = the packed fp16 pair
+// k = 2c, 2c + 1 of the 16-wide K slice starting at a_tmem), executed by a
+// converged warp and issued by the lane with `issue` set: the descriptor
+// arithmetic stays warp-uniform
 __device__ __forceinline__ void umma_ts_by(bool issue, uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
                                            uint32_t acc) {
   asm volatile(
@@ -1227,8 +1255,8 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
       if (tid == 0 && ok) {
         tc_fence_after();
 #pragma unroll
-        for (int kc2 = 0; kc2 < kD / 16; ++kc2) umma_f16_by(true, tmem, dQ + kc2 * 16, dK + kc2 * 16, kIdescS, kc2 > 0 ? 1u : 0u);
-        umma_commit_by(true, bar_s);
+        for (int kc2 = 0; kc2 < kD / 16; ++kc2) umma_f16(tmem, dQ + kc2 * 16, dK + kc2 * 16, kIdescS, kc2 > 0 ? 1u : 0u);
+        umma_commit(bar_s);
       }
       ok = mbar_wait(bar_s, ph_s, p.status, abort_flag) && ok;
       ok = __all_sync(0xffffffffu, ok);
@@ -1341,8 +1369,8 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
         tc_fence_after();
 #pragma unroll
         for (int kc2 = 0; kc2 < kTTok / 16; ++kc2)
-          umma_f16_by(true, tmem + 128, dP + kc2 * 16, dV + kc2 * 256, kIdescPV, (first_pv && kc2 == 0) ? 0u : 1u);
-        umma_commit_by(true, bar_pv);
+          umma_f16(tmem + 128, dP + kc2 * 16, dV + kc2 * 256, kIdescPV, (first_pv && kc2 == 0) ? 0u : 1u);
+        umma_commit(bar_pv);
       }
       first_pv = false;
       any_pv = true;
@@ -1469,8 +1497,8 @@ constexpr int kWK = 0;                                // kWStages K tiles
 constexpr int kWV = kWK + kWStages * kWStageBytes;    // kWStages V tiles
 constexpr int kWKN = kWV + kWStages * kWStageBytes;   // K norms, kWStages x 64 fp32
 constexpr int kWVN = kWKN + kWStages * kWTok * 4;     // V norms
-constexpr int kWRed = kWVN + kWStages * kWTok * 4;    // row maxima [2][2][128] and sums [2][128]
-constexpr int kWBar = kWRed + 6 * kWRows * 4;         // 2 kWStages + 8 mbarriers
+constexpr int kWRed = kWVN + kWStages * kWTok * 4;    // row maxima [2][2][128], sums [2][128], |q| maxima [2][128]
+constexpr int kWBar = kWRed + 8 * kWRows * 4;         // 2 kWStages + 8 mbarriers
 constexpr int kWMisc = kWBar + (2 * kWStages + 8) * 8;  // tensor-memory base, abort flag, MMA-issued flag
 constexpr int kWLoc = kWMisc + 16;                    // walk start + scan scratch
 constexpr int kWSmemBytes = kWLoc + (4 + kWThreads / 32) * 8;
@@ -1478,8 +1506,9 @@ static_assert(kWK % 128 == 0 && kWV % 128 == 0, "UMMA tile alignment");
 static_assert(kWBar % 8 == 0 && kWLoc % 8 == 0, "barrier alignment");
 
 // the walk's tiles: for each page of [gs, ge), its 64-token tiles within the
-// stream's horizon; f(wk, t0, first, last) with first / last = the stream's
-// first / last tile in this CTA.  Every role runs the same sequence.
+// stream's horizon; f(wk, t0, first, last, more) with first / last = the
+// stream's first / last tile in this CTA and more = another tile follows.
+// Every role runs the same sequence.
 template <typename F>
 __device__ __forceinline__ void for_each_tile(const PartialParams &p, int64_t gs, int64_t ge, int u0, int off0,
                                               F &&f) {
@@ -1488,10 +1517,16 @@ __device__ __forceinline__ void for_each_tile(const PartialParams &p, int64_t gs
   UWalk wk;
   wk.start(p, kWRows, u0, off0);
   for (int64_t g = gs; g < ge; ++g) {
-    const bool seg_start = (g == gs) || (wk.j == 0);
-    const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
-    const int nt = (wk.page_tokens(ps) + kWTok - 1) / kWTok;
-    for (int ti = 0; ti < nt; ++ti) f(wk, ti * kWTok, seg_start && ti == 0, seg_end && ti == nt - 1);
+    if (wk.real()) {
+      const bool seg_start = (g == gs) || (wk.j == 0);
+      const bool seg_end = (g + 1 == ge) || (wk.j + 1 == wk.np);
+      // the next real page: the next one of this block, or the first of the
+      // next block after the work-free pages
+      const bool more_pages = g + 1 + (wk.j + 1 < wk.np ? 0 : p.vpages) < ge;
+      const int nt = (wk.page_tokens(ps) + kWTok - 1) / kWTok;
+      for (int ti = 0; ti < nt; ++ti)
+        f(wk, ti * kWTok, seg_start && ti == 0, seg_end && ti == nt - 1, more_pages || ti + 1 < nt);
+    }
     if (g + 1 < ge) wk.advance(p, kWRows);
   }
 }
@@ -1572,7 +1607,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         umma_commit_by(leader, pv_done);
         umma_commit_by(leader, &kv_free[t % kWStages]);
       };
-      for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &, int, bool first, bool last) {
+      for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &, int, bool first, bool last, bool) {
         const uint32_t st = T % kWStages, sb = T & 1u;
         if (first) ok = mbar_wait<4096>(q_full, seg & 1u, p.status, abort_flag) && ok;
         ok = mbar_wait<4096>(&kv_full[st], (T / kWStages) & 1u, p.status, abort_flag) && ok;
@@ -1621,7 +1656,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
     int cur_page = -1, cur_h = -1, cur_u = -1;
     const uint32_t *cw = nullptr;
     const __half *nw = nullptr;
-    for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &wk, int t0, bool, bool) {
+    for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &wk, int t0, bool, bool, bool) {
       if (T % kWDecGroups == static_cast<uint32_t>(grp)) {
         const uint32_t st = T % kWStages;
         uint8_t *tile = tile0 + st * kWStageBytes;
@@ -1683,53 +1718,85 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
     float m_run = -INFINITY, l_half = 0.f, rs = 1.f;
     int lim = 0;
     bool row_valid = false;
-    for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &wk, int t0, bool first, bool last) {
-      const uint32_t st = T % kWStages, sb = T & 1u;
+    // this thread's 64 dims of row r of stream (wk.rg, wk.b, wk.h)
+    auto q_row = [&](const UWalk &wk) {
       const int row = wk.rg * kWRows + r;
-      if (first) {
-        // the stream's rows as Q~ in tensor memory (high parts, low parts),
-        // each row prescaled by a power of two so that its largest |q|
-        // lands in [2^14, 2^15).  Every S of the previous stream has been
-        // read.
-        row_valid = row < p.R;
-        const int qi = row_valid ? row / p.G : 0;
-        const int hq = wk.h * p.G + (row_valid ? row % p.G : 0);
-        const float *qp = p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD;
-        float mx = 0.f;
-        for (int d = 0; d < kD; d += 4) {
-          const float4 v = row_valid ? *reinterpret_cast<const float4 *>(qp + d) : make_float4(0.f, 0.f, 0.f, 0.f);
-          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        }
-        mx *= p.qfold;
-        int ex = 0;
-        if (mx > 0.f) frexpf(mx, &ex);
-        ex = max(ex, -100);
-        const float up = ldexpf(1.f, 15 - ex) * p.qfold;
-        rs = ldexpf(1.f, ex - 15);
-        for (int c16 = 0; c16 < 2; ++c16) {
-          // dims 64 hf + 32 c16 .. + 31: 16 packed columns of each part
-          uint32_t wh[16], wl[16];
+      const bool valid = row < p.R;
+      const int qi = valid ? row / p.G : 0;
+      const int hq = wk.h * p.G + (valid ? row % p.G : 0);
+      return p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD + 64 * hf;
+    };
+    // Q~ of a stream into tensor memory (high parts, low parts), each row
+    // prescaled by a power of two so that its largest |q| lands in
+    // [2^14, 2^15); sets rs and releases the MMA warp.  The thread reads its
+    // 64 dims (16 independent 16-byte loads), takes the row's maximum with
+    // its partner and reads them again from L1 to convert them.  Called
+    // when no S of the previous stream is pending.
+    auto build_q = [&](const UWalk &wk) {
+      const bool valid = wk.rg * kWRows + r < p.R;
+      const float4 *qp = reinterpret_cast<const float4 *>(q_row(wk));
+      float mx = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int d = 64 * hf + 32 * c16 + 2 * e;
-            const float a = row_valid ? qp[d] * up : 0.f;
-            const float bb = row_valid ? qp[d + 1] * up : 0.f;
-            const __half2 h = __floats2half2_rn(a, bb);
-            const float2 hf2 = __half22float2(h);
-            wh[e] = *reinterpret_cast<const uint32_t *>(&h);
-            wl[e] = pack_half2(a - hf2.x, bb - hf2.y);
-          }
-          tmem_st16u(tl + kWColQh + 32 * hf + 16 * c16, wh);
-          tmem_st16u(tl + kWColQl + 32 * hf + 16 * c16, wl);
+      for (int c = 0; c < 16; ++c) {
+        const float4 v = valid ? __ldg(qp + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
+      float *rq = red + 6 * kWRows;  // [2 halves][128 rows]
+      rq[hf * kWRows + r] = mx;
+      named_bar_sync(1, 2 * kWRows);
+      mx = fmaxf(rq[r], rq[kWRows + r]) * p.qfold;
+      int ex = 0;
+      if (mx > 0.f) frexpf(mx, &ex);
+      ex = max(ex, -100);
+      const float up = ldexpf(1.f, 15 - ex) * p.qfold;
+      rs = ldexpf(1.f, ex - 15);
+#pragma unroll
+      for (int c16 = 0; c16 < 2; ++c16) {
+        // dims 64 hf + 32 c16 .. + 31: 16 packed columns of each part
+        uint32_t wh[16], wl[16];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          // read again: the first pass left the line in L1
+          const float4 v = valid ? __ldg(qp + 8 * c16 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float a0 = v.x * up, a1 = v.y * up, a2 = v.z * up, a3 = v.w * up;
+          const __half2 h0 = __floats2half2_rn(a0, a1), h1 = __floats2half2_rn(a2, a3);
+          const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+          wh[2 * e] = *reinterpret_cast<const uint32_t *>(&h0);
+          wh[2 * e + 1] = *reinterpret_cast<const uint32_t *>(&h1);
+          wl[2 * e] = pack_half2(a0 - f0.x, a1 - f0.y);
+          wl[2 * e + 1] = pack_half2(a2 - f1.x, a3 - f1.y);
         }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tmem_st16u(tl + kWColQh + 32 * hf + 16 * c16, wh);
+        tmem_st16u(tl + kWColQl + 32 * hf + 16 * c16, wl);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
+    };
+    for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &wk, int t0, bool first, bool last, bool more) {
+      const uint32_t st = T % kWStages, sb = T & 1u;
+      if (first) {
+        // the CTA's first stream builds its Q~ here; every later one was
+        // built at the end of the stream before it
+        if (T == 0) build_q(wk);
+        const int row = wk.rg * kWRows + r;
+        row_valid = row < p.R;
         const int L = p.seq_lens[wk.b];
-        lim = row_valid ? (p.causal ? L - p.nq + qi + 1 : L) : 0;
+        lim = row_valid ? (p.causal ? L - p.nq + row / p.G + 1 : L) : 0;
         m_run = -INFINITY;
         l_half = 0.f;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full);
+      }
+      if (last && more) {
+        // the next stream: its queries are fetched into L2 now, so that
+        // building its Q~ after this tile waits on L2, not on HBM
+        UWalk nx = wk;
+        nx.next_block(p, kWRows);
+        const char *qn = reinterpret_cast<const char *>(q_row(nx));
+        if (nx.rg * kWRows + r < p.R) {
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(qn));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(qn + 128));
+        }
       }
       // ---- scores of tile T, this thread's 32 tokens
       ok = mbar_wait<4096>(&s_full[sb], (T >> 1) & 1u, p.status, abort_flag) && ok;
@@ -1783,11 +1850,9 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         }
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-          // high part: the pair rounded to fp16; low part: what rounding lost
-          const __half2 h = __floats2half2_rn(w[e], w[e + 1]);
-          const float2 hf2 = __half22float2(h);
-          ph[(t + e) >> 1] = *reinterpret_cast<const uint32_t *>(&h);
-          pl[(t + e) >> 1] = pack_half2(w[e] - hf2.x, w[e + 1] - hf2.y);
+          const float h0 = hi_part(w[e]), h1 = hi_part(w[e + 1]);
+          ph[(t + e) >> 1] = pack_half2(h0, h1);
+          pl[(t + e) >> 1] = pack_half2(w[e] - h0, w[e + 1] - h1);
         }
       }
       tmem_st16u(tl + kWColP + 64 * sb + 16 * hf, ph);
@@ -1816,9 +1881,16 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
       if (last) {
-        // ---- the stream's record: (m, l) and the row's O after the last P.V
+        // ---- end of the stream in this CTA: once its last P.V completed,
+        // the next stream's Q~ goes in (so that the MMA warp starts on it
+        // while the record is written), then the record: (m, l) and O
         ok = mbar_wait<4096>(pv_done, T & 1u, p.status, abort_flag) && ok;
         tc_fence_after();
+        if (more) {
+          UWalk nx = wk;
+          nx.next_block(p, kWRows);
+          build_q(nx);
+        }
         float *rl = red + 4 * kWRows;  // [2 halves][128 rows]
         rl[hf * kWRows + r] = l_half;
         named_bar_sync(1, 2 * kWRows);
@@ -1885,8 +1957,9 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
     // tcgen05 kernels: the partial kernel wrote the pages before each unit
     const int64_t u = static_cast<int64_t>(rg) * p.B + b;
     const int64_t a0 = __ldcg(p.prefix + u), a1 = __ldcg(p.prefix + u + 1);
-    np = static_cast<int>(a1 - a0) / p.H;
-    g0 = a0 + h * np;
+    const int nb = static_cast<int>(a1 - a0) / p.H;  // real pages + work-free ones, or 0
+    np = nb > 0 ? nb - p.vpages : 0;
+    g0 = a0 + static_cast<int64_t>(h) * nb;
     total = __ldcg(p.prefix + static_cast<int64_t>(p.RG) * p.B);
   } else {
     np = pages_of(p.seq_lens[b], ps);
@@ -1923,7 +1996,7 @@ constexpr int kWideMinRows = ISOQUANT_WIDE_MIN_ROWS;
 static_assert(kWideMinRows >= kTRows, "the 128-row kernel serves shapes of 64+ rows");
 struct TilePlan {
   int kind;  // 0: mma.sync kernel, 1: k_attend_tiles, 2: k_attend_wide
-  int rps, streams, n_cta;
+  int rps, streams, n_cta, vpages;
   size_t prefix_off, bytes;
 };
 TilePlan tile_plan(const AttendShape &s, int num_sms) {
@@ -1933,6 +2006,9 @@ TilePlan tile_plan(const AttendShape &s, int num_sms) {
   t.rps = t.kind == 2 ? kWRows : kTRows;
   t.n_cta = t.kind == 2 ? num_sms : num_sms * kTCtasPerSm;
   t.streams = (s.rows + t.rps - 1) / t.rps;
+  // a stream switch in k_attend_wide costs about 6 tiles of work: 512 tokens
+  // of work-free pages per (unit, head) block
+  t.vpages = t.kind == 2 ? 512 / s.page_size : 0;
   const size_t slots = (static_cast<size_t>(t.n_cta) +
                         static_cast<size_t>(t.streams) * static_cast<size_t>(s.batch) * s.kv_heads) *
                        static_cast<size_t>(t.rps / 8);
@@ -2009,6 +2085,7 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
   if (t.kind != 0) {
     p.RG = t.streams;
     p.n_cta = t.n_cta;
+    p.vpages = t.vpages;
     p.prefix = reinterpret_cast<int64_t *>(static_cast<char *>(ws) + t.prefix_off);
     if (t.kind == 2) return launch_pdl(k_attend_wide, dim3(p.n_cta), dim3(kWThreads), kWSmemBytes, stream, p);
     return launch_pdl(k_attend_tiles, dim3(p.n_cta), dim3(kTThreads), kTSmemBytes, stream, p);
@@ -2038,6 +2115,7 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
     p.RG = t.streams;
     p.n_cta = t.n_cta;
     p.rps = t.rps;
+    p.vpages = t.vpages;
     p.prefix = reinterpret_cast<const int64_t *>(static_cast<const char *>(ws) + t.prefix_off);
   }
   const int64_t rows = static_cast<int64_t>(s.batch) * s.nq * s.q_heads;

@@ -138,7 +138,8 @@ class Workload:
 
 
 def workloads(small: bool = False) -> dict:
-    """The five workloads (sizes as stated in their names).
+    """The workloads (sizes as stated in their names): the five the method is
+    measured on, plus causal prefill attention over a packed prompt.
 
     ``small`` shrinks contexts (and the prefill) to sizes the fp64 oracle
     checks in seconds while keeping several pages, split boundaries and a
@@ -160,6 +161,11 @@ def workloads(small: bool = False) -> dict:
     w["verify_b8_nq16_q32_kv8_L16384"] = Workload(
         "verify_b8_nq16_q32_kv8_L16384", 8, 32, 8, [16384 if not small else 600] * 8, nq=16, causal=True,
         seed=1004, note="16 consecutive query positions per sequence, causal within the chunk")
+    w["prefill_attend_b1_q32_kv8_L32768"] = Workload(
+        "prefill_attend_b1_q32_kv8_L32768", 1, 32, 8, [32768 if not small else 600], nq=32768 if not small else 600,
+        causal=True, seed=1006, shuffle_pages=False,
+        note="causal self-attention of a 32768-token prompt over its own packed K/V: each step compresses the "
+             "prompt's K/V into the cache, rotates its 32768 x 32 queries and attends")
     w["prefill_32768_kv8_layers48"] = Workload(
         "prefill_32768_kv8_layers48", 1, 32, 8, [32768 if not small else 2048], seed=1005,
         layers=48 if not small else 2, shuffle_pages=False,
