@@ -166,6 +166,10 @@ def workloads(small: bool = False) -> dict:
         causal=True, seed=1006, shuffle_pages=False,
         note="causal self-attention of a 32768-token prompt over its own packed K/V: each step compresses the "
              "prompt's K/V into the cache, rotates its 32768 x 32 queries and attends")
+    w["prefill_attend_b1_q32_kv8_L8192"] = Workload(
+        "prefill_attend_b1_q32_kv8_L8192", 1, 32, 8, [8192 if not small else 400], nq=8192 if not small else 400,
+        causal=True, seed=1007, shuffle_pages=False,
+        note="the same at an 8192-token prompt (the profiling case of the prefill attention kernel)")
     w["prefill_32768_kv8_layers48"] = Workload(
         "prefill_32768_kv8_layers48", 1, 32, 8, [32768 if not small else 2048], seed=1005,
         layers=48 if not small else 2, shuffle_pages=False,
