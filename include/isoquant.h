@@ -134,7 +134,10 @@ int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
 /* Workspace bytes isoquant_attend_decode (and the partial/combine pair)
  * needs for this shape: a 256-byte header and one partial record of
  * (16 + 8 * 128) floats per slot, a slot per CTA plus one per
- * (row group, sequence, KV head) pair. */
+ * (row group, sequence, KV head) pair; with 64 or more query rows per KV
+ * head (nq * num_q_heads / num_kv_heads), room for the tensor-core
+ * kernels' records and their work prefix too.  A smaller workspace that
+ * still holds the first part runs the mma.sync kernel. */
 int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
                             int num_q_heads, size_t *bytes);
 
@@ -142,6 +145,12 @@ int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
  * the splits with R^-1 applied once per output row (RotaryQuant, Abstract:
  * attention on the packed codes in the rotated space).  Two kernel launches,
  * the second a programmatic dependent launch that overlaps the first's tail.
+ * The same call serves decode (nq = 1), verification chunks and causal
+ * prefill (nq = the prompt length, causal = 1): with 64 or more query rows
+ * per KV head, pages of at least 64 tokens and the full workspace, the
+ * partial step runs on tcgen05 tensor cores (streams of 64 rows, or of 128
+ * rows from 128 rows up), each stream walking only the pages inside its
+ * causal horizon.
  *   q_rot:      device float [batch][nq][num_q_heads][128] (from rotate_q)
  *   page_table: device int32 [batch][max_pages]
  *   seq_lens:   device int32 [batch]; tokens 0..seq_lens[b]-1 are in the

@@ -1,0 +1,29 @@
+"""Host-side helpers of bench.py that feed reported numbers: the count of
+visible (query, key) pairs behind the prefill-attention FLOP figure, against
+brute force over the causal rule (query i of nq positions over a sequence of L
+tokens sees tokens 0 .. L - nq + i)."""
+import pytest
+
+import bench
+from compressed_space_decode_b200.synthetic import Workload
+
+
+def brute_pairs(lens, nq):
+    n = 0
+    for L in lens:
+        for i in range(nq):
+            for t in range(L):
+                if t <= L - nq + i:
+                    n += 1
+    return n
+
+
+@pytest.mark.parametrize("lens,nq", [([64], 64), ([100], 7), ([5, 40, 0], 12), ([33], 50), ([1], 1)])
+def test_causal_pairs_matches_brute_force(lens, nq):
+    wl = Workload("t", len(lens), 4, 1, lens, nq=nq, causal=True)
+    assert bench.causal_pairs(wl) == brute_pairs(lens, nq)
+
+
+def test_causal_pairs_full_prefill_is_the_triangle():
+    wl = Workload("t", 1, 32, 8, [32768], nq=32768, causal=True)
+    assert bench.causal_pairs(wl) == 32768 * 32769 // 2
