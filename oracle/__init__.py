@@ -23,6 +23,8 @@ D = 128
 BLOCKS = 32
 WORDS = 13
 LEVELS = 8
+# other bit widths: words per vector (floor(32 / bits) codes per word)
+WORDS_FOR = {2: 8, 3: 13, 4: 16}
 
 _lib = None
 
@@ -44,8 +46,12 @@ def lib():
         L.orc_hadamard_entry.restype = ctypes.c_int
         L.orc_hadamard_entry.argtypes = [ctypes.c_int, ctypes.c_int]
         L.orc_compress.restype = ctypes.c_int
+        L.orc_compress_b.restype = ctypes.c_int
         L.orc_attend.restype = None
         L.orc_attend_bruteforce.restype = None
+        L.orc_attend_b.restype = None
+        L.orc_attend_bruteforce_b.restype = None
+        L.orc_format.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -75,11 +81,14 @@ def gauss_distortion(levels, thresholds):
     return lib().orc_gauss_distortion(len(lv), _p(lv, ctypes.c_double), _p(th, ctypes.c_double))
 
 
-def codebook():
-    """(levels16 [8], thresholds [7]): fp16-rounded levels and midpoints."""
-    lv = np.zeros(LEVELS)
-    th = np.zeros(LEVELS - 1)
-    lib().orc_codebook(_p(lv, ctypes.c_double), _p(th, ctypes.c_double))
+def codebook(bits=3):
+    """(levels16 [2^bits], thresholds [2^bits - 1]): fp16-rounded Lloyd-Max
+    levels and midpoints (bits 3: the method's codebook; 2 and 4: the other
+    widths)."""
+    n = 1 << bits
+    lv = np.zeros(n)
+    th = np.zeros(n - 1)
+    lib().orc_codebook_b(ctypes.c_int(bits), _p(lv, ctypes.c_double), _p(th, ctypes.c_double))
     return lv, th
 
 
@@ -165,61 +174,61 @@ def unrotate(signs, quats_raw, y):
 
 
 # ------------------------------------------------------- quantize and pack
-def compress(signs, quats_raw, x, want_z=False):
+def compress(signs, quats_raw, x, want_z=False, bits=3):
     """Compress vectors x [n][128] (any float dtype, read as fp64).
 
-    Returns codes uint32 [n][13], norms uint16 [n] (fp16 bits), z [n][128]
-    (or None) and the number of saturated norms.
+    Returns codes uint32 [n][WORDS_FOR[bits]], norms uint16 [n] (fp16 bits),
+    z [n][128] (or None) and the number of saturated norms.
     """
     s = _signs(signs)
     uq = normalise_quats(quats_raw)
     x = _f64(np.asarray(x, dtype=np.float64).reshape(-1, D))
     n = x.shape[0]
-    codes = np.zeros((n, WORDS), dtype=np.uint32)
+    codes = np.zeros((n, WORDS_FOR[bits]), dtype=np.uint32)
     norms = np.zeros(n, dtype=np.uint16)
     z = np.zeros((n, D)) if want_z else None
-    sat = lib().orc_compress(ctypes.c_int(n), _p(x, ctypes.c_double), _p(s, ctypes.c_int8),
-                             _p(uq, ctypes.c_double), _p(codes, ctypes.c_uint32),
-                             _p(norms, ctypes.c_uint16),
-                             _p(z, ctypes.c_double) if want_z else None)
+    sat = lib().orc_compress_b(ctypes.c_int(bits), ctypes.c_int(n), _p(x, ctypes.c_double), _p(s, ctypes.c_int8),
+                               _p(uq, ctypes.c_double), _p(codes, ctypes.c_uint32),
+                               _p(norms, ctypes.c_uint16),
+                               _p(z, ctypes.c_double) if want_z else None)
     return codes, norms, z, sat
 
 
-def unpack(words):
-    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, WORDS)
+def unpack(words, bits=3):
+    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, WORDS_FOR[bits])
     out = np.zeros((words.shape[0], D), dtype=np.uint8)
     L = lib()
     for r in range(words.shape[0]):
         w = np.ascontiguousarray(words[r])
         c = np.zeros(D, dtype=np.uint8)
-        L.orc_unpack(_p(w, ctypes.c_uint32), _p(c, ctypes.c_uint8))
+        L.orc_unpack_b(ctypes.c_int(bits), _p(w, ctypes.c_uint32), _p(c, ctypes.c_uint8))
         out[r] = c
     return out
 
 
-def dequantize(signs, quats_raw, words, norms):
+def dequantize(signs, quats_raw, words, norms, bits=3):
     s = _signs(signs)
     uq = normalise_quats(quats_raw)
-    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, WORDS)
+    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1, WORDS_FOR[bits])
     norms = np.ascontiguousarray(norms, dtype=np.uint16).reshape(-1)
     out = np.zeros((words.shape[0], D))
     L = lib()
     for r in range(words.shape[0]):
         w = np.ascontiguousarray(words[r])
         xr = np.zeros(D)
-        L.orc_dequantize(_p(w, ctypes.c_uint32), ctypes.c_uint16(int(norms[r])), _p(s, ctypes.c_int8),
-                         _p(uq, ctypes.c_double), _p(xr, ctypes.c_double))
+        L.orc_dequantize_b(ctypes.c_int(bits), _p(w, ctypes.c_uint32), ctypes.c_uint16(int(norms[r])),
+                           _p(s, ctypes.c_int8), _p(uq, ctypes.c_double), _p(xr, ctypes.c_double))
         out[r] = xr
     return out
 
 
 # ------------------------------------------------------------------ attention
-def _attend_args(signs, quats_raw, q, kcodes, knorms, vcodes, vnorms, limits):
+def _attend_args(signs, quats_raw, q, kcodes, knorms, vcodes, vnorms, limits, bits=3):
     s = _signs(signs)
     uq = normalise_quats(quats_raw)
     q = _f64(np.asarray(q, dtype=np.float64).reshape(-1, D))
-    kc = np.ascontiguousarray(kcodes, dtype=np.uint32).reshape(-1, WORDS)
-    vc = np.ascontiguousarray(vcodes, dtype=np.uint32).reshape(-1, WORDS)
+    kc = np.ascontiguousarray(kcodes, dtype=np.uint32).reshape(-1, WORDS_FOR[bits])
+    vc = np.ascontiguousarray(vcodes, dtype=np.uint32).reshape(-1, WORDS_FOR[bits])
     kn = np.ascontiguousarray(knorms, dtype=np.uint16).reshape(-1)
     vn = np.ascontiguousarray(vnorms, dtype=np.uint16).reshape(-1)
     assert kc.shape[0] == vc.shape[0] == kn.shape[0] == vn.shape[0]
@@ -228,28 +237,28 @@ def _attend_args(signs, quats_raw, q, kcodes, knorms, vcodes, vnorms, limits):
     return s, uq, q, kc, kn, vc, vn, lim
 
 
-def attend(signs, quats_raw, q, kcodes, knorms, vcodes, vnorms, limits, scale=None, brute=False):
+def attend(signs, quats_raw, q, kcodes, knorms, vcodes, vnorms, limits, scale=None, brute=False, bits=3):
     """Attention of rows q [R][128] (un-rotated) over one KV head's packed cache.
 
     limits[r] = number of leading tokens row r sees.  scale defaults to
     1/sqrt(128).  Returns out [R][128] in the un-rotated space.
     """
     s, uq, q, kc, kn, vc, vn, lim = _attend_args(signs, quats_raw, q, kcodes, knorms, vcodes, vnorms,
-                                                 limits)
+                                                 limits, bits)
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     R, L = q.shape[0], kc.shape[0]
     out = np.zeros((R, D))
-    fn = lib().orc_attend_bruteforce if brute else lib().orc_attend
-    fn(ctypes.c_int(R), ctypes.c_int(L), _p(q, ctypes.c_double), _p(kc, ctypes.c_uint32),
+    fn = lib().orc_attend_bruteforce_b if brute else lib().orc_attend_b
+    fn(ctypes.c_int(bits), ctypes.c_int(R), ctypes.c_int(L), _p(q, ctypes.c_double), _p(kc, ctypes.c_uint32),
        _p(kn, ctypes.c_uint16), _p(vc, ctypes.c_uint32), _p(vn, ctypes.c_uint16),
        _p(lim, ctypes.c_int32), ctypes.c_double(scale), _p(s, ctypes.c_int8),
        _p(uq, ctypes.c_double), _p(out, ctypes.c_double))
     return out
 
 
-def near_boundary(z, band=1e-6):
+def near_boundary(z, band=1e-6, bits=3):
     """Mask of coordinates whose fp64 z lies within `band` of a threshold."""
-    _, th = codebook()
+    _, th = codebook(bits)
     z = np.asarray(z, dtype=np.float64)
     return (np.abs(z[..., None] - th) < band).any(axis=-1)

@@ -123,13 +123,28 @@ double orc_f16_to_f64(uint16_t h) {
   return sign ? -v : v;
 }
 
-void orc_codebook(double levels16[ORC_LEVELS], double thresholds[ORC_LEVELS - 1]) {
-  double lv[ORC_LEVELS], th[ORC_LEVELS - 1], dist;
-  orc_lloyd_max_gauss(ORC_LEVELS, lv, th, &dist);
-  for (int i = 0; i < ORC_LEVELS; ++i)
+int orc_format(int bits, int *levels, int *per_word, int *words) {
+  if (bits < 2 || bits > 4) return -1;
+  const int cpw = 32 / bits;
+  if (levels) *levels = 1 << bits;
+  if (per_word) *per_word = cpw;
+  if (words) *words = (ORC_D + cpw - 1) / cpw;
+  return 0;
+}
+
+void orc_codebook_b(int bits, double *levels16, double *thresholds) {
+  int nlev = 0;
+  orc_format(bits, &nlev, NULL, NULL);
+  double lv[ORC_MAX_LEVELS], th[ORC_MAX_LEVELS - 1], dist;
+  orc_lloyd_max_gauss(nlev, lv, th, &dist);
+  for (int i = 0; i < nlev; ++i)
     levels16[i] = orc_f16_to_f64(orc_f64_to_f16(lv[i], NULL));
-  for (int k = 0; k < ORC_LEVELS - 1; ++k)
+  for (int k = 0; k < nlev - 1; ++k)
     thresholds[k] = 0.5 * (levels16[k] + levels16[k + 1]);
+}
+
+void orc_codebook(double levels16[ORC_LEVELS], double thresholds[ORC_LEVELS - 1]) {
+  orc_codebook_b(3, levels16, thresholds);
 }
 
 /* ---------------------------------------------------------------- rotation */
@@ -200,11 +215,13 @@ void orc_unrotate(const int8_t *signs, const double *uq, const double *y,
 
 /* ------------------------------------------------------ quantize and pack */
 
-int orc_compress(int n, const double *x, const int8_t *signs,
-                 const double *uq, uint32_t *codes, uint16_t *norms,
-                 double *z_out) {
-  double lv[ORC_LEVELS], th[ORC_LEVELS - 1];
-  orc_codebook(lv, th);
+int orc_compress_b(int bits, int n, const double *x, const int8_t *signs,
+                   const double *uq, uint32_t *codes, uint16_t *norms,
+                   double *z_out) {
+  int nlev, cpw, nw;
+  orc_format(bits, &nlev, &cpw, &nw);
+  double lv[ORC_MAX_LEVELS], th[ORC_MAX_LEVELS - 1];
+  orc_codebook_b(bits, lv, th);
   int saturated = 0;
   for (int v = 0; v < n; ++v) {
     const double *xv = x + (size_t)v * ORC_D;
@@ -216,40 +233,56 @@ int orc_compress(int n, const double *x, const int8_t *signs,
     saturated += sat;
     double y[ORC_D];
     orc_rotate(signs, uq, xv, y);
-    uint32_t *w = codes + (size_t)v * ORC_WORDS;
-    memset(w, 0, sizeof(uint32_t) * ORC_WORDS);
+    uint32_t *w = codes + (size_t)v * nw;
+    memset(w, 0, sizeof(uint32_t) * nw);
     for (int j = 0; j < ORC_D; ++j) {
       double z = (nrm > 0.0) ? sqrt((double)ORC_D) * y[j] / nrm : 0.0;
       if (z_out) z_out[(size_t)v * ORC_D + j] = z;
       uint32_t c = 0;
-      for (int k = 0; k < ORC_LEVELS - 1; ++k) c += (z > th[k]) ? 1u : 0u;
-      w[j / 10] |= c << (3 * (j % 10));
+      for (int k = 0; k < nlev - 1; ++k) c += (z > th[k]) ? 1u : 0u;
+      w[j / cpw] |= c << (bits * (j % cpw));
     }
   }
   return saturated;
 }
 
-void orc_unpack(const uint32_t *words, uint8_t *codes) {
-  for (int j = 0; j < ORC_D; ++j)
-    codes[j] = (uint8_t)((words[j / 10] >> (3 * (j % 10))) & 7u);
+int orc_compress(int n, const double *x, const int8_t *signs,
+                 const double *uq, uint32_t *codes, uint16_t *norms,
+                 double *z_out) {
+  return orc_compress_b(3, n, x, signs, uq, codes, norms, z_out);
 }
+
+void orc_unpack_b(int bits, const uint32_t *words, uint8_t *codes) {
+  int cpw;
+  orc_format(bits, NULL, &cpw, NULL);
+  const uint32_t mask = (1u << bits) - 1u;
+  for (int j = 0; j < ORC_D; ++j)
+    codes[j] = (uint8_t)((words[j / cpw] >> (bits * (j % cpw))) & mask);
+}
+
+void orc_unpack(const uint32_t *words, uint8_t *codes) { orc_unpack_b(3, words, codes); }
 
 /* Centroid vector in rotated space, scaled by the stored norm:
  * (n16 / sqrt(128)) * C[code_j]. */
-static void centroid_scaled(const uint32_t *words, uint16_t norm16,
+static void centroid_scaled(int bits, const uint32_t *words, uint16_t norm16,
                             const double *lv, double *out) {
   uint8_t c[ORC_D];
-  orc_unpack(words, c);
+  orc_unpack_b(bits, words, c);
   double s = orc_f16_to_f64(norm16) / sqrt((double)ORC_D);
   for (int j = 0; j < ORC_D; ++j) out[j] = s * lv[c[j]];
 }
 
+void orc_dequantize_b(int bits, const uint32_t *words, uint16_t norm16,
+                      const int8_t *signs, const double *uq, double *x_hat) {
+  double lv[ORC_MAX_LEVELS], th[ORC_MAX_LEVELS - 1], yhat[ORC_D];
+  orc_codebook_b(bits, lv, th);
+  centroid_scaled(bits, words, norm16, lv, yhat);
+  orc_unrotate(signs, uq, yhat, x_hat);
+}
+
 void orc_dequantize(const uint32_t *words, uint16_t norm16,
                     const int8_t *signs, const double *uq, double *x_hat) {
-  double lv[ORC_LEVELS], th[ORC_LEVELS - 1], yhat[ORC_D];
-  orc_codebook(lv, th);
-  centroid_scaled(words, norm16, lv, yhat);
-  orc_unrotate(signs, uq, yhat, x_hat);
+  orc_dequantize_b(3, words, norm16, signs, uq, x_hat);
 }
 
 /* ---------------------------------------------------------------- attention */
@@ -271,19 +304,21 @@ static void softmax_weighted_sum(int L, int limit, const double *scores,
   (void)L;
 }
 
-void orc_attend(int R, int L, const double *q, const uint32_t *kcodes,
-                const uint16_t *knorms, const uint32_t *vcodes,
-                const uint16_t *vnorms, const int *limit, double scale,
-                const int8_t *signs, const double *uq, double *out) {
-  double lv[ORC_LEVELS], th[ORC_LEVELS - 1];
-  orc_codebook(lv, th);
+void orc_attend_b(int bits, int R, int L, const double *q, const uint32_t *kcodes,
+                  const uint16_t *knorms, const uint32_t *vcodes,
+                  const uint16_t *vnorms, const int *limit, double scale,
+                  const int8_t *signs, const double *uq, double *out) {
+  int nw;
+  orc_format(bits, NULL, NULL, &nw);
+  double lv[ORC_MAX_LEVELS], th[ORC_MAX_LEVELS - 1];
+  orc_codebook_b(bits, lv, th);
   double *kc = (double *)malloc(sizeof(double) * (size_t)L * ORC_D + 8);
   double *vc = (double *)malloc(sizeof(double) * (size_t)L * ORC_D + 8);
   double *sc = (double *)malloc(sizeof(double) * (size_t)L + 8);
   /* rotated-space centroids of every token, norm applied */
   for (int t = 0; t < L; ++t) {
-    centroid_scaled(kcodes + (size_t)t * ORC_WORDS, knorms[t], lv, kc + (size_t)t * ORC_D);
-    centroid_scaled(vcodes + (size_t)t * ORC_WORDS, vnorms[t], lv, vc + (size_t)t * ORC_D);
+    centroid_scaled(bits, kcodes + (size_t)t * nw, knorms[t], lv, kc + (size_t)t * ORC_D);
+    centroid_scaled(bits, vcodes + (size_t)t * nw, vnorms[t], lv, vc + (size_t)t * ORC_D);
   }
   for (int r = 0; r < R; ++r) {
     double qr[ORC_D], o[ORC_D];
@@ -301,18 +336,27 @@ void orc_attend(int R, int L, const double *q, const uint32_t *kcodes,
   free(kc); free(vc); free(sc);
 }
 
-void orc_attend_bruteforce(int R, int L, const double *q,
-                           const uint32_t *kcodes, const uint16_t *knorms,
-                           const uint32_t *vcodes, const uint16_t *vnorms,
-                           const int *limit, double scale,
-                           const int8_t *signs, const double *uq,
-                           double *out) {
+void orc_attend(int R, int L, const double *q, const uint32_t *kcodes,
+                const uint16_t *knorms, const uint32_t *vcodes,
+                const uint16_t *vnorms, const int *limit, double scale,
+                const int8_t *signs, const double *uq, double *out) {
+  orc_attend_b(3, R, L, q, kcodes, knorms, vcodes, vnorms, limit, scale, signs, uq, out);
+}
+
+void orc_attend_bruteforce_b(int bits, int R, int L, const double *q,
+                             const uint32_t *kcodes, const uint16_t *knorms,
+                             const uint32_t *vcodes, const uint16_t *vnorms,
+                             const int *limit, double scale,
+                             const int8_t *signs, const double *uq,
+                             double *out) {
+  int nw;
+  orc_format(bits, NULL, NULL, &nw);
   double *kx = (double *)malloc(sizeof(double) * (size_t)L * ORC_D + 8);
   double *vx = (double *)malloc(sizeof(double) * (size_t)L * ORC_D + 8);
   double *sc = (double *)malloc(sizeof(double) * (size_t)L + 8);
   for (int t = 0; t < L; ++t) {
-    orc_dequantize(kcodes + (size_t)t * ORC_WORDS, knorms[t], signs, uq, kx + (size_t)t * ORC_D);
-    orc_dequantize(vcodes + (size_t)t * ORC_WORDS, vnorms[t], signs, uq, vx + (size_t)t * ORC_D);
+    orc_dequantize_b(bits, kcodes + (size_t)t * nw, knorms[t], signs, uq, kx + (size_t)t * ORC_D);
+    orc_dequantize_b(bits, vcodes + (size_t)t * nw, vnorms[t], signs, uq, vx + (size_t)t * ORC_D);
   }
   for (int r = 0; r < R; ++r) {
     int lim = limit[r] < L ? limit[r] : L;
@@ -324,4 +368,13 @@ void orc_attend_bruteforce(int R, int L, const double *q,
     softmax_weighted_sum(L, lim, sc, vx, out + (size_t)r * ORC_D);
   }
   free(kx); free(vx); free(sc);
+}
+
+void orc_attend_bruteforce(int R, int L, const double *q,
+                           const uint32_t *kcodes, const uint16_t *knorms,
+                           const uint32_t *vcodes, const uint16_t *vnorms,
+                           const int *limit, double scale,
+                           const int8_t *signs, const double *uq,
+                           double *out) {
+  orc_attend_bruteforce_b(3, R, L, q, kcodes, knorms, vcodes, vnorms, limit, scale, signs, uq, out);
 }

@@ -37,6 +37,7 @@
 #define ORC_BLOCKS 32
 #define ORC_WORDS 13
 #define ORC_LEVELS 8
+#define ORC_MAX_LEVELS 16
 
 #ifdef __cplusplus
 extern "C" {
@@ -60,6 +61,33 @@ double orc_f16_to_f64(uint16_t h);
 /* The canonical codebook: fp16-rounded Lloyd-Max levels (as doubles) and
  * the midpoints between adjacent levels. */
 void orc_codebook(double levels16[ORC_LEVELS], double thresholds[ORC_LEVELS - 1]);
+
+/* Other bit widths (the pages' system quantizes weights at 2, 4 and 8 bits;
+ * its KV path is 3-bit): bits in {2, 3, 4} gives 2^bits fp16-rounded
+ * Lloyd-Max levels and midpoint thresholds, floor(32 / bits) codes per word
+ * (16, 10, 8; code j at bits bits*(j % per_word) of word j / per_word) and
+ * ceil(128 / per_word) words per vector (8, 13, 16).  orc_format returns -1
+ * for other widths.  The *_b functions below take the width; the functions
+ * without the suffix are bits = 3. */
+int orc_format(int bits, int *levels, int *per_word, int *words);
+void orc_codebook_b(int bits, double *levels16, double *thresholds);
+int orc_compress_b(int bits, int n, const double *x, const int8_t *signs,
+                   const double *unit_quats, uint32_t *codes, uint16_t *norms,
+                   double *z);
+void orc_unpack_b(int bits, const uint32_t *words, uint8_t *codes);
+void orc_dequantize_b(int bits, const uint32_t *words, uint16_t norm16,
+                      const int8_t *signs, const double *unit_quats,
+                      double *x_hat);
+void orc_attend_b(int bits, int R, int L, const double *q, const uint32_t *kcodes,
+                  const uint16_t *knorms, const uint32_t *vcodes,
+                  const uint16_t *vnorms, const int *limit, double scale,
+                  const int8_t *signs, const double *unit_quats, double *out);
+void orc_attend_bruteforce_b(int bits, int R, int L, const double *q,
+                             const uint32_t *kcodes, const uint16_t *knorms,
+                             const uint32_t *vcodes, const uint16_t *vnorms,
+                             const int *limit, double scale,
+                             const int8_t *signs, const double *unit_quats,
+                             double *out);
 
 /* Hamilton product out = a (x) b, quaternions as (w, x, y, z). */
 void orc_qmul(const double a[4], const double b[4], double out[4]);
