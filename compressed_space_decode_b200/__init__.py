@@ -17,6 +17,7 @@ from . import synthetic  # noqa: F401  (seeded inputs; no method arithmetic)
 
 HEAD_DIM = 128
 WORDS = 13
+WORDS_FOR = {2: 8, 3: 13, 4: 16}  # code words per vector by code width
 
 F32, BF16, F16 = 0, 1, 2
 _DTYPES = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
@@ -34,7 +35,7 @@ SYMBOLS = [
     "isoquant_compress_kv", "isoquant_rotate_q", "isoquant_workspace_size", "isoquant_attend_decode",
     "isoquant_attend_partial", "isoquant_attend_combine", "isoquant_get_status", "isoquant_last_launch_count",
     "isoquant_attend_decode_static", "isoquant_decode_prep", "isoquant_step_workspace_size",
-    "isoquant_decode_step",
+    "isoquant_decode_step", "isoquant_init_bits", "isoquant_codebook_bits",
 ]
 
 
@@ -61,6 +62,8 @@ def lib():
         cp = ctypes.POINTER(_Cache)
         sig = {
             "isoquant_init": ([ctypes.POINTER(vp), i32, i32, vp, vp], i32),
+            "isoquant_init_bits": ([ctypes.POINTER(vp), i32, i32, vp, vp, i32], i32),
+            "isoquant_codebook_bits": ([i32, vp, vp], i32),
             "isoquant_destroy": ([vp], None),
             "isoquant_strerror": ([i32], ctypes.c_char_p),
             "isoquant_codebook": ([vp, vp], i32),
@@ -121,10 +124,11 @@ def _dtype(t):
 class Context:
     """An isoquant_ctx*: per-head rotation parameters on one device."""
 
-    def __init__(self, handle, num_kv_heads, device):
+    def __init__(self, handle, num_kv_heads, device, bits=3):
         self.handle = handle
         self.num_kv_heads = num_kv_heads
         self.device = device
+        self.bits = bits
 
     def close(self):
         if self.handle:
@@ -139,8 +143,9 @@ class Context:
 
 
 class PagedCache:
-    """Caller-owned packed cache: codes int32 [pages][2][H][13][page_size]
-    (bit patterns of uint32 words), norms float16 [pages][2][H][page_size]."""
+    """Caller-owned packed cache: codes int32 [pages][2][H][W][page_size]
+    (bit patterns of uint32 words; W = 13 at 3 bits, 8 at 2, 16 at 4),
+    norms float16 [pages][2][H][page_size]."""
 
     def __init__(self, codes, norms, page_size):
         assert codes.dtype == torch.int32 and norms.dtype == torch.float16
@@ -150,8 +155,9 @@ class PagedCache:
         self.page_size = page_size
 
     @staticmethod
-    def allocate(num_kv_heads, num_pages, page_size, device="cuda"):
-        codes = torch.zeros((num_pages, 2, num_kv_heads, WORDS, page_size), dtype=torch.int32, device=device)
+    def allocate(num_kv_heads, num_pages, page_size, device="cuda", bits=3):
+        codes = torch.zeros((num_pages, 2, num_kv_heads, WORDS_FOR[bits], page_size), dtype=torch.int32,
+                            device=device)
         norms = torch.zeros((num_pages, 2, num_kv_heads, page_size), dtype=torch.float16, device=device)
         return PagedCache(codes, norms, page_size)
 
@@ -160,20 +166,29 @@ class PagedCache:
 
 
 # ----------------------------------------------------------------- C ABI calls
-def isoquant_init(signs, quats, head_dim=HEAD_DIM):
-    """signs: int8 [H][128] (+-1); quats: float32 [H][32][2][4] (host arrays)."""
+def isoquant_init(signs, quats, head_dim=HEAD_DIM, bits=3):
+    """signs: int8 [H][128] (+-1); quats: float32 [H][32][2][4] (host arrays);
+    bits: code width, 3 (the method's) or 2 / 4 (isoquant_init_bits)."""
     signs = torch.as_tensor(signs, dtype=torch.int8).contiguous().cpu()
     quats = torch.as_tensor(quats, dtype=torch.float32).contiguous().cpu()
     H = signs.shape[0]
     h = ctypes.c_void_p()
-    _check(lib().isoquant_init(ctypes.byref(h), H, head_dim, _ptr(signs), _ptr(quats)), "isoquant_init")
-    return Context(h, H, torch.cuda.current_device())
+    if bits == 3:
+        _check(lib().isoquant_init(ctypes.byref(h), H, head_dim, _ptr(signs), _ptr(quats)), "isoquant_init")
+    else:
+        _check(lib().isoquant_init_bits(ctypes.byref(h), H, head_dim, _ptr(signs), _ptr(quats), bits),
+               "isoquant_init_bits")
+    return Context(h, H, torch.cuda.current_device(), bits)
 
 
-def isoquant_codebook():
-    lv = (ctypes.c_float * 8)()
-    th = (ctypes.c_float * 7)()
-    _check(lib().isoquant_codebook(lv, th), "isoquant_codebook")
+def isoquant_codebook(bits=3):
+    n = 1 << bits
+    lv = (ctypes.c_float * n)()
+    th = (ctypes.c_float * (n - 1))()
+    if bits == 3:
+        _check(lib().isoquant_codebook(lv, th), "isoquant_codebook")
+    else:
+        _check(lib().isoquant_codebook_bits(bits, lv, th), "isoquant_codebook_bits")
     return list(lv), list(th)
 
 

@@ -13,38 +13,42 @@
 
 namespace isoquant {
 
-// Lloyd's conditions for the 8-level minimum-MSE quantizer of N(0,1): each
-// decision threshold is the midpoint of its neighbouring levels and each
-// level is the mean of the standard normal restricted to its cell,
+// Lloyd's conditions for the 2^bits-level minimum-MSE quantizer of N(0,1):
+// each decision threshold is the midpoint of its neighbouring levels and
+// each level is the mean of the standard normal restricted to its cell,
 // (pdf(a) - pdf(b)) / (cdf(b) - cdf(a)).  Iterated from evenly spaced levels;
 // the levels are then rounded to fp16 (the stored decode values) and the
-// thresholds taken as midpoints of the rounded levels.
-int build_codebook(Codebook *cb) {
+// thresholds taken as midpoints of the rounded levels.  Unused entries (past
+// 2^bits) are zero.
+int build_codebook(Codebook *cb, int bits) {
   const double inv_sqrt2pi = 0.39894228040143267794;
   auto pdf = [&](double z) { return inv_sqrt2pi * std::exp(-0.5 * z * z); };
   auto cdf = [](double z) { return 0.5 * std::erfc(-z * 0.70710678118654752440); };
-  double lv[kLevels], th[kLevels - 1];
-  for (int i = 0; i < kLevels; ++i) lv[i] = 3.0 * (2.0 * i + 1.0 - kLevels) / kLevels;
-  for (int iter = 0; iter < 100000; ++iter) {
-    for (int k = 0; k < kLevels - 1; ++k) th[k] = 0.5 * (lv[k] + lv[k + 1]);
+  const int n = 1 << bits;
+  *cb = Codebook{};
+  cb->bits = bits;
+  double lv[kMaxLevels], th[kMaxLevels - 1];
+  for (int i = 0; i < n; ++i) lv[i] = 3.0 * (2.0 * i + 1.0 - n) / n;
+  for (int iter = 0; iter < 200000; ++iter) {
+    for (int k = 0; k < n - 1; ++k) th[k] = 0.5 * (lv[k] + lv[k + 1]);
     double moved = 0.0;
-    for (int i = 0; i < kLevels; ++i) {
+    for (int i = 0; i < n; ++i) {
       const double pa = i == 0 ? 0.0 : pdf(th[i - 1]);
-      const double pb = i == kLevels - 1 ? 0.0 : pdf(th[i]);
+      const double pb = i == n - 1 ? 0.0 : pdf(th[i]);
       const double ca = i == 0 ? 0.0 : cdf(th[i - 1]);
-      const double cbv = i == kLevels - 1 ? 1.0 : cdf(th[i]);
+      const double cbv = i == n - 1 ? 1.0 : cdf(th[i]);
       const double c = (pa - pb) / (cbv - ca);
       moved = std::fmax(moved, std::fabs(c - lv[i]));
       lv[i] = c;
     }
     if (moved < 1e-15) break;
   }
-  for (int i = 0; i < kLevels; ++i) {
+  for (int i = 0; i < n; ++i) {
     const __half h = __double2half(lv[i]);
     cb->level16[i] = __half_as_ushort(h);
     cb->level[i] = __half2float(h);
   }
-  for (int k = 0; k < kLevels - 1; ++k) {
+  for (int k = 0; k < n - 1; ++k) {
     cb->threshold64[k] = 0.5 * (static_cast<double>(cb->level[k]) + cb->level[k + 1]);
     cb->threshold[k] = static_cast<float>(cb->threshold64[k]);
   }
@@ -118,6 +122,7 @@ int make_shape(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, int 
   s->row_groups = (s->rows + 7) / 8;
   s->page_size = page_size;
   s->causal = causal ? 1 : 0;
+  s->bits = ctx->codebook.bits;
   s->n_cta = ctx->num_sms * attend_ctas_per_sm();
   s->slots = static_cast<size_t>(s->n_cta) +
              static_cast<size_t>(s->row_groups) * static_cast<size_t>(batch) * ctx->num_kv_heads;
@@ -174,25 +179,35 @@ const char *isoquant_strerror(int status) {
 }
 
 int isoquant_codebook(float levels[8], float thresholds[7]) {
+  return isoquant_codebook_bits(3, levels, thresholds);
+}
+
+int isoquant_codebook_bits(int bits, float *levels, float *thresholds) {
   if (levels == nullptr || thresholds == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 4) return ISOQUANT_ERR_UNSUPPORTED;
   Codebook cb;
-  build_codebook(&cb);
-  for (int i = 0; i < kLevels; ++i) levels[i] = cb.level[i];
-  for (int k = 0; k < kLevels - 1; ++k) thresholds[k] = cb.threshold[k];
+  build_codebook(&cb, bits);
+  for (int i = 0; i < (1 << bits); ++i) levels[i] = cb.level[i];
+  for (int k = 0; k < (1 << bits) - 1; ++k) thresholds[k] = cb.threshold[k];
   return ISOQUANT_OK;
 }
 
 int isoquant_init(isoquant_ctx **out, int num_kv_heads, int head_dim, const int8_t *signs, const float *quats) {
+  return isoquant_init_bits(out, num_kv_heads, head_dim, signs, quats, 3);
+}
+
+int isoquant_init_bits(isoquant_ctx **out, int num_kv_heads, int head_dim, const int8_t *signs, const float *quats,
+                       int bits) {
   if (out == nullptr || signs == nullptr || quats == nullptr || num_kv_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
   *out = nullptr;
-  if (head_dim != kD) return ISOQUANT_ERR_UNSUPPORTED;
+  if (head_dim != kD || bits < 2 || bits > 4) return ISOQUANT_ERR_UNSUPPORTED;
   std::vector<HeadParams> host(static_cast<size_t>(num_kv_heads));
   for (int h = 0; h < num_kv_heads; ++h)
     if (!build_head(signs + static_cast<size_t>(h) * kD, quats + static_cast<size_t>(h) * kBlocks * 8, &host[h]))
       return ISOQUANT_ERR_INVALID_ARG;
   isoquant_ctx *ctx = new (std::nothrow) isoquant_ctx();
   if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
-  build_codebook(&ctx->codebook);
+  build_codebook(&ctx->codebook, bits);
   ctx->num_kv_heads = num_kv_heads;
   if (cudaGetDevice(&ctx->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess ||
@@ -226,7 +241,7 @@ int isoquant_cache_bytes(const isoquant_ctx *ctx, int num_pages, int page_size, 
   if (ctx == nullptr || code_bytes == nullptr || norm_bytes == nullptr || num_pages < 0) return ISOQUANT_ERR_INVALID_ARG;
   if (!valid_page_size(page_size)) return ISOQUANT_ERR_UNSUPPORTED;
   const size_t vecs = static_cast<size_t>(num_pages) * 2 * ctx->num_kv_heads * page_size;
-  *code_bytes = vecs * kWords * sizeof(uint32_t);
+  *code_bytes = vecs * words_for(ctx->codebook.bits) * sizeof(uint32_t);
   *norm_bytes = vecs * sizeof(uint16_t);
   return ISOQUANT_OK;
 }
@@ -360,6 +375,7 @@ int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache, cons
   AttendShape s;
   st = make_shape(ctx, batch, nq, num_q_heads, cache->page_size, causal, &s);
   if (st != ISOQUANT_OK) return st;
+  if (s.bits != 3 && s.page_size < 64) return ISOQUANT_ERR_UNSUPPORTED;  // tcgen05 kernels: 64-token tiles
   if (!(scale >= 0.0f) || !std::isfinite(scale)) return ISOQUANT_ERR_INVALID_ARG;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(kD));
   if (batch == 0) return ISOQUANT_OK;
@@ -383,6 +399,7 @@ int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq, int num_q_head
   AttendShape s;
   int st = make_shape(ctx, batch, nq, num_q_heads, page_size, 0, &s);
   if (st != ISOQUANT_OK) return st;
+  if (s.bits != 3 && s.page_size < 64) return ISOQUANT_ERR_UNSUPPORTED;
   if (batch == 0) return ISOQUANT_OK;
   if (seq_lens == nullptr || workspace == nullptr || out == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   if (!aligned(workspace, 16) || !aligned(out, 16) || !aligned(seq_lens, 4)) return ISOQUANT_ERR_ALIGNMENT;

@@ -90,7 +90,8 @@ struct PartialParams {
   const int32_t *seq_lens;
   int B, nq, Hq, H, G, R, RG, causal;
   float qfold;  // scale * log2(e) / sqrt(128)
-  float level[kLevels];
+  float level[kMaxLevels];
+  int bits;  // code width of the cache (2, 3 or 4)
   float *records;
   uint32_t *status;
   int n_cta;
@@ -385,6 +386,56 @@ __device__ __forceinline__ void word_pairs(uint32_t w, uint32_t lane4, uint32_t 
   out[2] = lut_at(lut_off<5>(w, lane4));
   out[3] = lut_at(lut_off<11>(w, lane4));
   out[4] = lut_at(lut_off<17>(w, lane4));
+}
+
+// The tcgen05 kernels' decode tables, one copy per lane: BITS = 3: entry i =
+// half2(C[i & 7], C[i >> 3]) for the 64 code pairs; BITS = 2: the 16 pairs,
+// half2(C[i & 3], C[i >> 2]); BITS = 4: the 16 single codes, C[i] in the
+// low half (a pair is assembled from two entries).
+template <int BITS>
+__device__ __forceinline__ void fill_lut(const float *level, int tid, int nthreads) {
+  constexpr int kEntries = BITS == 3 ? 64 : 16;
+  for (int e = tid; e < kEntries * 32; e += nthreads) {
+    const int idx = e >> 5;
+    if constexpr (BITS == 3) s_lut[e] = pack_half2(level[idx & 7], level[idx >> 3]);
+    else if constexpr (BITS == 2) s_lut[e] = pack_half2(level[idx & 3], level[idx >> 2]);
+    else s_lut[e] = pack_half2(level[idx], 0.f);
+  }
+}
+// One token's code words (word w at cw[w * ps + t]) ...
+template <int BITS>
+__device__ __forceinline__ void load_token_words(const uint32_t *cw, int ps, int t, uint32_t (&x)[words_for(BITS)]) {
+#pragma unroll
+  for (int w = 0; w < words_for(BITS); ++w) x[w] = __ldg(cw + w * ps + t);
+}
+// ... into its 128 fp16 centroids as 64 half2 (dims 2i, 2i + 1 in out[i])
+template <int BITS>
+__device__ __forceinline__ void decode_token_words(const uint32_t (&x)[words_for(BITS)], uint32_t lane4,
+                                                   uint32_t (&out)[64]) {
+  if constexpr (BITS == 3) {
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) {
+#pragma unroll
+      for (int k = 0; k < 5; ++k)
+        if (w < 12 || k < 4) out[5 * w + k] = lut_at((((x[w] >> (6 * k)) & 63u) << 7) | lane4);
+    }
+  } else if constexpr (BITS == 2) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) out[8 * w + k] = lut_at((((x[w] >> (4 * k)) & 15u) << 7) | lane4);
+    }
+  } else {
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = lut_at((((x[w] >> (8 * k)) & 15u) << 7) | lane4);
+        const uint32_t hi = lut_at((((x[w] >> (8 * k + 4)) & 15u) << 7) | lane4);
+        out[4 * w + k] = __byte_perm(lo, hi, 0x5410);
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
@@ -1103,6 +1154,7 @@ __device__ __forceinline__ uint32_t canon_off(int row, int col, int group_bytes)
   return static_cast<uint32_t>((row >> 3) * group_bytes + (col >> 3) * 128 + (row & 7) * 16 + (col & 7) * 2);
 }
 
+template <int BITS>
 __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const PartialParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1112,10 +1164,7 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kTMisc + 4);
   const int ps = p.page_size;
 
-  for (int e = tid; e < 64 * 32; e += kTThreads) {
-    const int idx = e >> 5;
-    s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
-  }
+  fill_lut<BITS>(p.level, tid, kTThreads);
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                  "r"(kTCols));
@@ -1210,7 +1259,7 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
       phys = 0;
     }
     const int64_t blk = (static_cast<int64_t>(phys) * 2 + (lo_half ? 1 : 0)) * p.H + wk.h;
-    const uint32_t *cw = p.codes + blk * kWords * ps;
+    const uint32_t *cw = p.codes + blk * words_for(BITS) * ps;
     const __half *nw = reinterpret_cast<const __half *>(p.norms) + blk * ps;
 
     const int ntile = (wk.page_tokens(ps) + kTTok - 1) / kTTok;  // tiles within the stream's horizon
@@ -1230,17 +1279,11 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
       // ---- 1. decode token t0 + r of K (threads 0..63) or V (64..127)
       {
         const int t = t0 + r;
-        uint32_t x[kWords];
-#pragma unroll
-        for (int w = 0; w < kWords; ++w) x[w] = __ldg(cw + w * ps + t);
+        uint32_t x[words_for(BITS)];
+        load_token_words<BITS>(cw, ps, t, x);
         const float nrm = __half2float(nw[t]);
         uint32_t out[64];
-#pragma unroll
-        for (int w = 0; w < kWords; ++w) {
-#pragma unroll
-          for (int k = 0; k < 5; ++k)
-            if (w < 12 || k < 4) out[5 * w + k] = lut_at((((x[w] >> (6 * k)) & 63u) << 7) | lane4);
-        }
+        decode_token_words<BITS>(x, lane4, out);
         uint8_t *tile = smem + (lo_half ? kTV : kTK);
 #pragma unroll
         for (int c = 0; c < 16; ++c)
@@ -1531,6 +1574,7 @@ __device__ __forceinline__ void for_each_tile(const PartialParams &p, int64_t gs
   }
 }
 
+template <int BITS>
 __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1543,10 +1587,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
   int64_t *loc = reinterpret_cast<int64_t *>(smem + kWLoc);
   const int ps = p.page_size;
 
-  for (int e = tid; e < 64 * 32; e += kWThreads) {
-    const int idx = e >> 5;
-    s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
-  }
+  fill_lut<BITS>(p.level, tid, kWThreads);
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                  "r"(kWCols));
@@ -1672,27 +1713,21 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
             phys = 0;
           }
           const int64_t blk = (static_cast<int64_t>(phys) * 2 + (is_v ? 1 : 0)) * p.H + wk.h;
-          cw = p.codes + blk * kWords * ps;
+          cw = p.codes + blk * words_for(BITS) * ps;
           nw = reinterpret_cast<const __half *>(p.norms) + blk * ps;
         }
         // the code words are loaded first: their latency overlaps the wait
         // for stage st, free once the P.V of tile T - kWStages has completed
         const int t = t0 + r;
-        uint32_t x[kWords];
-#pragma unroll
-        for (int w = 0; w < kWords; ++w) x[w] = __ldg(cw + w * ps + t);
+        uint32_t x[words_for(BITS)];
+        load_token_words<BITS>(cw, ps, t, x);
         const __half nh = nw[t];
         if (T >= kWStages)
           ok = mbar_wait<4096>(&kv_free[st], ((T / kWStages) + 1u) & 1u, p.status, abort_flag) && ok;
         if (ok) {
           const float nrm = __half2float(nh);
           uint32_t out[64];
-#pragma unroll
-          for (int w = 0; w < kWords; ++w) {
-#pragma unroll
-            for (int k = 0; k < 5; ++k)
-              if (w < 12 || k < 4) out[5 * w + k] = lut_at((((x[w] >> (6 * k)) & 63u) << 7) | lane4);
-          }
+          decode_token_words<BITS>(x, lane4, out);
 #pragma unroll
           for (int c = 0; c < 16; ++c)
             *reinterpret_cast<uint4 *>(tile + canon_off(r, 8 * c, 2048)) =
@@ -2001,7 +2036,9 @@ struct TilePlan {
 };
 TilePlan tile_plan(const AttendShape &s, int num_sms) {
   TilePlan t{};
-  if (s.rows < kTRows || s.page_size < kTTok) return t;
+  // 2- and 4-bit codes always run on the tcgen05 kernels (the mma.sync
+  // kernel's unpacking is 3-bit); 3-bit ones from 64 rows per KV head
+  if ((s.bits == 3 && s.rows < kTRows) || s.page_size < kTTok) return t;
   t.kind = s.rows >= kWideMinRows ? 2 : 1;
   t.rps = t.kind == 2 ? kWRows : kTRows;
   t.n_cta = t.kind == 2 ? num_sms : num_sms * kTCtasPerSm;
@@ -2024,6 +2061,10 @@ TilePlan use_tiles(const isoquant_ctx *ctx, const AttendShape &s, size_t ws_byte
 }  // namespace
 
 size_t attend_workspace_min_bytes(const AttendShape &s) {
+  if (s.bits != 3) {
+    const TilePlan t = tile_plan(s, s.n_cta / kCtasPerSm);
+    return t.kind != 0 ? t.bytes : kWsHeader;
+  }
   return kWsHeader + s.slots * kRecordFloats * sizeof(float);
 }
 
@@ -2034,6 +2075,26 @@ size_t attend_workspace_bytes(const AttendShape &s) {
   const TilePlan t = tile_plan(s, s.n_cta / kCtasPerSm);
   return t.kind != 0 && t.bytes > mma ? t.bytes : mma;
 }
+
+namespace {
+template <int BITS>
+cudaError_t configure_tcgen05() {
+  cudaError_t e = cudaFuncSetAttribute(k_attend_tiles<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_attend_tiles<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_attend_wide<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_attend_wide<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
+}
+template <int BITS>
+cudaError_t launch_tcgen05(int kind, const PartialParams &p, cudaStream_t stream) {
+  if (kind == 2) return launch_pdl(k_attend_wide<BITS>, dim3(p.n_cta), dim3(kWThreads), kWSmemBytes, stream, p);
+  return launch_pdl(k_attend_tiles<BITS>, dim3(p.n_cta), dim3(kTThreads), kTSmemBytes, stream, p);
+}
+}  // namespace
 
 cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache, const AttendShape &s,
                                   const float *q_rot, const int32_t *page_table, int max_pages,
@@ -2046,15 +2107,9 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
     e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_attend_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_attend_tiles, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_attend_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_attend_wide, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
+    e = configure_tcgen05<3>();
+    if (e == cudaSuccess) e = configure_tcgen05<2>();
+    if (e == cudaSuccess) e = configure_tcgen05<4>();
     if (e != cudaSuccess) return e;
     configured_device = ctx->device;
   }
@@ -2076,7 +2131,8 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
   p.RG = s.row_groups;
   p.causal = s.causal;
   p.qfold = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 / std::sqrt(128.0));
-  for (int i = 0; i < kLevels; ++i) p.level[i] = ctx->codebook.level[i];
+  for (int i = 0; i < kMaxLevels; ++i) p.level[i] = ctx->codebook.level[i];
+  p.bits = ctx->codebook.bits;
   p.records = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
   p.status = ctx->status;
   p.n_cta = s.n_cta;
@@ -2087,9 +2143,13 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
     p.n_cta = t.n_cta;
     p.vpages = t.vpages;
     p.prefix = reinterpret_cast<int64_t *>(static_cast<char *>(ws) + t.prefix_off);
-    if (t.kind == 2) return launch_pdl(k_attend_wide, dim3(p.n_cta), dim3(kWThreads), kWSmemBytes, stream, p);
-    return launch_pdl(k_attend_tiles, dim3(p.n_cta), dim3(kTThreads), kTSmemBytes, stream, p);
+    switch (p.bits) {
+      case 2: return launch_tcgen05<2>(t.kind, p, stream);
+      case 4: return launch_tcgen05<4>(t.kind, p, stream);
+      default: return launch_tcgen05<3>(t.kind, p, stream);
+    }
   }
+  if (p.bits != 3) return cudaErrorInvalidValue;  // the callers check shapes first
   return launch_pdl(k_attend_partial, dim3(s.n_cta), dim3(kThreads), kSmemBytes, stream, p);
 }
 

@@ -187,7 +187,7 @@ __device__ __forceinline__ void pack_store_wide(uint64_t cbits, int q, bool stor
 // The fp64 path for one vector, by the whole warp (lane l: coordinates
 // 4l..4l+3): norm, rotation and codes all in fp64.  Used for the few vectors
 // whose fp16 norm rounding or codes the fp32 fast path cannot decide.
-template <typename T>
+template <typename T, int BITS>
 __device__ void compress_one_fp64(const HeadParams &hp, const Codebook &cb, const T *src, uint32_t *codes,
                                   uint16_t *norms, int64_t block, int off, int ps_shift, int lane) {
   float xv[4];
@@ -206,8 +206,22 @@ __device__ void compress_one_fp64(const HeadParams &hp, const Codebook &cb, cons
     const double z = n > 0.0 ? y64[k] / n : 0.0;
     uint32_t code = 0;
 #pragma unroll
-    for (int t = 0; t < kLevels - 1; ++t) code += (z > cb.threshold64[t]) ? 1u : 0u;
+    for (int t = 0; t < (1 << BITS) - 1; ++t) code += (z > cb.threshold64[t]) ? 1u : 0u;
     c[k] = code;
+  }
+  if constexpr (BITS != 3) {
+    // 2 bits: word w = codes 16w..16w+15 = lanes 4w..4w+3 (8 bits each);
+    // 4 bits: word w = codes 8w..8w+7 = lanes 2w, 2w+1 (16 bits each)
+    constexpr int kLanesPerWord = 32 / (4 * BITS);
+    constexpr int kW = words_for(BITS);
+    const uint32_t cl = c[0] | (c[1] << BITS) | (c[2] << (2 * BITS)) | (c[3] << (3 * BITS));
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < kLanesPerWord; ++i)
+      word |= __shfl_sync(0xffffffffu, cl, (kLanesPerWord * lane + i) & 31) << (4 * BITS * i);
+    if (lane < kW) codes[((block * kW + lane) << ps_shift) + off] = word;
+    if (lane == 0) norms[(block << ps_shift) + off] = n16;
+    return;
   }
   // word w holds codes 10w..10w+9, i.e. coordinates of lanes
   // floor(10w/4) .. +2; an odd word starts two codes into its first lane.
@@ -227,8 +241,10 @@ __device__ void compress_one_fp64(const HeadParams &hp, const Codebook &cb, cons
 
 // Warp w of the K (kv = 0) or V (kv = 1) half: rotate, quantize and pack
 // tokens strip * (w / H) .. + strip - 1 of head w % H, four at a time.
-template <typename T>
+template <typename T, int BITS>
 __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uint32_t w, int lane) {
+  constexpr int kHalf = 1 << (BITS - 1);  // codes below kHalf are the negative levels
+  constexpr int kW = words_for(BITS);
   const int H = g.H, n_tok = g.n_tok, ps_shift = g.ps_shift;
   const uint32_t strips = (static_cast<uint32_t>(n_tok) + g.strip - 1) / g.strip;
   const uint32_t sidx = w / static_cast<uint32_t>(H);
@@ -250,7 +266,10 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
       mrow[k][4 * r] = row.x; mrow[k][4 * r + 1] = row.y; mrow[k][4 * r + 2] = row.z; mrow[k][4 * r + 3] = row.w;
     }
   }
-  const float t4 = cb.threshold[4], t5 = cb.threshold[5], t6 = cb.threshold[6];
+  // the positive thresholds (the codebook is symmetric; the middle one is 0)
+  float tp[kHalf - 1];
+#pragma unroll
+  for (int i = 0; i < kHalf - 1; ++i) tp[i] = cb.threshold[kHalf + i];
 
   const int t_begin = static_cast<int>(sidx) * g.strip;
   const int t_end = min(t_begin + g.strip, n_tok);
@@ -302,8 +321,8 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
 #pragma unroll
     for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(__float_as_uint(x[i]) ^ (((sbits >> i) & 1u) << 31));
     wht128_wide(x, q);
-    // codes from |z| and the three positive thresholds (the codebook is
-    // symmetric): z > 0 -> 4 + #{|z| > t}, otherwise 3 - #{|z| >= t}
+    // codes from |z| and the positive thresholds (the codebook is
+    // symmetric): z > 0 -> half + #{|z| > t}, otherwise half - 1 - #{|z| >= t}
     uint64_t cbits = 0;
     bool near = false;
 #pragma unroll
@@ -315,12 +334,17 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
                                    fmaf(mrow[k][4 * r + 1], x[4 * k + 1], mrow[k][4 * r] * x[4 * k])));
         const float z = yr * inv;
         const float a = fabsf(z);
-        const uint32_t gt = (a > t4 ? 1u : 0u) + (a > t5 ? 1u : 0u) + (a > t6 ? 1u : 0u);
-        const uint32_t ge = (a >= t4 ? 1u : 0u) + (a >= t5 ? 1u : 0u) + (a >= t6 ? 1u : 0u);
-        const uint32_t c = z > 0.f ? 4u + gt : 3u - ge;
-        cbits |= static_cast<uint64_t>(c) << (3 * (4 * k + r));
-        near |= (a < kRecheckBand) | (fabsf(a - t4) < kRecheckBand) | (fabsf(a - t5) < kRecheckBand) |
-                (fabsf(a - t6) < kRecheckBand);
+        uint32_t gt = 0, ge = 0;
+        bool nr = a < kRecheckBand;
+#pragma unroll
+        for (int i = 0; i < kHalf - 1; ++i) {
+          gt += a > tp[i] ? 1u : 0u;
+          ge += a >= tp[i] ? 1u : 0u;
+          nr |= fabsf(a - tp[i]) < kRecheckBand;
+        }
+        const uint32_t c = z > 0.f ? kHalf + gt : kHalf - 1 - ge;
+        cbits |= static_cast<uint64_t>(c) << (BITS * (4 * k + r));
+        near |= nr;
       }
     }
     // the group's verdict: any lane near a threshold sends the vector to
@@ -330,7 +354,21 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
     const int off = static_cast<int>(slot & ((1 << ps_shift) - 1));
     const int64_t block = (page * 2 + kv) * H + h;
     const bool fast = valid && !slow;
-    pack_store_wide(cbits, q, fast, g.codes + off, block * kWords, ps_shift);
+    if constexpr (BITS == 3) {
+      pack_store_wide(cbits, q, fast, g.codes + off, block * kWords, ps_shift);
+    } else {
+      // the lane's 16 codes are whole words: word q (2 bits) or words 2q,
+      // 2q + 1 (4 bits)
+      uint32_t *cw = g.codes + off;
+      if (fast) {
+        if constexpr (BITS == 2) {
+          cw[(block * kW + q) << ps_shift] = static_cast<uint32_t>(cbits);
+        } else {
+          cw[(block * kW + 2 * q) << ps_shift] = static_cast<uint32_t>(cbits);
+          cw[(block * kW + 2 * q + 1) << ps_shift] = static_cast<uint32_t>(cbits >> 32);
+        }
+      }
+    }
     if (fast && q == 0) g.norms[(block << ps_shift) + off] = hb;
     // vectors for the fp64 path, one at a time by the whole warp
     uint32_t todo = __ballot_sync(0xffffffffu, valid && slow && q == 0);
@@ -341,18 +379,18 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
       const int tv = tb + gv;
       const int64_t sl = __shfl_sync(0xffffffffu, slot, src_lane);
       const int64_t pg = sl >> ps_shift;
-      compress_one_fp64<T>(hp, cb, src + (static_cast<int64_t>(tv) * H + h) * kD, g.codes, g.norms,
+      compress_one_fp64<T, BITS>(hp, cb, src + (static_cast<int64_t>(tv) * H + h) * kD, g.codes, g.norms,
                            (pg * 2 + kv) * H + h, static_cast<int>(sl & ((1 << ps_shift) - 1)), ps_shift, lane);
     }
   }
 }
 
 // warps per compress block; blockIdx.y selects K or V
-template <typename T>
+template <typename T, int BITS>
 __global__ void __launch_bounds__(256, 2) k_compress(const CompressArgs g) {
   pdl_trigger();
   pdl_wait();
-  compress_warp<T>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), threadIdx.x & 31);
+  compress_warp<T, BITS>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), threadIdx.x & 31);
 }
 
 struct RotateArgs {
@@ -388,7 +426,7 @@ __global__ void __launch_bounds__(256) k_rotate_q(const RotateArgs g) {
 // One launch for the two independent halves of a decode step's preparation:
 // blocks [0, 2 nbc) compress the new K (first nbc) and V tokens, the rest
 // rotate the queries.  Their latency chains overlap instead of adding up.
-template <typename T>
+template <typename T, int BITS>
 __global__ void __launch_bounds__(256) k_decode_prep(const CompressArgs c, const RotateArgs r, int nbc) {
   pdl_trigger();
   pdl_wait();
@@ -397,7 +435,7 @@ __global__ void __launch_bounds__(256) k_decode_prep(const CompressArgs c, const
   const int bx = static_cast<int>(blockIdx.x);
   if (bx < 2 * nbc) {
     const int kv = bx >= nbc ? 1 : 0;
-    compress_warp<T>(c, kv, static_cast<uint32_t>(bx - kv * nbc) * (blockDim.x >> 5) + warp, lane);
+    compress_warp<T, BITS>(c, kv, static_cast<uint32_t>(bx - kv * nbc) * (blockDim.x >> 5) + warp, lane);
   } else {
     rotate_warp<T>(r, static_cast<uint32_t>(bx - 2 * nbc) * (blockDim.x >> 5) + warp, lane);
   }
@@ -457,6 +495,26 @@ int64_t rotate_blocks(int n_rows, int num_q_heads) {
 
 }  // namespace
 
+namespace {
+template <int BITS>
+cudaError_t launch_compress_t(int dtype, dim3 grid, dim3 block, cudaStream_t stream, const CompressArgs &g) {
+  switch (dtype) {
+    case ISOQUANT_F32: return launch_pdl(k_compress<float, BITS>, grid, block, 0, stream, g);
+    case ISOQUANT_BF16: return launch_pdl(k_compress<__nv_bfloat16, BITS>, grid, block, 0, stream, g);
+    default: return launch_pdl(k_compress<__half, BITS>, grid, block, 0, stream, g);
+  }
+}
+template <int BITS>
+cudaError_t launch_prep_t(int dtype, dim3 grid, dim3 block, cudaStream_t stream, const CompressArgs &c,
+                          const RotateArgs &r, int nb) {
+  switch (dtype) {
+    case ISOQUANT_F32: return launch_pdl(k_decode_prep<float, BITS>, grid, block, 0, stream, c, r, nb);
+    case ISOQUANT_BF16: return launch_pdl(k_decode_prep<__nv_bfloat16, BITS>, grid, block, 0, stream, c, r, nb);
+    default: return launch_pdl(k_decode_prep<__half, BITS>, grid, block, 0, stream, c, r, nb);
+  }
+}
+}  // namespace
+
 cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k,
                             const void *v, int dtype, int n_tok, const int64_t *slot_mapping,
                             cudaStream_t stream) {
@@ -465,10 +523,10 @@ cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
   const CompressArgs g = compress_args(ctx, cache, k, v, n_tok, slot_mapping);
   const dim3 grid(static_cast<unsigned>(blocks), 2), block(256);
-  switch (dtype) {
-    case ISOQUANT_F32: return launch_pdl(k_compress<float>, grid, block, 0, stream, g);
-    case ISOQUANT_BF16: return launch_pdl(k_compress<__nv_bfloat16>, grid, block, 0, stream, g);
-    default: return launch_pdl(k_compress<__half>, grid, block, 0, stream, g);
+  switch (ctx->codebook.bits) {
+    case 2: return launch_compress_t<2>(dtype, grid, block, stream, g);
+    case 4: return launch_compress_t<4>(dtype, grid, block, stream, g);
+    default: return launch_compress_t<3>(dtype, grid, block, stream, g);
   }
 }
 
@@ -497,10 +555,10 @@ cudaError_t launch_decode_prep(const isoquant_ctx *ctx, const isoquant_cache *ca
   const RotateArgs r = rotate_args(ctx, q, n_rows, num_q_heads, q_rot);
   const dim3 grid(static_cast<unsigned>(blocks)), block(256);
   const int nb = static_cast<int>(nbc);
-  switch (dtype) {
-    case ISOQUANT_F32: return launch_pdl(k_decode_prep<float>, grid, block, 0, stream, c, r, nb);
-    case ISOQUANT_BF16: return launch_pdl(k_decode_prep<__nv_bfloat16>, grid, block, 0, stream, c, r, nb);
-    default: return launch_pdl(k_decode_prep<__half>, grid, block, 0, stream, c, r, nb);
+  switch (ctx->codebook.bits) {
+    case 2: return launch_prep_t<2>(dtype, grid, block, stream, c, r, nb);
+    case 4: return launch_prep_t<4>(dtype, grid, block, stream, c, r, nb);
+    default: return launch_prep_t<3>(dtype, grid, block, stream, c, r, nb);
   }
 }
 

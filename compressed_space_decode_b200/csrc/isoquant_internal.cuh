@@ -15,8 +15,17 @@ namespace isoquant {
 
 constexpr int kD = 128;
 constexpr int kBlocks = 32;
-constexpr int kWords = 13;
+constexpr int kWords = 13;  // 3-bit codes (the method's): words per vector
 constexpr int kLevels = 8;
+constexpr int kMaxLevels = 16;
+
+// Code formats: `bits` in {2, 3, 4}, floor(32 / bits) codes per 32-bit word
+// (16, 10, 8; code j at bits bits * (j % per_word) of word j / per_word),
+// ceil(128 / per_word) words per vector (8, 13, 16).
+__host__ __device__ constexpr int codes_per_word(int bits) { return 32 / bits; }
+__host__ __device__ constexpr int words_for(int bits) {
+  return (kD + codes_per_word(bits) - 1) / codes_per_word(bits);
+}
 
 // Per-head parameter block in device memory.
 struct HeadParams {
@@ -26,12 +35,13 @@ struct HeadParams {
   uint32_t pad[4];
 };
 
-// Codebook handed to the kernels by value.
+// Codebook handed to the kernels by value (2^bits levels used).
 struct Codebook {
-  float level[kLevels];       // fp16-rounded Lloyd-Max levels, ascending
-  float threshold[kLevels - 1];
-  double threshold64[kLevels - 1];
-  uint16_t level16[kLevels];  // fp16 bits of the levels
+  float level[kMaxLevels];       // fp16-rounded Lloyd-Max levels, ascending
+  float threshold[kMaxLevels - 1];
+  double threshold64[kMaxLevels - 1];
+  uint16_t level16[kMaxLevels];  // fp16 bits of the levels
+  int bits;
 };
 
 }  // namespace isoquant
@@ -49,7 +59,7 @@ struct isoquant_ctx {
 namespace isoquant {
 
 // ------------------------------------------------------------ host helpers
-int build_codebook(Codebook *cb);
+int build_codebook(Codebook *cb, int bits);
 
 // launchers (defined in compress.cu / attend.cu)
 cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k,
@@ -63,6 +73,7 @@ cudaError_t launch_decode_prep(const isoquant_ctx *ctx, const isoquant_cache *ca
 
 struct AttendShape {
   int batch, nq, q_heads, kv_heads, group, rows, row_groups, page_size, causal;
+  int bits;  // code width of the context
   int n_cta;
   size_t slots;       // partial records
 };

@@ -15,8 +15,9 @@ class DecodeState:
     """Packed cache holding ``wl.seq_lens`` tokens per sequence, plus room for
     ``growth`` appended tokens per sequence."""
 
-    def __init__(self, wl, growth=0, device="cuda", fill=True, page_size=None):
+    def __init__(self, wl, growth=0, device="cuda", fill=True, page_size=None, bits=3):
         self.wl = wl
+        self.bits = bits
         self.device = device
         self.H = wl.kv_heads
         self.Hq = wl.q_heads
@@ -24,7 +25,7 @@ class DecodeState:
         self.B = wl.batch
         self.ps = page_size or wl.page_size
         self.signs, self.quats = synthetic.rotation_params(wl.seed, self.H)
-        self.ctx = isoquant_init(self.signs, self.quats)
+        self.ctx = isoquant_init(self.signs, self.quats, bits=bits)
         self.seq_lens = list(wl.seq_lens)
         cap = [L + growth for L in self.seq_lens]
         self.max_pages = max(1, max(math.ceil(c / self.ps) for c in cap))
@@ -38,7 +39,7 @@ class DecodeState:
             off += pages[b]
         self.page_table_cpu = pt
         self.page_table = pt.to(device)
-        self.cache = PagedCache.allocate(self.H, total, self.ps, device=device)
+        self.cache = PagedCache.allocate(self.H, total, self.ps, device=device, bits=bits)
         self.scales = synthetic.workload_scales(wl)
         if fill:
             for b in range(self.B):
@@ -80,7 +81,7 @@ class DecodeState:
 
     # ----------------------------------------------------- canonical views
     def gather(self, b, h, kv, t0, t1):
-        """Canonical packed vectors of tokens [t0, t1): (uint32 words [n][13]
+        """Canonical packed vectors of tokens [t0, t1): (uint32 words [n][W]
         as int64, fp16 norm bits [n] as int64), read back from the cache."""
         t = torch.arange(t0, t1, dtype=torch.int64)
         pages = self.page_table_cpu[b, t // self.ps].to(torch.int64).to(self.device)

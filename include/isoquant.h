@@ -73,6 +73,7 @@ typedef struct isoquant_ctx isoquant_ctx;
 
 /* Paged packed KV cache, caller-owned device memory.
  *   codes: uint32 [num_pages][2 (K,V)][num_kv_heads][13][page_size]
+ *          (8 or 16 words instead of 13 for contexts of 2 or 4 bits)
  *          (word-major inside a page: word w of every token, then word w+1)
  *   norms: uint16 (fp16 bits) [num_pages][2][num_kv_heads][page_size]
  * Token t of a sequence lives in page page_table[b][t / page_size] at
@@ -98,6 +99,20 @@ typedef struct {
 int isoquant_init(isoquant_ctx **out, int num_kv_heads, int head_dim,
                   const int8_t *signs, const float *quats);
 
+/* isoquant_init with another code width (RotaryQuant, Abstract: the KV path
+ * is 3-bit; the system quantizes elsewhere at 2, 4 and 8 bits).  bits in
+ * {2, 3, 4}: 2^bits fp16-rounded Lloyd-Max levels for N(0,1) with midpoint
+ * thresholds, floor(32 / bits) codes per word (16, 10, 8; code j at bits
+ * bits * (j % per_word) of word j / per_word) and ceil(128 / per_word)
+ * words per vector (8, 13, 16) in the cache's code array instead of 13;
+ * everything else as isoquant_init.  A context's width fixes the layout of
+ * every cache used with it.  At 2 and 4 bits attention always runs on the
+ * tensor-core kernels, which need pages of at least 64 tokens (otherwise
+ * UNSUPPORTED) and the full workspace of isoquant_workspace_size.
+ * Errors: as isoquant_init; UNSUPPORTED for another width. */
+int isoquant_init_bits(isoquant_ctx **out, int num_kv_heads, int head_dim,
+                       const int8_t *signs, const float *quats, int bits);
+
 /* Free the context and its device memory (synchronises the device). */
 void isoquant_destroy(isoquant_ctx *ctx);
 
@@ -108,6 +123,10 @@ const char *isoquant_strerror(int status);
  * rounded Lloyd-Max levels for N(0,1), ascending, widened to float, and the
  * 7 decision thresholds (midpoints, exact in float). */
 int isoquant_codebook(float levels[8], float thresholds[7]);
+
+/* The codebook of another width: levels[2^bits], thresholds[2^bits - 1].
+ * Errors: INVALID_ARG (null), UNSUPPORTED (bits not 2, 3 or 4). */
+int isoquant_codebook_bits(int bits, float *levels, float *thresholds);
 
 /* Bytes of the two cache arrays for `num_pages` pages. */
 int isoquant_cache_bytes(const isoquant_ctx *ctx, int num_pages, int page_size,

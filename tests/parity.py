@@ -25,19 +25,19 @@ def near_f16_midpoint(n, rel=BOUNDARY_BAND):
     return (np.abs(mids - n) <= rel * np.abs(n)).any(axis=0)
 
 
-def compare_compressed(x64, signs, quats, gpu_codes, gpu_norms):
+def compare_compressed(x64, signs, quats, gpu_codes, gpu_norms, bits=3):
     """Oracle-compress x64 [n][128] and compare with the GPU's canonical words.
 
     Returns a dict of counts; raises AssertionError on any non-exempt mismatch."""
-    codes, norms, z, _ = oracle.compress(signs, quats, x64, want_z=True)
+    codes, norms, z, _ = oracle.compress(signs, quats, x64, want_z=True, bits=bits)
     gpu_codes = np.asarray(gpu_codes, dtype=np.uint32).reshape(codes.shape)
     gpu_norms = np.asarray(gpu_norms, dtype=np.uint16).reshape(norms.shape)
-    near = oracle.near_boundary(z, BOUNDARY_BAND)
+    near = oracle.near_boundary(z, BOUNDARY_BAND, bits=bits)
     stats = {"vectors": codes.shape[0], "coords": codes.shape[0] * 128, "near_boundary": int(near.sum())}
     word_diff = codes != gpu_codes
     if word_diff.any():
-        oc = oracle.unpack(codes[word_diff.any(1)])
-        gc = oracle.unpack(gpu_codes[word_diff.any(1)])
+        oc = oracle.unpack(codes[word_diff.any(1)], bits=bits)
+        gc = oracle.unpack(gpu_codes[word_diff.any(1)], bits=bits)
         bad = (oc != gc) & ~near[word_diff.any(1)]
         stats["code_mismatch"] = int((oc != gc).sum())
         assert not bad.any(), f"{int(bad.sum())} code mismatches outside the boundary band"
@@ -80,7 +80,7 @@ def oracle_rows(state, b, h, q_cpu, limits_fn, ora, scale=None):
             idx.append((i, hq))
             lims.append(limits_fn(L, i))
     out = oracle.attend(state.signs[h].numpy(), state.quats[h].numpy(), np.stack(rows), kc, kn, vc, vn,
-                        np.array(lims), scale)
+                        np.array(lims), scale, bits=getattr(state, "bits", 3))
     return out, idx
 
 
