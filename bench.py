@@ -33,7 +33,6 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-BYTES_PER_KV_TOKEN_HEAD = 2 * (13 * 4 + 2)  # K and V: 13 words + fp16 norm
 METRIC = "decode attention KV-token·heads/s on packed 3-bit KV; achieved HBM GB/s vs ~8 TB/s"
 UNIT = "KV-token·heads/s"
 DEFAULT_WORKLOAD = "gqa_b16_q32_kv4_L32768_paged"
@@ -158,7 +157,8 @@ def run_ours(args):
     wl = multi.shard_workload(synthetic.workloads()[args.workload], rank, world)
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     growth = args.warmup + args.steps + e2e_steps + 2
-    st = DecodeState(wl, growth=growth, device=dev)
+    st = DecodeState(wl, growth=growth, device=dev, bits=args.bits)
+    bytes_per_token_head = 2 * (csd.WORDS_FOR[args.bits] * 4 + 2)
     B, H, Hq, nq = st.B, st.H, st.Hq, wl.nq
     stream = torch.cuda.current_stream(dev)
 
@@ -230,11 +230,13 @@ def run_ours(args):
     value = units / (ms / 1e3)
 
     # roofline of the attention kernel: algorithmic bytes per launch / duration
-    bytes_per_launch = BYTES_PER_KV_TOKEN_HEAD * units_local / args.steps
+    bytes_per_launch = bytes_per_token_head * units_local / args.steps
     achieved = bytes_per_launch / (attn_avg_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
+    # the profiled traffic is that of the 3-bit mma.sync kernel
     traffic = profiled_traffic(["compressed_space_decode_b200/csrc/attend.cu",
-                                "compressed_space_decode_b200/csrc/isoquant_internal.cuh"], bytes_per_launch)
+                                "compressed_space_decode_b200/csrc/isoquant_internal.cuh"],
+                               bytes_per_launch) if args.bits == 3 else None
 
     # end to end through the public API from pinned host buffers
     attn_events = None
@@ -278,7 +280,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds)
+        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds, bits=args.bits)
 
     if world > 1:
         dist.barrier()
@@ -288,16 +290,20 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32 accumulate (3-bit codes -> f16 centroids, hi/lo f16 queries on mma.sync)",
+        "dtype": ("f32 accumulate (3-bit codes -> f16 centroids, hi/lo f16 queries on mma.sync)" if args.bits == 3 else
+                  f"f32 accumulate ({args.bits}-bit codes -> f16 centroids, hi/lo f16 queries and weights on tcgen05)"),
         "data": "synthetic (seeded bf16 Student-t(4) K/V, log-uniform channel scales, x20 outliers)",
         "config": {"workload": wl.name.split("@")[0], "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
                    "context_start": lens0[0], "page_size": st.ps, "page_table": "shuffled",
                    "step": "decode_prep (append 1 token/seq + rotate q, one launch) + attend_decode (split-K attention + combine); programmatic launches",
                    "l2": f"packed cache {bytes_per_launch / 1e6:.0f} MB > 126 MB L2; no flush",
-                   "parallelism": f"dp{world} (independent shards)"},
+                   "parallelism": f"dp{world} (independent shards)", "code_bits": args.bits,
+                   "bytes_per_kv_token_head": bytes_per_token_head},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "roofline": {"bound": "hbm", "kernel": "isoquant_attend_decode (k_attend_partial + k_attend_combine)", "achieved": achieved, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": ("isoquant_attend_decode (k_attend_partial + k_attend_combine)" if args.bits == 3
+                                                else "isoquant_attend_decode (k_attend_tiles + k_attend_combine)"),
+                     "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
                      "bytes_per_launch": bytes_per_launch, "avg_launch_ms": attn_avg_ms,
                      "frac_of_8TBps": achieved / 8000.0},
@@ -309,7 +315,7 @@ def run_ours(args):
     print(json.dumps(line))
 
 
-def oracle_sample(wl, b, h):
+def oracle_sample(wl, b, h, bits=3):
     """Oracle state for one (sequence, KV head) of workload `wl`: its own
     codes of the context, the appended token and the step's query rows.
     Inputs come from the seeded generators only."""
@@ -320,12 +326,12 @@ def oracle_sample(wl, b, h):
     k, v = synthetic.workload_kv_tokens(wl, b, 0, L + 1, device="cuda")
     signs, quats = synthetic.rotation_params(wl.seed, wl.kv_heads)
     s, qt = signs[h].numpy(), quats[h].numpy()
-    kc, kn, _, _ = oracle.compress(s, qt, k[:L, h].double().cpu().numpy())
-    vc, vn, _, _ = oracle.compress(s, qt, v[:L, h].double().cpu().numpy())
+    kc, kn, _, _ = oracle.compress(s, qt, k[:L, h].double().cpu().numpy(), bits=bits)
+    vc, vn, _, _ = oracle.compress(s, qt, v[:L, h].double().cpu().numpy(), bits=bits)
     newk = k[L:L + 1, h].double().cpu().numpy()
     newv = v[L:L + 1, h].double().cpu().numpy()
     q = synthetic.workload_queries(wl, 0, device="cuda")[b, 0, h * G:(h + 1) * G].double().cpu().numpy()
-    return dict(s=s, qt=qt, kc=kc, kn=kn, vc=vc, vn=vn, newk=newk, newv=newv, q=q, L=L, G=G)
+    return dict(s=s, qt=qt, kc=kc, kn=kn, vc=vc, vn=vn, newk=newk, newv=newv, q=q, L=L, G=G, bits=bits)
 
 
 def oracle_step(o):
@@ -334,20 +340,20 @@ def oracle_step(o):
     import numpy as np
 
     import oracle
-    kc1, kn1, _, _ = oracle.compress(o["s"], o["qt"], o["newk"])
-    vc1, vn1, _, _ = oracle.compress(o["s"], o["qt"], o["newv"])
+    kc1, kn1, _, _ = oracle.compress(o["s"], o["qt"], o["newk"], bits=o["bits"])
+    vc1, vn1, _, _ = oracle.compress(o["s"], o["qt"], o["newv"], bits=o["bits"])
     kc = np.concatenate([o["kc"], kc1])
     kn = np.concatenate([o["kn"], kn1])
     vc = np.concatenate([o["vc"], vc1])
     vn = np.concatenate([o["vn"], vn1])
     R = o["q"].shape[0]
-    return oracle.attend(o["s"], o["qt"], o["q"], kc, kn, vc, vn, [o["L"] + 1] * R)
+    return oracle.attend(o["s"], o["qt"], o["q"], kc, kn, vc, vn, [o["L"] + 1] * R, bits=o["bits"])
 
 
-def cpu_baseline(wl, budget_s=12.0):
+def cpu_baseline(wl, budget_s=12.0, bits=3):
     """The fp64 oracle, as it stands, on the host cores: a bounded sample of
     the same decode step (whole (sequence, KV head) units, repeated)."""
-    o = oracle_sample(wl, 0, 0)
+    o = oracle_sample(wl, 0, 0, bits)
     units, t0 = 0, time.perf_counter()
     while time.perf_counter() - t0 < budget_s:
         oracle_step(o)
@@ -372,7 +378,7 @@ def run_reference(args):
     torch.cuda.set_device(local_rank)
     wl = synthetic.workloads()[args.workload]
     if args.workload.startswith("prefill_attend"):
-        ostep, oflops, text = prefill_oracle_sample(wl)
+        ostep, oflops, text = prefill_oracle_sample(wl, bits=args.bits)
         for _ in range(args.warmup):
             ostep()
         t0 = time.perf_counter()
@@ -391,7 +397,7 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }))
         return
-    o = oracle_sample(wl, 0, 0)
+    o = oracle_sample(wl, 0, 0, args.bits)
     for _ in range(args.warmup):
         oracle_step(o)
     t0 = time.perf_counter()
@@ -407,7 +413,8 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.q_heads, "kv_heads": wl.kv_heads,
-                   "head_dim": 128, "context_start": wl.seq_lens[0], "page_size": wl.page_size},
+                   "head_dim": 128, "context_start": wl.seq_lens[0], "page_size": wl.page_size,
+                   "code_bits": args.bits},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
@@ -425,7 +432,7 @@ def causal_pairs(wl):
     return int(sum(np.clip(L - wl.nq + i + 1, 0, L).sum() for L in wl.seq_lens))
 
 
-def prefill_oracle_sample(wl, rows=32):
+def prefill_oracle_sample(wl, rows=32, bits=3):
     """The oracle on a bounded sample of the prefill attention: KV head 0 of
     sequence 0, its own codes of the whole prompt, and the last rows / G
     query positions of its G query heads.  Returns (step, flops, text)."""
@@ -437,8 +444,8 @@ def prefill_oracle_sample(wl, rows=32):
     k, v = synthetic.workload_kv_tokens(wl, 0, 0, L, device="cuda")
     signs, quats = synthetic.rotation_params(wl.seed, wl.kv_heads)
     s, qt = signs[0].numpy(), quats[0].numpy()
-    kc, kn, _, _ = oracle.compress(s, qt, k[:, 0].double().cpu().numpy())
-    vc, vn, _, _ = oracle.compress(s, qt, v[:, 0].double().cpu().numpy())
+    kc, kn, _, _ = oracle.compress(s, qt, k[:, 0].double().cpu().numpy(), bits=bits)
+    vc, vn, _, _ = oracle.compress(s, qt, v[:, 0].double().cpu().numpy(), bits=bits)
     npos = max(1, rows // G)
     q = synthetic.workload_queries(wl, 0, device="cuda")[0, nq - npos:, 0:G].double().cpu().numpy()
     q = q.reshape(npos * G, 128)
@@ -446,7 +453,7 @@ def prefill_oracle_sample(wl, rows=32):
     flops = 4 * 128 * sum(lim)
 
     def step():
-        return oracle.attend(s, qt, q, kc, kn, vc, vn, lim)
+        return oracle.attend(s, qt, q, kc, kn, vc, vn, lim, bits=bits)
     text = (f"sequence 0, KV head 0 of {wl.name}: the last {npos} query positions x {G} q heads "
             f"({npos * G} rows over up to {L} tokens)")
     return step, flops, text
@@ -472,7 +479,7 @@ def run_prefill_attend(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    st = DecodeState(wl, device=dev, fill=False)
+    st = DecodeState(wl, device=dev, fill=False, bits=args.bits)
     B, H, Hq, nq = st.B, st.H, st.Hq, wl.nq
     kv = [st.kv_tokens(b, 0, wl.seq_lens[b]) for b in range(B)]
     ks = torch.cat([k for k, _ in kv]).contiguous()
@@ -560,6 +567,7 @@ def run_prefill_attend(args):
         "data": "synthetic (seeded bf16 Student-t(4) K/V, log-uniform channel scales, x20 outliers; N(0,1) queries)",
         "config": {"workload": wl.name, "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
                    "prompt": wl.seq_lens[0], "query_positions": nq, "causal": True, "page_size": st.ps,
+                   "code_bits": args.bits,
                    "step": "decode_prep (compress the prompt's K/V + rotate its queries, one launch) + "
                            "attend_partial (tcgen05, causal horizon per 128-row stream) + attend_combine",
                    "l2": "two query sets of 268 MB alternate; no flush"},
@@ -572,7 +580,7 @@ def run_prefill_attend(args):
         "gpu_launches": launches[0], "clocks": clocks,
     }
     if not args.no_cpu_baseline:
-        ostep, oflops, text = prefill_oracle_sample(wl)
+        ostep, oflops, text = prefill_oracle_sample(wl, bits=args.bits)
         n, c0 = 0, time.perf_counter()
         while time.perf_counter() - c0 < args.cpu_seconds:
             ostep()
@@ -656,6 +664,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bits", type=int, default=3, choices=[2, 3, 4],
+                    help="code width of the decode workload (3: the method's; 2 and 4: other widths)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
