@@ -408,34 +408,25 @@ __device__ __forceinline__ void load_token_words(const uint32_t *cw, int ps, int
 #pragma unroll
   for (int w = 0; w < words_for(BITS); ++w) x[w] = __ldg(cw + w * ps + t);
 }
-// ... into its 128 fp16 centroids as 64 half2 (dims 2i, 2i + 1 in out[i])
+// ... pair p of its codes (dims 2p, 2p + 1) as half2 ...
+template <int BITS>
+__device__ __forceinline__ uint32_t decode_pair(const uint32_t (&x)[words_for(BITS)], uint32_t lane4, int p) {
+  if constexpr (BITS == 3) {
+    return lut_at((((x[p / 5] >> (6 * (p % 5))) & 63u) << 7) | lane4);
+  } else if constexpr (BITS == 2) {
+    return lut_at((((x[p / 8] >> (4 * (p % 8))) & 15u) << 7) | lane4);
+  } else {
+    const uint32_t lo = lut_at((((x[p / 4] >> (8 * (p % 4))) & 15u) << 7) | lane4);
+    const uint32_t hi = lut_at((((x[p / 4] >> (8 * (p % 4) + 4)) & 15u) << 7) | lane4);
+    return __byte_perm(lo, hi, 0x5410);
+  }
+}
+// ... or all 128 fp16 centroids as 64 half2 (dims 2i, 2i + 1 in out[i])
 template <int BITS>
 __device__ __forceinline__ void decode_token_words(const uint32_t (&x)[words_for(BITS)], uint32_t lane4,
                                                    uint32_t (&out)[64]) {
-  if constexpr (BITS == 3) {
 #pragma unroll
-    for (int w = 0; w < kWords; ++w) {
-#pragma unroll
-      for (int k = 0; k < 5; ++k)
-        if (w < 12 || k < 4) out[5 * w + k] = lut_at((((x[w] >> (6 * k)) & 63u) << 7) | lane4);
-    }
-  } else if constexpr (BITS == 2) {
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) out[8 * w + k] = lut_at((((x[w] >> (4 * k)) & 15u) << 7) | lane4);
-    }
-  } else {
-#pragma unroll
-    for (int w = 0; w < 16; ++w) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t lo = lut_at((((x[w] >> (8 * k)) & 15u) << 7) | lane4);
-        const uint32_t hi = lut_at((((x[w] >> (8 * k + 4)) & 15u) << 7) | lane4);
-        out[4 * w + k] = __byte_perm(lo, hi, 0x5410);
-      }
-    }
-  }
+  for (int i = 0; i < 64; ++i) out[i] = decode_pair<BITS>(x, lane4, i);
 }
 
 __device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
@@ -1100,6 +1091,22 @@ __device__ __forceinline__ void umma_ts_by(bool issue, uint32_t d_tmem, uint32_t
       "r"(0u)
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
@@ -1484,10 +1491,10 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
 // k_attend_wide: 128 or more query rows per KV head (causal prefill, long
 // verification chunks).  One CTA per SM, warp-specialised, streams of 128
 // query rows, 64-token tiles, the same unit walk as above:
-//   * the decoder warps (groups of 4 after the softmax warps) take the
-//     CTA's tiles in turn into stage T % 2, each thread one token of K
-//     (threads 0..63 of the group) or V (64..127), as in k_attend_tiles.
-//     Two groups in flight hide the load latency of the code words;
+//   * the decoder warps (after the softmax warps) unpack every tile into
+//     stage T % kWStages of a shared-memory ring, a thread one token of K
+//     and of V (2 warps) or of K or V (4 warps), as in k_attend_tiles; they
+//     load a tile's code words before waiting for its stage;
 //   * the last warp, one thread, issues the tensor-core products: S_T = Q~ K_T^T
 //     into one of two score buffers in tensor memory (16 MMAs: the queries'
 //     fp16 high parts, then their low parts, accumulated), and, once the
@@ -1495,10 +1502,12 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
 //     (8 MMAs: the weights' high parts, then their low parts).  S_{T+1} is
 //     issued before P.V_T, so the tensor pipe computes the next scores while
 //     the softmax warps work;
-//   * warps 0..7 run the online softmax: two threads per row r (tensor-
-//     memory lane r of S and O), one per half of the tile's tokens, which
-//     exchange their maxima through shared memory (one warp per row would
-//     leave each SM sub-partition a single latency-bound softmax warp):
+//   * warps 0 .. 4 kWParts - 1 run the online softmax: kWParts threads per
+//     row r (tensor-memory lane r of S and O, reached by warps r / 32 + 4 k),
+//     each with a slice of the tile's tokens and of the row's Q~ dims and O
+//     columns, exchanging their maxima through shared memory (one warp per
+//     row would leave each SM sub-partition a single latency-bound softmax
+//     warp):
 //     scores times the K norms and the row's prescale, causal and length
 //     limits, running max and per-half sums, p * n_v split into fp16
 //     high and low parts (the A operands of P.V, double-buffered so that
@@ -1514,12 +1523,19 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
 // roles skip their work and fall through to the end.
 constexpr int kWRows = 128;
 constexpr int kWTok = 64;
-constexpr int kWSoftWarps = 8;  // two warpgroups: each row's tokens split in halves
-#ifndef ISOQUANT_WIDE_DEC_GROUPS
-#define ISOQUANT_WIDE_DEC_GROUPS 1
+// softmax threads per row (one warpgroup each): a tile's tokens and a row's
+// Q~ dims and O columns are split among them
+#ifndef ISOQUANT_WIDE_PARTS
+#define ISOQUANT_WIDE_PARTS 4
 #endif
-constexpr int kWDecGroups = ISOQUANT_WIDE_DEC_GROUPS;  // decoder groups of 4 warps, taking tiles in turn
-constexpr int kWDecWarps = 4 * kWDecGroups;
+constexpr int kWParts = ISOQUANT_WIDE_PARTS;
+static_assert(kWParts == 2 || kWParts == 4, "two or four softmax warpgroups");
+constexpr int kWSoftWarps = 4 * kWParts;
+constexpr int kWTpt = kWTok / kWParts;  // tokens of a tile per softmax thread
+constexpr int kWDpt = kD / kWParts;     // Q~ dims / O columns per softmax thread
+// decoder warps: 4 (a thread decodes one token of K or V per tile) or 2 (a
+// thread decodes one token of K and of V), keeping registers in budget
+constexpr int kWDecWarps = kWParts == 2 ? 4 : 2;
 constexpr int kWMmaWarp = kWSoftWarps + kWDecWarps;
 constexpr int kWThreads = (kWMmaWarp + 1) * 32;
 // Tensor memory (512 columns, one CTA per SM): S buffers 0 and 1, O, then
@@ -1540,13 +1556,27 @@ constexpr int kWK = 0;                                // kWStages K tiles
 constexpr int kWV = kWK + kWStages * kWStageBytes;    // kWStages V tiles
 constexpr int kWKN = kWV + kWStages * kWStageBytes;   // K norms, kWStages x 64 fp32
 constexpr int kWVN = kWKN + kWStages * kWTok * 4;     // V norms
-constexpr int kWRed = kWVN + kWStages * kWTok * 4;    // row maxima [2][2][128], sums [2][128], |q| maxima [2][128]
-constexpr int kWBar = kWRed + 8 * kWRows * 4;         // 2 kWStages + 8 mbarriers
+constexpr int kWRed = kWVN + kWStages * kWTok * 4;    // per part: row maxima [2 tiles], sums, |q| maxima
+constexpr int kWBar = kWRed + 4 * kWParts * kWRows * 4;  // 2 kWStages + 8 mbarriers
 constexpr int kWMisc = kWBar + (2 * kWStages + 8) * 8;  // tensor-memory base, abort flag, MMA-issued flag
 constexpr int kWLoc = kWMisc + 16;                    // walk start + scan scratch
 constexpr int kWSmemBytes = kWLoc + (4 + kWThreads / 32) * 8;
 static_assert(kWK % 128 == 0 && kWV % 128 == 0, "UMMA tile alignment");
 static_assert(kWBar % 8 == 0 && kWLoc % 8 == 0, "barrier alignment");
+
+// tensor-memory loads / stores by the width of the register array
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float (&v)[N]) {
+  static_assert(N == 16 || N == 32, "x16 or x32");
+  if constexpr (N == 32) tmem_ld32(taddr, v);
+  else tmem_ld16(taddr, v);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t (&v)[N]) {
+  static_assert(N == 8 || N == 16, "x8 or x16");
+  if constexpr (N == 16) tmem_st16u(taddr, v);
+  else tmem_st8u(taddr, v);
+}
 
 // the walk's tiles: for each page of [gs, ge), its 64-token tiles within the
 // stream's horizon; f(wk, t0, first, last, more) with first / last = the
@@ -1596,7 +1626,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
   }
   if (tid == 0) {
     for (int s = 0; s < kWStages; ++s) {
-      mbar_init(&kv_full[s], 4);
+      mbar_init(&kv_full[s], kWDecWarps);
       mbar_init(&kv_free[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -1685,109 +1715,126 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
     }
   } else if (warp >= kWSoftWarps) {
     // ------------------------------------------------------------ decoders
-    const int grp = (warp - kWSoftWarps) >> 2;
-    const int i = tid - (kWSoftWarps + 4 * grp) * 32;
+    // thread i: token r = i % 64 of the tile; with 4 warps K (i < 64) or V,
+    // with 2 warps K then V
+    constexpr int kJobs = kWDecWarps == 4 ? 1 : 2;
+    const int i = tid - kWSoftWarps * 32;
     const int r = i & 63;
-    const bool is_v = i >= 64;
+    const int kv0 = kWDecWarps == 4 ? (i >> 6) : 0;
     const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
-    uint8_t *tile0 = smem + (is_v ? kWV : kWK);
-    float *nrm0 = reinterpret_cast<float *>(smem + (is_v ? kWVN : kWKN));
     bool ok = true;
     uint32_t T = 0;
     int cur_page = -1, cur_h = -1, cur_u = -1;
-    const uint32_t *cw = nullptr;
-    const __half *nw = nullptr;
+    const uint32_t *cw[kJobs];
+    const __half *nw[kJobs];
     for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &wk, int t0, bool, bool, bool) {
-      if (T % kWDecGroups == static_cast<uint32_t>(grp)) {
-        const uint32_t st = T % kWStages;
-        uint8_t *tile = tile0 + st * kWStageBytes;
-        float *nrm_out = nrm0 + st * kWTok;
-        if (wk.j != cur_page || wk.h != cur_h || wk.u != cur_u) {
-          cur_page = wk.j;
-          cur_h = wk.h;
-          cur_u = wk.u;
-          int phys = -1;
-          if (wk.j < p.max_pages) phys = p.page_table[static_cast<int64_t>(wk.b) * p.max_pages + wk.j];
-          if (phys < 0 || phys >= p.num_pages) {
-            if (i == 0) set_status(p.status, ISOQUANT_DEVERR_PAGE_RANGE);
-            phys = 0;
-          }
-          const int64_t blk = (static_cast<int64_t>(phys) * 2 + (is_v ? 1 : 0)) * p.H + wk.h;
-          cw = p.codes + blk * words_for(BITS) * ps;
-          nw = reinterpret_cast<const __half *>(p.norms) + blk * ps;
+      const uint32_t st = T % kWStages;
+      if (wk.j != cur_page || wk.h != cur_h || wk.u != cur_u) {
+        cur_page = wk.j;
+        cur_h = wk.h;
+        cur_u = wk.u;
+        int phys = -1;
+        if (wk.j < p.max_pages) phys = p.page_table[static_cast<int64_t>(wk.b) * p.max_pages + wk.j];
+        if (phys < 0 || phys >= p.num_pages) {
+          if (i == 0) set_status(p.status, ISOQUANT_DEVERR_PAGE_RANGE);
+          phys = 0;
         }
-        // the code words are loaded first: their latency overlaps the wait
-        // for stage st, free once the P.V of tile T - kWStages has completed
-        const int t = t0 + r;
-        uint32_t x[words_for(BITS)];
-        load_token_words<BITS>(cw, ps, t, x);
-        const __half nh = nw[t];
-        if (T >= kWStages)
-          ok = mbar_wait<4096>(&kv_free[st], ((T / kWStages) + 1u) & 1u, p.status, abort_flag) && ok;
-        if (ok) {
-          const float nrm = __half2float(nh);
-          uint32_t out[64];
-          decode_token_words<BITS>(x, lane4, out);
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            *reinterpret_cast<uint4 *>(tile + canon_off(r, 8 * c, 2048)) =
-                make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
-          nrm_out[r] = nrm;
+        for (int jb = 0; jb < kJobs; ++jb) {
+          const int64_t blk = (static_cast<int64_t>(phys) * 2 + kv0 + jb) * p.H + wk.h;
+          cw[jb] = p.codes + blk * words_for(BITS) * ps;
+          nw[jb] = reinterpret_cast<const __half *>(p.norms) + blk * ps;
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(&kv_full[st]);
       }
+      // the code words are loaded first: their latency overlaps the wait
+      // for stage st, free once the P.V of tile T - kWStages has completed
+      const int t = t0 + r;
+      uint32_t x[kJobs][words_for(BITS)];
+      __half nh[kJobs];
+#pragma unroll
+      for (int jb = 0; jb < kJobs; ++jb) {
+        load_token_words<BITS>(cw[jb], ps, t, x[jb]);
+        nh[jb] = nw[jb][t];
+      }
+      if (T >= kWStages)
+        ok = mbar_wait<4096>(&kv_free[st], ((T / kWStages) + 1u) & 1u, p.status, abort_flag) && ok;
+      if (ok) {
+#pragma unroll
+        for (int jb = 0; jb < kJobs; ++jb) {
+          const bool is_v = kv0 + jb == 1;
+          uint8_t *tile = smem + (is_v ? kWV : kWK) + st * kWStageBytes;
+          // two halves of 64 dims, so that only 32 decoded words are live
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t out[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) out[q] = decode_pair<BITS>(x[jb], lane4, 32 * hh + q);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4 *>(tile + canon_off(r, 64 * hh + 8 * c, 2048)) =
+                  make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+          }
+          reinterpret_cast<float *>(smem + (is_v ? kWVN : kWKN))[st * kWTok + r] = __half2float(nh[jb]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&kv_full[st]);
       ++T;
     });
   } else {
     // ------------------------------------------------------------- softmax
-    // thread (r, hf): row r of the stream (tensor-memory lane r), tokens
-    // 32 hf .. 32 hf + 31 of each tile, Q~ dims and O columns 64 hf ..
-    // 64 hf + 63
-    const int r = tid & (kWRows - 1), hf = tid >> 7;
+    // thread (r, part): row r of the stream (tensor-memory lane r), tokens
+    // kWTpt * part .. + kWTpt - 1 of each tile, Q~ dims and O columns
+    // kWDpt * part .. + kWDpt - 1
+    const int r = tid & (kWRows - 1), part = tid >> 7;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);  // this warp's lanes
-    float *red = reinterpret_cast<float *>(smem + kWRed);  // [2 tiles][2 halves][128 rows]
+    float *red = reinterpret_cast<float *>(smem + kWRed);
+    float *rl = red + 2 * kWParts * kWRows;  // [part][row]: sums
+    float *rq = red + 3 * kWParts * kWRows;  // [part][row]: |q| maxima
+    constexpr int kSoftThreads = kWParts * kWRows;
     bool ok = true;
     uint32_t T = 0;
-    float m_run = -INFINITY, l_half = 0.f, rs = 1.f;
+    float m_run = -INFINITY, l_part = 0.f, rs = 1.f;
     int lim = 0;
     bool row_valid = false;
-    // this thread's 64 dims of row r of stream (wk.rg, wk.b, wk.h)
+    // this thread's dims of row r of stream (wk.rg, wk.b, wk.h)
     auto q_row = [&](const UWalk &wk) {
       const int row = wk.rg * kWRows + r;
       const bool valid = row < p.R;
       const int qi = valid ? row / p.G : 0;
       const int hq = wk.h * p.G + (valid ? row % p.G : 0);
-      return p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD + 64 * hf;
+      return p.q_rot + ((static_cast<int64_t>(wk.b) * p.nq + qi) * p.Hq + hq) * kD + kWDpt * part;
     };
     // Q~ of a stream into tensor memory (high parts, low parts), each row
     // prescaled by a power of two so that its largest |q| lands in
     // [2^14, 2^15); sets rs and releases the MMA warp.  The thread reads its
-    // 64 dims (16 independent 16-byte loads), takes the row's maximum with
-    // its partner and reads them again from L1 to convert them.  Called
-    // when no S of the previous stream is pending.
+    // dims (independent 16-byte loads), takes the row's maximum with its
+    // partners and reads them again from L1 to convert them.  Called when no
+    // S of the previous stream is pending.
     auto build_q = [&](const UWalk &wk) {
       const bool valid = wk.rg * kWRows + r < p.R;
       const float4 *qp = reinterpret_cast<const float4 *>(q_row(wk));
       float mx = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < kWDpt / 4; ++c) {
         const float4 v = valid ? __ldg(qp + c) : make_float4(0.f, 0.f, 0.f, 0.f);
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
       }
-      float *rq = red + 6 * kWRows;  // [2 halves][128 rows]
-      rq[hf * kWRows + r] = mx;
-      named_bar_sync(1, 2 * kWRows);
-      mx = fmaxf(rq[r], rq[kWRows + r]) * p.qfold;
+      rq[part * kWRows + r] = mx;
+      named_bar_sync(1, kSoftThreads);
+      mx = 0.f;
+#pragma unroll
+      for (int q = 0; q < kWParts; ++q) mx = fmaxf(mx, rq[q * kWRows + r]);
+      mx *= p.qfold;
       int ex = 0;
       if (mx > 0.f) frexpf(mx, &ex);
       ex = max(ex, -100);
       const float up = ldexpf(1.f, 15 - ex) * p.qfold;
       rs = ldexpf(1.f, ex - 15);
 #pragma unroll
-      for (int c16 = 0; c16 < 2; ++c16) {
-        // dims 64 hf + 32 c16 .. + 31: 16 packed columns of each part
+      for (int c16 = 0; c16 < kWDpt / 32; ++c16) {
+        // dims kWDpt part + 32 c16 .. + 31: 16 packed columns of each part
         uint32_t wh[16], wl[16];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -1801,8 +1848,8 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
           wl[2 * e] = pack_half2(a0 - f0.x, a1 - f0.y);
           wl[2 * e + 1] = pack_half2(a2 - f1.x, a3 - f1.y);
         }
-        tmem_st16u(tl + kWColQh + 32 * hf + 16 * c16, wh);
-        tmem_st16u(tl + kWColQl + 32 * hf + 16 * c16, wl);
+        tmem_st16u(tl + kWColQh + (kWDpt / 2) * part + 16 * c16, wh);
+        tmem_st16u(tl + kWColQl + (kWDpt / 2) * part + 16 * c16, wl);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
@@ -1820,7 +1867,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         const int L = p.seq_lens[wk.b];
         lim = row_valid ? (p.causal ? L - p.nq + row / p.G + 1 : L) : 0;
         m_run = -INFINITY;
-        l_half = 0.f;
+        l_part = 0.f;
       }
       if (last && more) {
         // the next stream: its queries are fetched into L2 now, so that
@@ -1829,25 +1876,25 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         nx.next_block(p, kWRows);
         const char *qn = reinterpret_cast<const char *>(q_row(nx));
         if (nx.rg * kWRows + r < p.R) {
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(qn));
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(qn + 128));
+#pragma unroll
+          for (int ln = 0; ln < kWDpt * 4; ln += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(qn + ln));
         }
       }
-      // ---- scores of tile T, this thread's 32 tokens
+      // ---- scores of tile T, this thread's tokens
       ok = mbar_wait<4096>(&s_full[sb], (T >> 1) & 1u, p.status, abort_flag) && ok;
       tc_fence_after();
-      float sv[32];
-      tmem_ld32(tl + kWColS + 64 * sb + 32 * hf, sv);
+      float sv[kWTpt];
+      tmem_ld_n(tl + kWColS + 64 * sb + kWTpt * part, sv);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
-      const float *kn = reinterpret_cast<const float *>(smem + kWKN) + st * kWTok + 32 * hf;
-      const float *vn = reinterpret_cast<const float *>(smem + kWVN) + st * kWTok + 32 * hf;
-      const int pos0 = wk.j * ps + t0 + 32 * hf;
-      const bool masked = __any_sync(0xffffffffu, pos0 + 32 > lim);
+      const float *kn = reinterpret_cast<const float *>(smem + kWKN) + st * kWTok + kWTpt * part;
+      const float *vn = reinterpret_cast<const float *>(smem + kWVN) + st * kWTok + kWTpt * part;
+      const int pos0 = wk.j * ps + t0 + kWTpt * part;
+      const bool masked = __any_sync(0xffffffffu, pos0 + kWTpt > lim);
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four chains, not one
 #pragma unroll
-      for (int t = 0; t < 32; t += 4) {
+      for (int t = 0; t < kWTpt; t += 4) {
         const float4 k4 = *reinterpret_cast<const float4 *>(kn + t);
         const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
@@ -1858,20 +1905,23 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
           mx4[e] = fmaxf(mx4[e], x);
         }
       }
-      // the row's maximum over both halves (exchange buffer alternates by tile)
-      float *rt = red + sb * (2 * kWRows);
-      rt[hf * kWRows + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      named_bar_sync(1, 2 * kWRows);
-      const float m_new = fmaxf(m_run, fmaxf(rt[r], rt[kWRows + r]) * rs);
+      // the row's maximum over the parts (exchange buffer alternates by tile)
+      float *rt = red + sb * (kWParts * kWRows);
+      rt[part * kWRows + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      named_bar_sync(1, kSoftThreads);
+      float mt = rt[r];
+#pragma unroll
+      for (int q = 1; q < kWParts; ++q) mt = fmaxf(mt, rt[q * kWRows + r]);
+      const float m_new = fmaxf(m_run, mt * rs);
       const float corr = (m_run == -INFINITY || m_new == m_run) ? 1.f : ex2(m_run - m_new);
       const float mm = m_new == -INFINITY ? 0.f : m_new;
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};
       // P' into tensor-memory buffer sb (its last reader, the P.V of tile
       // T - 2, has completed: this thread waited for it at tile T - 1 or at
       // the end of the previous stream)
-      uint32_t ph[16], pl[16];
+      uint32_t ph[kWTpt / 2], pl[kWTpt / 2];
 #pragma unroll
-      for (int t = 0; t < 32; t += 8) {
+      for (int t = 0; t < kWTpt; t += 8) {
         const float4 va = *reinterpret_cast<const float4 *>(vn + t);
         const float4 vb = *reinterpret_cast<const float4 *>(vn + t + 4);
         const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
@@ -1890,17 +1940,17 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
           pl[(t + e) >> 1] = pack_half2(w[e] - h0, w[e + 1] - h1);
         }
       }
-      tmem_st16u(tl + kWColP + 64 * sb + 16 * hf, ph);
-      tmem_st16u(tl + kWColP + 64 * sb + 32 + 16 * hf, pl);
+      tmem_st_n(tl + kWColP + 64 * sb + (kWTpt / 2) * part, ph);
+      tmem_st_n(tl + kWColP + 64 * sb + 32 + (kWTpt / 2) * part, pl);
       // O is still accumulated by the previous tile's P.V; this thread
-      // rescales O columns 64 hf .. 64 hf + 63 of its row
+      // rescales its O columns of its row
       if (!first) {
         ok = mbar_wait<4096>(pv_done, (T - 1u) & 1u, p.status, abort_flag) && ok;
         tc_fence_after();
         if (__any_sync(0xffffffffu, corr != 1.f)) {
-          const uint32_t to = tl + kWColO + 64 * hf;
+          const uint32_t to = tl + kWColO + kWDpt * part;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < kWDpt / 32; ++c) {
             float ov[32];
             tmem_ld32(to + 32 * c, ov);
 #pragma unroll
@@ -1910,7 +1960,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         }
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      l_half = l_half * corr + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
+      l_part = l_part * corr + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
       m_run = m_new;
       tc_fence_before();
       __syncwarp();
@@ -1926,25 +1976,27 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
           nx.next_block(p, kWRows);
           build_q(nx);
         }
-        float *rl = red + 4 * kWRows;  // [2 halves][128 rows]
-        rl[hf * kWRows + r] = l_half;
-        named_bar_sync(1, 2 * kWRows);
+        rl[part * kWRows + r] = l_part;
+        named_bar_sync(1, kSoftThreads);
         const int64_t stream = static_cast<int64_t>(wk.u) * p.H + wk.h;
         float *rec = p.records + ((blockIdx.x + stream) * (kWRows / 8) + (r >> 3)) * static_cast<int64_t>(kRecordFloats);
         const int rr = r & 7;
-        if (row_valid && hf == 0) {
-          rec[2 * rr] = m_run;
-          rec[2 * rr + 1] = rl[r] + rl[kWRows + r];
-        }
-        const uint32_t to = tl + kWColO + 64 * hf;
+        if (row_valid && part == 0) {
+          float l = 0.f;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+          for (int q = 0; q < kWParts; ++q) l += rl[q * kWRows + r];
+          rec[2 * rr] = m_run;
+          rec[2 * rr + 1] = l;
+        }
+        const uint32_t to = tl + kWColO + kWDpt * part;
+#pragma unroll
+        for (int c = 0; c < kWDpt / 32; ++c) {
           float ov[32];
           tmem_ld32(to + 32 * c, ov);
           if (row_valid) {
 #pragma unroll
             for (int k = 0; k < 32; k += 4)
-              *reinterpret_cast<float4 *>(rec + 16 + rr * kD + 64 * hf + 32 * c + k) =
+              *reinterpret_cast<float4 *>(rec + 16 + rr * kD + kWDpt * part + 32 * c + k) =
                   make_float4(ov[k], ov[k + 1], ov[k + 2], ov[k + 3]);
           }
         }
