@@ -2021,22 +2021,33 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
 // SM has room, and wait there for the partial kernel to complete.
 constexpr int kCombineThreads = 128;
 
+// One warp per NR consecutive query heads of a (sequence, position): NR
+// divides the GQA group (up to 8), so the rows share a KV head, a stream and
+// a record, and their loads overlap in one merge.
+template <int NR>
 __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const CombineParams p) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
-  const uint32_t row_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint32_t n_rows = static_cast<uint32_t>(p.B) * p.nq * p.Hq;
-  if (row_id >= n_rows) return;
-  const int hq = static_cast<int>(row_id % static_cast<uint32_t>(p.Hq));
-  const uint32_t bi = row_id / static_cast<uint32_t>(p.Hq);
+  const uint32_t grp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t per_bi = static_cast<uint32_t>(p.Hq / NR);
+  const uint32_t n_groups = static_cast<uint32_t>(p.B) * p.nq * per_bi;
+  if (grp_id >= n_groups) return;
+  const int hq0 = static_cast<int>(grp_id % per_bi) * NR;
+  const uint32_t bi = grp_id / per_bi;
   const int i = static_cast<int>(bi % static_cast<uint32_t>(p.nq));
   const int b = static_cast<int>(bi / static_cast<uint32_t>(p.nq));
-  const int h = hq / p.G, g = hq % p.G;
+  const int h = hq0 / p.G, gq = hq0 % p.G;
   // stream rg holds rows rg * rps .. ; record `sub` of a CTA holds 8 of them
-  const int r = i * p.G + g, rg = r / p.rps, sub = (r % p.rps) >> 3, rr = r & 7;
+  const int r0 = i * p.G + gq, rg = r0 / p.rps, sub = (r0 % p.rps) >> 3;
   const int ps = p.page_size;
-  float *dst = p.out + static_cast<int64_t>(row_id) * kD + 4 * lane;
+  int rows[NR];
+  float *dsts[NR];
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    rows[k] = (r0 + k) & 7;
+    dsts[k] = p.out + (static_cast<int64_t>(bi) * p.Hq + hq0 + k) * kD + 4 * lane;
+  }
 
   int np;
   int64_t g0, total;
@@ -2055,15 +2066,14 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
     g0 = rg * p_rg + static_cast<int64_t>(p.H) * pages_before(p.seq_lens, b, ps, lane) + static_cast<int64_t>(h) * np;
   }
   if (np == 0) {
-    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < NR; ++k) *reinterpret_cast<float4 *>(dsts[k]) = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
   const int64_t N = p.n_cta;
   const int64_t c_lo = cta_of_page(g0, N, total), c_hi = cta_of_page(g0 + np - 1, N, total);
   const int64_t pair = (static_cast<int64_t>(rg) * p.B + b) * p.H + h;
-  const int rows[1] = {rr};
-  float *const dsts[1] = {dst};
-  merge_rows<1>(p.records, pair, p.rps >> 3, sub, c_lo, c_hi, N, total, rows, dsts, p.params[h], lane);
+  merge_rows<NR>(p.records, pair, p.rps >> 3, sub, c_lo, c_hi, N, total, rows, dsts, p.params[h], lane);
 }
 
 }  // namespace
@@ -2230,10 +2240,23 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
     p.vpages = t.vpages;
     p.prefix = reinterpret_cast<const int64_t *>(static_cast<const char *>(ws) + t.prefix_off);
   }
-  const int64_t rows = static_cast<int64_t>(s.batch) * s.nq * s.q_heads;
-  const int64_t blocks = (rows * 32 + kCombineThreads - 1) / kCombineThreads;
+  // rows per warp: one while there are few rows (decode: a row's merge has
+  // many split records, and more warps overlap more of them); with many
+  // rows (prefill: one or two records each), the largest of 8, 4, 2 that
+  // divides the GQA group, so a warp's rows overlap their loads
+  const int64_t n_rows = static_cast<int64_t>(s.batch) * s.nq * s.q_heads;
+  const bool many = n_rows >= static_cast<int64_t>(64) * ctx->num_sms;
+  const int nr = !many ? 1 : s.group % 8 == 0 ? 8 : s.group % 4 == 0 ? 4 : s.group % 2 == 0 ? 2 : 1;
+  const int64_t warps = static_cast<int64_t>(s.batch) * s.nq * (s.q_heads / nr);
+  const int64_t blocks = (warps * 32 + kCombineThreads - 1) / kCombineThreads;
   if (blocks == 0) return cudaSuccess;
-  return launch_pdl(k_attend_combine, dim3(static_cast<unsigned>(blocks)), dim3(kCombineThreads), 0, stream, p);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(kCombineThreads);
+  switch (nr) {
+    case 8: return launch_pdl(k_attend_combine<8>, grid, block, 0, stream, p);
+    case 4: return launch_pdl(k_attend_combine<4>, grid, block, 0, stream, p);
+    case 2: return launch_pdl(k_attend_combine<2>, grid, block, 0, stream, p);
+    default: return launch_pdl(k_attend_combine<1>, grid, block, 0, stream, p);
+  }
 }
 
 }  // namespace isoquant

@@ -485,3 +485,21 @@ def test_tcgen05_rows_kernel_matches_mma_path(cuda_lib, case):
         if st.seq_lens[b] == 0:
             continue
         check_pair(st, b, (b * 3) % st.H, qc, tiles)
+
+
+@pytest.mark.parametrize("hq,h,nq,L", [(32, 8, 300, 400), (32, 4, 300, 350), (16, 8, 600, 700)])
+def test_combine_grouped_rows(cuda_lib, hq, h, nq, L):
+    """With many output rows (at least 64 per SM) the combine kernel merges
+    the rows of a GQA group (8, 4 or 2 of them) in one warp; every row still
+    matches the oracle."""
+    from compressed_space_decode_b200.synthetic import Workload
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert nq * hq >= 64 * n_sms
+    wl = Workload("grouped", 1, hq, h, [L], nq=nq, page_size=64, causal=True, seed=70 + hq // h)
+    st = DecodeState(wl)
+    q, _, out = run_attend(csd, st)
+    assert torch.isfinite(out).all()
+    for hh in (0, st.H - 1):
+        check_pair(st, 0, hh, q, out)
