@@ -291,7 +291,7 @@ def isoquant_attend_decode(ctx, cache, q_rot, page_table, seq_lens, workspace, o
 def isoquant_attend_decode_static(ctx, cache, q_rot, page_table, seq_lens, out, causal=False, scale=0.0,
                                   stream=None):
     """isoquant_attend_decode for callers that cannot allocate device memory
-    or lend a workspace: the split records go to a fixed 8 MiB array inside
+    or lend a workspace: the split records go to a fixed 16 MiB array inside
     the library.  Its first call on a device must precede any stream
     capture; calls that overlap on the GPU race on the shared array."""
     B, nq, Hq, maxp = _attend_args(q_rot, page_table, seq_lens)

@@ -9,7 +9,7 @@
 // partial records of the split-context attention live in a fixed array
 // compiled into the library.
 //
-// The array is a file-scope __device__ variable of kScratchBytes (8 MiB):
+// The array is a file-scope __device__ variable of kScratchBytes (16 MiB):
 // every GPU that loads the library holds it until the process exits.  In
 // host code its name is only a host-side stand-in, so the device address is
 // looked up with cudaGetSymbolAddress, once per device, with that device
@@ -28,7 +28,7 @@
 namespace isoquant {
 namespace {
 
-constexpr size_t kScratchBytes = size_t(8) << 20;
+constexpr size_t kScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -233,8 +233,8 @@ int isoquant_decode_step(isoquant_ctx *ctx, const isoquant_cache *cache,
  * must not risk the device-wide synchronisation of cudaMalloc/cudaFree).
  * The paper has no counterpart to this call; it is a deployment aid.
  * Same arguments and result as isoquant_attend_decode.  The split records
- * live in an 8 MiB array compiled into the library (held by every GPU that
- * loads it until exit); a shape whose minimum workspace exceeds 8 MiB
+ * live in a 16 MiB array compiled into the library (held by every GPU that
+ * loads it until exit); a shape whose minimum workspace exceeds 16 MiB
  * is rejected with ISOQUANT_ERR_WORKSPACE.  The first call on a device looks
  * up the array's device address and must come before any stream capture.
  * Calls share the array: calls whose kernels overlap on the GPU race and

@@ -82,3 +82,54 @@ def test_small_pages_are_unsupported_below_3_bits(cuda_lib):
     with pytest.raises(csd.IsoquantError) as e:
         csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, _ws(csd, st), out)
     assert e.value.status == -2
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_decode_step_and_static_entry(cuda_lib, bits):
+    """The one-call step (append + rotate in one launch, then attention) and
+    the allocation-free entry give the separate calls' results at 2 and 4
+    bits."""
+    from compressed_space_decode_b200.synthetic import Workload
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    wl = Workload("step", 2, 16, 4, [300, 129], nq=16, page_size=64, causal=True, seed=65)
+    sa, sb = DecodeState(wl, growth=16, bits=bits), DecodeState(wl, growth=16, bits=bits)
+    k = torch.stack([sa.kv_tokens(b, sa.seq_lens[b], sa.seq_lens[b] + 16)[0] for b in range(sa.B)], 1)
+    v = torch.stack([sa.kv_tokens(b, sa.seq_lens[b], sa.seq_lens[b] + 16)[1] for b in range(sa.B)], 1)
+    k, v = k.reshape(-1, sa.H, D).contiguous(), v.reshape(-1, sa.H, D).contiguous()
+    slots = sa.slot_matrix(sa.seq_lens, 16).reshape(-1).contiguous()
+    for st in (sa, sb):
+        st.seq_lens = [L + 16 for L in st.seq_lens]
+        st.seq_lens_dev += 16
+    q = sa.queries(0)
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    out_a = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    csd.isoquant_compress_kv(sa.ctx, sa.cache, k, v, slots)
+    csd.isoquant_rotate_q(sa.ctx, q.reshape(-1, sa.Hq, D), q_rot.view(-1, sa.Hq, D))
+    csd.isoquant_attend_decode(sa.ctx, sa.cache, q_rot, sa.page_table, sa.seq_lens_dev, _ws(csd, sa), out_a,
+                               causal=True)
+    out_b = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    ws_b = csd.alloc_step_workspace(sb.ctx, sb.B, 16, sb.Hq).fill_(0x7FC00000)
+    csd.isoquant_decode_step(sb.ctx, sb.cache, k, v, slots, q.contiguous(), sb.page_table, sb.seq_lens_dev, ws_b,
+                             out_b, causal=True)
+    out_c = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    csd.isoquant_attend_decode_static(sa.ctx, sa.cache, q_rot, sa.page_table, sa.seq_lens_dev, out_c, causal=True)
+    torch.cuda.synchronize()
+    assert csd.isoquant_get_status(sa.ctx) == 0 and csd.isoquant_get_status(sb.ctx) == 0
+    assert torch.equal(sa.cache.codes, sb.cache.codes) and torch.equal(sa.cache.norms, sb.cache.norms)
+    assert torch.equal(out_a, out_b)
+    assert torch.equal(out_a, out_c)
+
+
+def test_init_bits_rejects_other_widths(cuda_lib):
+    from compressed_space_decode_b200 import synthetic
+    csd = cuda_lib
+    signs, quats = synthetic.rotation_params(3, 2)
+    for bits in (1, 5, 8):
+        with pytest.raises(csd.IsoquantError) as e:
+            csd.isoquant_init(signs, quats, bits=bits)
+        assert e.value.status == -2
+    ctx = csd.isoquant_init(signs, quats, bits=2)
+    code_bytes, norm_bytes = csd.isoquant_cache_bytes(ctx, 3, 64)
+    assert code_bytes == 3 * 2 * 2 * 8 * 64 * 4 and norm_bytes == 3 * 2 * 2 * 64 * 2
+    ctx.close()

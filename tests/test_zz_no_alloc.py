@@ -51,7 +51,7 @@ def test_static_entry_rejects_oversized_shapes(cuda_lib):
     signs, quats = synthetic.rotation_params(3, 8)
     ctx = csd.isoquant_init(signs, quats)
     cache = csd.PagedCache.allocate(8, 1, 256)
-    # 2048 sequences x 8 KV heads of records need far more than 8 MiB
+    # 2048 sequences x 8 KV heads of records need far more than 16 MiB
     q_rot = torch.zeros((2048, 1, 8, 128), dtype=torch.float32, device="cuda")
     pt = torch.zeros((2048, 1), dtype=torch.int32, device="cuda")
     lens = torch.ones(2048, dtype=torch.int32, device="cuda")
