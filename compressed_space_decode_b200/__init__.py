@@ -35,7 +35,7 @@ SYMBOLS = [
     "isoquant_compress_kv", "isoquant_rotate_q", "isoquant_workspace_size", "isoquant_attend_decode",
     "isoquant_attend_partial", "isoquant_attend_combine", "isoquant_get_status", "isoquant_last_launch_count",
     "isoquant_attend_decode_static", "isoquant_decode_prep", "isoquant_step_workspace_size",
-    "isoquant_decode_step", "isoquant_init_bits", "isoquant_codebook_bits",
+    "isoquant_decode_step", "isoquant_init_bits", "isoquant_codebook_bits", "isoquant_selftest_wait",
 ]
 
 
@@ -84,6 +84,7 @@ def lib():
             "isoquant_step_workspace_size": ([vp, i32, i32, i32, ctypes.POINTER(sz)], i32),
             "isoquant_decode_step": ([vp, cp, vp, vp, i32, vp, vp, i32, i32, i32, i32, vp, i32, vp, i32,
                                       ctypes.c_float, vp, sz, vp, vp], i32),
+            "isoquant_selftest_wait": ([vp, ctypes.c_uint64, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -322,6 +323,19 @@ def isoquant_get_status(ctx, stream=None):
     s = ctypes.c_uint32()
     _check(lib().isoquant_get_status(ctx.handle, ctypes.byref(s), _stream(stream)), "isoquant_get_status")
     return s.value
+
+
+def isoquant_selftest_wait(ctx, limit_ns, elapsed=None, stream=None):
+    """Run the bounded-wait self-test: one device thread waits on a barrier
+    that nothing completes and gives up after limit_ns, raising the timeout
+    bit of the status word.  elapsed: optional int64 device tensor of one
+    element that receives the measured wait in nanoseconds."""
+    ptr = ctypes.c_void_p(0)
+    if elapsed is not None:
+        assert elapsed.dtype == torch.int64 and elapsed.numel() >= 1
+        ptr = _ptr(elapsed)
+    _check(lib().isoquant_selftest_wait(ctx.handle, int(limit_ns), ptr, _stream(stream)),
+           "isoquant_selftest_wait")
 
 
 def isoquant_last_launch_count(ctx):

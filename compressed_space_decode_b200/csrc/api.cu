@@ -163,6 +163,9 @@ int dtype_bytes(int dtype) {
 
 using namespace isoquant;
 
+// longest wait isoquant_selftest_wait accepts (10 s)
+static constexpr uint64_t kSelftestMaxNs = 10000000000ull;
+
 extern "C" {
 
 const char *isoquant_strerror(int status) {
@@ -439,5 +442,13 @@ int isoquant_get_status(isoquant_ctx *ctx, uint32_t *status, void *stream) {
 }
 
 int isoquant_last_launch_count(const isoquant_ctx *ctx) { return ctx ? ctx->last_launches : 0; }
+
+int isoquant_selftest_wait(isoquant_ctx *ctx, uint64_t limit_ns, uint64_t *elapsed_ns, void *stream) {
+  if (ctx == nullptr || limit_ns == 0 || limit_ns > kSelftestMaxNs) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 1;
+  return launch_wait_selftest(ctx, limit_ns, elapsed_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? ISOQUANT_OK
+             : ISOQUANT_ERR_CUDA;
+}
 
 }  // extern "C"

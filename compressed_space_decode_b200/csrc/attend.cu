@@ -78,7 +78,8 @@ constexpr int kLocate = kBarriers + 2 * kStages * 8;
 constexpr int kSmemBytes = kLocate + 64;
 static_assert(kStageBytes % 16 == 0, "stage alignment");
 
-constexpr uint32_t kSpinLimit = 1u << 25;
+constexpr uint32_t kSpinLimit = 1u << 25;  // polls (a backstop: the time limit ends a wait first)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct PartialParams {
   const uint32_t *codes;
@@ -130,19 +131,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: gives up after kSpinLimit polls, raising the timeout bit.
-// It spins (try_wait itself suspends briefly) for the first kSpin polls and
-// then backs off with __nanosleep.  A sleeping waiter wakes late, which costs
-// a hand-off between warp-specialised roles hundreds of cycles (those spin
-// long); where many threads of a CTA wait together, spinning takes issue
-// slots from the CTA beside it (those back off early).
-template <uint32_t kSpin = 64>
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended until the phase completes or `ns` nanoseconds pass, so a waiting
+// warp neither takes issue slots from the working ones nor wakes late.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t *bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: polls with a 1 us suspend hint (the hardware resumes the
+// thread as soon as the phase completes) and gives up after limit_ns,
+// raising the timeout bit, or as soon as another thread of the CTA has
+// raised the abort flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
-                                          volatile int *abort_flag) {
+                                          volatile int *abort_flag, uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_for(bar, parity, 1000u)) return true;
     if (abort_flag != nullptr && *abort_flag) return false;
-    if (i > kSpin) __nanosleep(64);
+    if (global_ns() - t0 > limit_ns) break;
   }
   set_status(status, ISOQUANT_DEVERR_WAIT_TIMEOUT);
   if (abort_flag != nullptr) *abort_flag = 1;
@@ -1663,7 +1680,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
       uint32_t T = 0, seg = 0, prev_T = 0;
       bool have_prev = false, prev_first = false;
       auto issue_pv = [&](uint32_t t, bool first) {
-        ok = mbar_wait<4096>(p_full, t & 1u, p.status, abort_flag) && ok;
+        ok = mbar_wait(p_full, t & 1u, p.status, abort_flag) && ok;
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (!ok) return;
@@ -1680,9 +1697,9 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
       };
       for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &, int, bool first, bool last, bool) {
         const uint32_t st = T % kWStages, sb = T & 1u;
-        if (first) ok = mbar_wait<4096>(q_full, seg & 1u, p.status, abort_flag) && ok;
-        ok = mbar_wait<4096>(&kv_full[st], (T / kWStages) & 1u, p.status, abort_flag) && ok;
-        if (T >= 2) ok = mbar_wait<4096>(&s_free[sb], ((T >> 1) + 1u) & 1u, p.status, abort_flag) && ok;
+        if (first) ok = mbar_wait(q_full, seg & 1u, p.status, abort_flag) && ok;
+        ok = mbar_wait(&kv_full[st], (T / kWStages) & 1u, p.status, abort_flag) && ok;
+        if (T >= 2) ok = mbar_wait(&s_free[sb], ((T >> 1) + 1u) & 1u, p.status, abort_flag) && ok;
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (ok) {
@@ -1757,7 +1774,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         nh[jb] = nw[jb][t];
       }
       if (T >= kWStages)
-        ok = mbar_wait<4096>(&kv_free[st], ((T / kWStages) + 1u) & 1u, p.status, abort_flag) && ok;
+        ok = mbar_wait(&kv_free[st], ((T / kWStages) + 1u) & 1u, p.status, abort_flag) && ok;
       if (ok) {
 #pragma unroll
         for (int jb = 0; jb < kJobs; ++jb) {
@@ -1881,7 +1898,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         }
       }
       // ---- scores of tile T, this thread's tokens
-      ok = mbar_wait<4096>(&s_full[sb], (T >> 1) & 1u, p.status, abort_flag) && ok;
+      ok = mbar_wait(&s_full[sb], (T >> 1) & 1u, p.status, abort_flag) && ok;
       tc_fence_after();
       float sv[kWTpt];
       tmem_ld_n(tl + kWColS + 64 * sb + kWTpt * part, sv);
@@ -1945,7 +1962,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
       // O is still accumulated by the previous tile's P.V; this thread
       // rescales its O columns of its row
       if (!first) {
-        ok = mbar_wait<4096>(pv_done, (T - 1u) & 1u, p.status, abort_flag) && ok;
+        ok = mbar_wait(pv_done, (T - 1u) & 1u, p.status, abort_flag) && ok;
         tc_fence_after();
         if (__any_sync(0xffffffffu, corr != 1.f)) {
           const uint32_t to = tl + kWColO + kWDpt * part;
@@ -1969,7 +1986,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         // ---- end of the stream in this CTA: once its last P.V completed,
         // the next stream's Q~ goes in (so that the MMA warp starts on it
         // while the record is written), then the record: (m, l) and O
-        ok = mbar_wait<4096>(pv_done, T & 1u, p.status, abort_flag) && ok;
+        ok = mbar_wait(pv_done, T & 1u, p.status, abort_flag) && ok;
         tc_fence_after();
         if (more) {
           UWalk nx = wk;
@@ -2009,7 +2026,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
-    if (*mma_issued) mbar_wait<4096>(mma_done, 0, p.status, nullptr);
+    if (*mma_issued) mbar_wait(mma_done, 0, p.status, nullptr);
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kWCols));
   }
@@ -2257,6 +2274,27 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
     case 2: return launch_pdl(k_attend_combine<2>, grid, block, 0, stream, p);
     default: return launch_pdl(k_attend_combine<1>, grid, block, 0, stream, p);
   }
+}
+
+namespace {
+// Failure-path self-test: one thread waits on a barrier that nothing
+// arrives on, so the bounded wait runs out after limit_ns, raises the
+// timeout bit and returns; the elapsed time goes to *elapsed_ns.
+__global__ void k_wait_selftest(uint32_t *status, uint64_t limit_ns, uint64_t *elapsed_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  const uint64_t t0 = global_ns();
+  const bool done = mbar_wait(&bar, 0, status, nullptr, limit_ns);
+  if (elapsed_ns != nullptr) *elapsed_ns = done ? 0 : global_ns() - t0;
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(const isoquant_ctx *ctx, uint64_t limit_ns, uint64_t *elapsed_ns,
+                                 cudaStream_t stream) {
+  k_wait_selftest<<<1, 32, 0, stream>>>(ctx->status, limit_ns, elapsed_ns);
+  return cudaGetLastError();
 }
 
 }  // namespace isoquant

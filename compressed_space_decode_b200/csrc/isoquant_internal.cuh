@@ -93,6 +93,8 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
 cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
                                   const int32_t *seq_lens, const void *ws, size_t ws_bytes, float *out,
                                   cudaStream_t stream);
+cudaError_t launch_wait_selftest(const isoquant_ctx *ctx, uint64_t limit_ns, uint64_t *elapsed_ns,
+                                 cudaStream_t stream);
 
 // ------------------------------------------------------------ launch chain
 // Every kernel of the library is a programmatic dependent launch: it may be

@@ -268,6 +268,17 @@ int isoquant_get_status(isoquant_ctx *ctx, uint32_t *status, void *stream);
 /* Number of kernels the most recent call on this context launched. */
 int isoquant_last_launch_count(const isoquant_ctx *ctx);
 
+/* Self-test of the failure path.  Launches one thread that waits, through
+ * the same bounded wait the pipelines use, on a barrier that nothing
+ * completes: the wait gives up after limit_ns nanoseconds (1 ns .. 10 s,
+ * else ISOQUANT_ERR_INVALID_ARG), sets ISOQUANT_DEVERR_WAIT_TIMEOUT in the
+ * status word and the kernel returns; nothing faults and the context stays
+ * usable.  elapsed_ns (device, may be NULL) receives the measured wait in
+ * nanoseconds.  Asynchronous on stream; read the bit with
+ * isoquant_get_status. */
+int isoquant_selftest_wait(isoquant_ctx *ctx, uint64_t limit_ns,
+                           uint64_t *elapsed_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
