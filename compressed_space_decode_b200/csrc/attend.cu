@@ -1095,19 +1095,6 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
                : "memory");
 }
-// A in tensor memory (row m = lane m, column c = the packed fp16 pair
-// k = 2c, 2c + 1 of the 16-wide K slice starting at a_tmem), executed by a
-// converged warp and issued by the lane with `issue` set: the descriptor
-// arithmetic stays warp-uniform
-__device__ __forceinline__ void umma_ts_by(bool issue, uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                           uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%6, %7, %8, %9}, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(static_cast<uint32_t>(issue)), "r"(0u), "r"(0u), "r"(0u),
-      "r"(0u)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(
@@ -1130,6 +1117,80 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[1
           taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+// Products with A in tensor memory (row m = lane m, column c = the packed
+// fp16 pair k = 2c, 2c + 1 of a 16-wide K slice), issued by the calling
+// thread as one asm block.
+// The 16 score products of a tile (Q~ high parts, then low parts, against
+// the K tile at descriptor bK: 8 K-slices of 16 dims each) in one asm block,
+// issued by the calling thread: per product one address add, one descriptor
+// add and the MMA.
+__device__ __forceinline__ void umma_scores16(uint32_t d, uint32_t qh, uint32_t ql, uint64_t bK, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred pz, pa;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 pz, %5, 0;\n\tsetp.eq.b32 pa, %5, 0;\n\t"
+      "add.u32 a, %1, 0;\n\tadd.s64 b, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pz;\n\t"
+      "add.u32 a, %1, 8;\n\tadd.s64 b, %3, 16;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 16;\n\tadd.s64 b, %3, 32;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 24;\n\tadd.s64 b, %3, 48;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 32;\n\tadd.s64 b, %3, 64;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 40;\n\tadd.s64 b, %3, 80;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 48;\n\tadd.s64 b, %3, 96;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 56;\n\tadd.s64 b, %3, 112;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 0;\n\tadd.s64 b, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 8;\n\tadd.s64 b, %3, 16;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 16;\n\tadd.s64 b, %3, 32;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 24;\n\tadd.s64 b, %3, 48;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 32;\n\tadd.s64 b, %3, 64;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 40;\n\tadd.s64 b, %3, 80;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 48;\n\tadd.s64 b, %3, 96;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %2, 56;\n\tadd.s64 b, %3, 112;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, {%5, %5, %5, %5}, pa;\n\t"
+      "}\n"
+      ::"r"(d), "r"(qh), "r"(ql), "l"(bK), "r"(idesc), "r"(0u)
+      : "memory");
+}
+// The 8 products O (+)= P'V of a tile (P' high parts, then low parts, 4
+// token slices of 16 each, against the V tile at descriptor bV); acc0 = 0
+// starts O with the first one.
+__device__ __forceinline__ void umma_pv8(uint32_t d, uint32_t pa, uint64_t bV, uint32_t idesc, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, pa;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 p0, %4, 0;\n\tsetp.eq.b32 pa, %5, 0;\n\t"
+      "add.u32 a, %1, 0;\n\tadd.s64 b, %2, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, p0;\n\t"
+      "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 32;\n\tadd.s64 b, %2, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 40;\n\tadd.s64 b, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 48;\n\tadd.s64 b, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, pa;\n\t"
+      "add.u32 a, %1, 56;\n\tadd.s64 b, %2, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, {%5, %5, %5, %5}, pa;\n\t"
+      "}\n"
+      ::"r"(d), "r"(pa), "l"(bV), "r"(idesc), "r"(acc0), "r"(0u)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit_by(bool issue, uint64_t *bar) {
@@ -1552,7 +1613,11 @@ constexpr int kWTpt = kWTok / kWParts;  // tokens of a tile per softmax thread
 constexpr int kWDpt = kD / kWParts;     // Q~ dims / O columns per softmax thread
 // decoder warps: 4 (a thread decodes one token of K or V per tile) or 2 (a
 // thread decodes one token of K and of V), keeping registers in budget
-constexpr int kWDecWarps = kWParts == 2 ? 4 : 2;
+#ifndef ISOQUANT_WIDE_DEC
+#define ISOQUANT_WIDE_DEC 0
+#endif
+constexpr int kWDecWarps = ISOQUANT_WIDE_DEC ? ISOQUANT_WIDE_DEC : (kWParts == 2 ? 4 : 2);
+static_assert(kWDecWarps == 2 || kWDecWarps == 4, "two or four decoder warps");
 constexpr int kWMmaWarp = kWSoftWarps + kWDecWarps;
 constexpr int kWThreads = (kWMmaWarp + 1) * 32;
 // Tensor memory (512 columns, one CTA per SM): S buffers 0 and 1, O, then
@@ -1686,14 +1751,12 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         if (!ok) return;
         const uint64_t so = (t % kWStages) * static_cast<uint32_t>(kWStageBytes >> 4);
         const uint32_t pa = tmem + kWColP + (t & 1u) * 64;
-#pragma unroll
-        for (int kc = 0; kc < kWTok / 16; ++kc)
-          umma_ts_by(leader, tmem + kWColO, pa + kc * 8, dV + so + kc * 256, kIdescPV, (first && kc == 0) ? 0u : 1u);
-#pragma unroll
-        for (int kc = 0; kc < kWTok / 16; ++kc)
-          umma_ts_by(leader, tmem + kWColO, pa + 32 + kc * 8, dV + so + kc * 256, kIdescPV, 1u);
-        umma_commit_by(leader, pv_done);
-        umma_commit_by(leader, &kv_free[t % kWStages]);
+        if (leader) {
+          umma_pv8(tmem + kWColO, pa, dV + so, kIdescPV, first ? 0u : 1u);
+          umma_commit(pv_done);
+          umma_commit(&kv_free[t % kWStages]);
+        }
+        __syncwarp();
       };
       for_each_tile(p, gs, ge, u0, off0, [&](const UWalk &, int, bool first, bool last, bool) {
         const uint32_t st = T % kWStages, sb = T & 1u;
@@ -1705,13 +1768,11 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         if (ok) {
           const uint64_t so = st * static_cast<uint32_t>(kWStageBytes >> 4);
           const uint32_t d = tmem + kWColS + 64 * sb;
-#pragma unroll
-          for (int kc = 0; kc < kD / 16; ++kc)
-            umma_ts_by(leader, d, tmem + kWColQh + kc * 8, dK + so + kc * 16, kIdescS, kc > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kc = 0; kc < kD / 16; ++kc)
-            umma_ts_by(leader, d, tmem + kWColQl + kc * 8, dK + so + kc * 16, kIdescS, 1u);
-          umma_commit_by(leader, &s_full[sb]);
+          if (leader) {
+            umma_scores16(d, tmem + kWColQh, tmem + kWColQl, dK + so, kIdescS);
+            umma_commit(&s_full[sb]);
+          }
+          __syncwarp();
           *mma_issued = 1;
         }
         // the previous tile's P.V (same stream) after this tile's scores
@@ -1809,7 +1870,11 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
     float *red = reinterpret_cast<float *>(smem + kWRed);
     float *rl = red + 2 * kWParts * kWRows;  // [part][row]: sums
     float *rq = red + 3 * kWParts * kWRows;  // [part][row]: |q| maxima
-    constexpr int kSoftThreads = kWParts * kWRows;
+    // the parts of row r are warps r / 32 + 4 k, all on one SM sub-partition:
+    // their exchanges (row maxima, |q| maxima, sums) use one named barrier per
+    // lane quarter, so the four quarters do not wait on one another
+    const int xbar = 1 + (warp & 3);
+    constexpr int kXThreads = kWParts * 32;
     bool ok = true;
     uint32_t T = 0;
     float m_run = -INFINITY, l_part = 0.f, rs = 1.f;
@@ -1839,7 +1904,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
       }
       rq[part * kWRows + r] = mx;
-      named_bar_sync(1, kSoftThreads);
+      named_bar_sync(xbar, kXThreads);
       mx = 0.f;
 #pragma unroll
       for (int q = 0; q < kWParts; ++q) mx = fmaxf(mx, rq[q * kWRows + r]);
@@ -1925,7 +1990,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
       // the row's maximum over the parts (exchange buffer alternates by tile)
       float *rt = red + sb * (kWParts * kWRows);
       rt[part * kWRows + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      named_bar_sync(1, kSoftThreads);
+      named_bar_sync(xbar, kXThreads);
       float mt = rt[r];
 #pragma unroll
       for (int q = 1; q < kWParts; ++q) mt = fmaxf(mt, rt[q * kWRows + r]);
@@ -1994,7 +2059,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParam
           build_q(nx);
         }
         rl[part * kWRows + r] = l_part;
-        named_bar_sync(1, kSoftThreads);
+        named_bar_sync(xbar, kXThreads);
         const int64_t stream = static_cast<int64_t>(wk.u) * p.H + wk.h;
         float *rec = p.records + ((blockIdx.x + stream) * (kWRows / 8) + (r >> 3)) * static_cast<int64_t>(kRecordFloats);
         const int rr = r & 7;
