@@ -290,6 +290,11 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, budget_s=args.cpu_seconds, bits=args.bits)
+    # the library's kernel choice: mma.sync below 64 query rows per KV head
+    # (or with pages under 64 tokens), tcgen05 from there
+    rows = wl.nq * (Hq // H)
+    partial_kernel = ("k_attend_partial" if rows < 64 or st.ps < 64 else
+                      "k_attend_wide" if rows >= 128 else "k_attend_tiles")
 
     if world > 1:
         dist.barrier()
@@ -299,7 +304,8 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": ("f32 accumulate (3-bit codes -> f16 centroids, hi/lo f16 queries on mma.sync)" if args.bits == 3 else
+        "dtype": (f"f32 accumulate ({args.bits}-bit codes -> f16 centroids, hi/lo f16 queries on mma.sync)"
+                  if partial_kernel == "k_attend_partial" else
                   f"f32 accumulate ({args.bits}-bit codes -> f16 centroids, hi/lo f16 queries and weights on tcgen05)"),
         "data": "synthetic (seeded bf16 Student-t(4) K/V, log-uniform channel scales, x20 outliers)",
         "config": {"workload": wl.name.split("@")[0], "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
@@ -310,8 +316,7 @@ def run_ours(args):
                    "bytes_per_kv_token_head": bytes_per_token_head},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "roofline": {"bound": "hbm", "kernel": ("isoquant_attend_decode (k_attend_partial + k_attend_combine)" if args.bits == 3
-                                                else "isoquant_attend_decode (k_attend_tiles + k_attend_combine)"),
+        "roofline": {"bound": "hbm", "kernel": f"isoquant_attend_decode ({partial_kernel} + k_attend_combine)",
                      "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
                      "bytes_per_launch": bytes_per_launch, "avg_launch_ms": attn_avg_ms,

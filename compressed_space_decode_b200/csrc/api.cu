@@ -378,7 +378,6 @@ int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache, cons
   AttendShape s;
   st = make_shape(ctx, batch, nq, num_q_heads, cache->page_size, causal, &s);
   if (st != ISOQUANT_OK) return st;
-  if (s.bits != 3 && s.page_size < 64) return ISOQUANT_ERR_UNSUPPORTED;  // tcgen05 kernels: 64-token tiles
   if (!(scale >= 0.0f) || !std::isfinite(scale)) return ISOQUANT_ERR_INVALID_ARG;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(static_cast<float>(kD));
   if (batch == 0) return ISOQUANT_OK;
@@ -402,7 +401,6 @@ int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq, int num_q_head
   AttendShape s;
   int st = make_shape(ctx, batch, nq, num_q_heads, page_size, 0, &s);
   if (st != ISOQUANT_OK) return st;
-  if (s.bits != 3 && s.page_size < 64) return ISOQUANT_ERR_UNSUPPORTED;
   if (batch == 0) return ISOQUANT_OK;
   if (seq_lens == nullptr || workspace == nullptr || out == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   if (!aligned(workspace, 16) || !aligned(out, 16) || !aligned(seq_lens, 4)) return ISOQUANT_ERR_ALIGNMENT;

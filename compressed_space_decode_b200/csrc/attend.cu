@@ -44,22 +44,6 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 #endif
 constexpr int kStages = ISOQUANT_ATTEND_STAGES;
 constexpr int kMaxPage = 256;
-// Shared-memory row strides (32-bit words) of the K and V code rows.  K rows
-// are read as word rows {3t, 3t+1, 3t+2} by the four threads of a quad; a
-// stride = 24 (mod 32) puts those rows in distinct 16-byte bank groups.  V
-// rows are read as rows {2p, 2p+1}; a stride = 4 (mod 32) interleaves them.
-#ifdef ISOQUANT_DENSE_STAGE
-constexpr int kStrideK = kMaxPage;  // smem row stride = page_size at run time
-constexpr int kStrideV = kMaxPage;
-#else
-constexpr int kStrideK = kMaxPage + 24;
-constexpr int kStrideV = kMaxPage + 4;
-#endif
-constexpr int kStageKC = 0;
-constexpr int kStageVC = kStageKC + kWords * kStrideK * 4;
-constexpr int kStageKN = kStageVC + kWords * kStrideV * 4;
-constexpr int kStageVN = kStageKN + kMaxPage * 2;
-constexpr int kStageBytes = kStageVN + kMaxPage * 2;
 // Merge scratch (o[warps][8 rows][128], m[warps][8], l[warps][8], e[8]) is
 // placed in the stage buffer being retired when a pair ends, after every
 // consumer warp has finished reading it and before the stage is released.
@@ -67,16 +51,45 @@ constexpr int kScratchO = 0;
 constexpr int kScratchM = kScratchO + kConsumerWarps * 8 * kD * 4;
 constexpr int kScratchL = kScratchM + kConsumerWarps * 8 * 4;
 constexpr int kScratchE = kScratchL + kConsumerWarps * 8 * 4;
-static_assert(kScratchE + 8 * 4 <= kStageBytes, "merge scratch must fit in one stage");
-// query A fragments of the current pair (hi/lo fp16, 8 k-chunks x 32 lanes x
-// 16 B) and the per-row power-of-two scale, shared by the consumer warps
-constexpr int kQFrag = kStages * kStageBytes;
-constexpr int kQScale = kQFrag + 8 * 32 * 16;
-constexpr int kBarriers = kQScale + 8 * 4;
-// abort flag (+0), CTA range and walk start (+8..+47)
-constexpr int kLocate = kBarriers + 2 * kStages * 8;
-constexpr int kSmemBytes = kLocate + 64;
-static_assert(kStageBytes % 16 == 0, "stage alignment");
+
+// Shared memory of the mma.sync kernel for BITS-bit codes.  A stage holds one
+// page of one (sequence, KV head): W code-word rows of K and of V (row w =
+// word w of every token of the page) and the K and V norms.  Row strides (in
+// 32-bit words): a quad's four threads read K rows {3t, 3t+1, 3t+2} (3 bits)
+// or {t, t+4, ...} (2 and 4 bits) as 16-byte vectors, which a stride = 24 or
+// 8 (mod 32) puts in distinct bank groups; V rows {g, g+1} are interleaved by
+// a stride = 4 (mod 32).
+template <int BITS>
+struct DecLayout {
+  static constexpr int W = words_for(BITS);
+  static constexpr int kCpw = codes_per_word(BITS);                     // codes per word
+  static constexpr int kPpw = kCpw / 2;                                 // code pairs per word
+  static constexpr int kKWords = 4;                                     // K words a thread reads per token
+  static constexpr int kVWords = BITS == 4 ? 2 : 1;                     // V words per token (2, 4 bits)
+  static constexpr int kStages = BITS == 4 ? 2 : ::isoquant::kStages;  // 4 bits: 2 stages fit 2 CTAs/SM
+  static constexpr int kStrideK = BITS == 3 ? kMaxPage + 24 : kMaxPage + 8;
+  static constexpr int kStrideV = kMaxPage + 4;
+  static constexpr int kStageKC = 0;
+  static constexpr int kStageVC = kStageKC + W * kStrideK * 4;
+  static constexpr int kStageKN = kStageVC + W * kStrideV * 4;
+  static constexpr int kStageVN = kStageKN + kMaxPage * 2;
+  static constexpr int kStageBytes = kStageVN + kMaxPage * 2;
+  // query A fragments of the current pair (hi/lo fp16, 8 k-chunks x 32
+  // lanes x 16 B) and the per-row power-of-two scale, shared by the warps
+  static constexpr int kQFrag = kStages * kStageBytes;
+  static constexpr int kQScale = kQFrag + 8 * 32 * 16;
+  static constexpr int kBarriers = kQScale + 8 * 4;
+  // abort flag (+0), CTA range and walk start (+8..+47)
+  static constexpr int kLocate = kBarriers + 2 * kStages * 8;
+  static constexpr int kSmemBytes = kLocate + 64;
+  // bytes a page's copies bring per token: K and V words, K and V norms
+  static constexpr int kTxPerToken = 8 * W + 4;
+  // pair table of the 2- and 4-bit kernels (the 3-bit one uses s_lut):
+  // entry i = half2(C[i mod 2^BITS], C[i >> BITS]), one copy per lane
+  static constexpr int kLutWords = BITS == 3 ? 4 : (1 << (2 * BITS)) * 32;
+  static_assert(kScratchE + 8 * 4 <= kStageBytes, "merge scratch must fit in one stage");
+  static_assert(kStageBytes % 16 == 0, "stage alignment");
+};
 
 constexpr uint32_t kSpinLimit = 1u << 25;  // polls (a backstop: the time limit ends a wait first)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -461,24 +474,76 @@ __device__ __forceinline__ uint32_t k_pair_c(const uint4 (&kw)[4], int j, uint32
     return lut_at((((u4_at(kw[3], j) << 7) >> sh12) & 0x1F80u) | lane4);
   }
 }
-__device__ __forceinline__ uint32_t k_pair(const uint4 (&kw)[4], int j, int k, uint32_t sh12, uint32_t lane4) {
-  switch (k) {
-    case 0: return k_pair_c<0>(kw, j, sh12, lane4);
-    case 1: return k_pair_c<1>(kw, j, sh12, lane4);
-    case 2: return k_pair_c<2>(kw, j, sh12, lane4);
-    case 3: return k_pair_c<3>(kw, j, sh12, lane4);
-    case 4: return k_pair_c<4>(kw, j, sh12, lane4);
-    case 5: return k_pair_c<5>(kw, j, sh12, lane4);
-    case 6: return k_pair_c<6>(kw, j, sh12, lane4);
-    case 7: return k_pair_c<7>(kw, j, sh12, lane4);
-    case 8: return k_pair_c<8>(kw, j, sh12, lane4);
-    case 9: return k_pair_c<9>(kw, j, sh12, lane4);
-    case 10: return k_pair_c<10>(kw, j, sh12, lane4);
-    case 11: return k_pair_c<11>(kw, j, sh12, lane4);
-    case 12: return k_pair_c<12>(kw, j, sh12, lane4);
-    case 13: return k_pair_c<13>(kw, j, sh12, lane4);
-    case 14: return k_pair_c<14>(kw, j, sh12, lane4);
-    default: return k_pair_c<15>(kw, j, sh12, lane4);
+// 2 and 4 bits: pair k (0..15) is pair k mod P (P = pairs per word) of word
+// k / P of the thread's words tq, tq + 4, ...: its 2 * BITS bits start at
+// bit 2 * BITS * (k mod P); the table has 2^(2 BITS) entries.
+template <int SH, uint32_t MASK>
+__device__ __forceinline__ uint32_t lut_off_m(uint32_t x, uint32_t lane4) {
+  const uint32_t y = (SH >= 0) ? (x >> (SH >= 0 ? SH : 0)) : (x << (SH < 0 ? -SH : 0));
+  return (y & MASK) | lane4;
+}
+__device__ __forceinline__ uint32_t lut_at2(const char *lut, uint32_t off) {
+  return *reinterpret_cast<const uint32_t *>(lut + off);
+}
+template <int BITS, int K>
+__device__ __forceinline__ uint32_t k_pair_w(const uint4 (&kw)[4], int j, uint32_t lane4, const char *lut) {
+  constexpr int kPpw = 16 / BITS;
+  constexpr uint32_t kMask = ((1u << (2 * BITS)) - 1u) << 7;
+  return lut_at2(lut, lut_off_m<2 * BITS * (K % kPpw) - 7, kMask>(u4_at(kw[K / kPpw], j), lane4));
+}
+// The kPpw 2*BITS-bit slots of a merged word, looked up in order
+template <int BITS>
+__device__ __forceinline__ void merged_pairs(uint32_t e, uint32_t lane4, const char *lut, uint32_t *out) {
+  constexpr int kPpw = 16 / BITS;
+  constexpr uint32_t kMask = ((1u << (2 * BITS)) - 1u) << 7;
+#pragma unroll
+  for (int k = 0; k < kPpw; ++k) {
+    const int sh = 2 * BITS * k - 7;
+    const uint32_t y = sh >= 0 ? (e >> sh) : (e << -sh);
+    out[k] = lut_at2(lut, (y & kMask) | lane4);
+  }
+}
+template <int BITS>
+__device__ __forceinline__ uint32_t k_pair(const uint4 (&kw)[4], int j, int k, uint32_t sh12, uint32_t lane4,
+                                           const char *lut) {
+  if constexpr (BITS == 3) {
+    switch (k) {
+      case 0: return k_pair_c<0>(kw, j, sh12, lane4);
+      case 1: return k_pair_c<1>(kw, j, sh12, lane4);
+      case 2: return k_pair_c<2>(kw, j, sh12, lane4);
+      case 3: return k_pair_c<3>(kw, j, sh12, lane4);
+      case 4: return k_pair_c<4>(kw, j, sh12, lane4);
+      case 5: return k_pair_c<5>(kw, j, sh12, lane4);
+      case 6: return k_pair_c<6>(kw, j, sh12, lane4);
+      case 7: return k_pair_c<7>(kw, j, sh12, lane4);
+      case 8: return k_pair_c<8>(kw, j, sh12, lane4);
+      case 9: return k_pair_c<9>(kw, j, sh12, lane4);
+      case 10: return k_pair_c<10>(kw, j, sh12, lane4);
+      case 11: return k_pair_c<11>(kw, j, sh12, lane4);
+      case 12: return k_pair_c<12>(kw, j, sh12, lane4);
+      case 13: return k_pair_c<13>(kw, j, sh12, lane4);
+      case 14: return k_pair_c<14>(kw, j, sh12, lane4);
+      default: return k_pair_c<15>(kw, j, sh12, lane4);
+    }
+  } else {
+    switch (k) {
+      case 0: return k_pair_w<BITS, 0>(kw, j, lane4, lut);
+      case 1: return k_pair_w<BITS, 1>(kw, j, lane4, lut);
+      case 2: return k_pair_w<BITS, 2>(kw, j, lane4, lut);
+      case 3: return k_pair_w<BITS, 3>(kw, j, lane4, lut);
+      case 4: return k_pair_w<BITS, 4>(kw, j, lane4, lut);
+      case 5: return k_pair_w<BITS, 5>(kw, j, lane4, lut);
+      case 6: return k_pair_w<BITS, 6>(kw, j, lane4, lut);
+      case 7: return k_pair_w<BITS, 7>(kw, j, lane4, lut);
+      case 8: return k_pair_w<BITS, 8>(kw, j, lane4, lut);
+      case 9: return k_pair_w<BITS, 9>(kw, j, lane4, lut);
+      case 10: return k_pair_w<BITS, 10>(kw, j, lane4, lut);
+      case 11: return k_pair_w<BITS, 11>(kw, j, lane4, lut);
+      case 12: return k_pair_w<BITS, 12>(kw, j, lane4, lut);
+      case 13: return k_pair_w<BITS, 13>(kw, j, lane4, lut);
+      case 14: return k_pair_w<BITS, 14>(kw, j, lane4, lut);
+      default: return k_pair_w<BITS, 15>(kw, j, lane4, lut);
+    }
   }
 }
 
@@ -603,22 +668,33 @@ __device__ __forceinline__ void merge_rows(const float *records, int64_t pair, i
 }
 
 // ------------------------------------------------------------ partial kernel
+template <int BITS>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const PartialParams p) {
+  using L = DecLayout<BITS>;
   extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(16) uint32_t lutw[L::kLutWords];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tq = lane & 3;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarriers);
-  uint64_t *empty = full + kStages;
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kLocate);
-  int64_t *loc = reinterpret_cast<int64_t *>(smem + kLocate + 8);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBarriers);
+  uint64_t *empty = full + L::kStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kLocate);
+  int64_t *loc = reinterpret_cast<int64_t *>(smem + L::kLocate + 8);
   const int ps = p.page_size;
 
-  for (int e = tid; e < 64 * 32; e += kThreads) {
-    const int idx = e >> 5;
-    s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
+  if constexpr (BITS == 3) {
+    for (int e = tid; e < 64 * 32; e += kThreads) {
+      const int idx = e >> 5;
+      s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
+    }
+  } else {
+    for (int e = tid; e < L::kLutWords; e += kThreads) {
+      const int idx = e >> 5;
+      lutw[e] = pack_half2(p.level[idx & ((1 << BITS) - 1)], p.level[idx >> BITS]);
+    }
   }
+  const char *lutb = reinterpret_cast<const char *>(lutw);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
@@ -666,8 +742,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
     // ------------------------------------------------------------ producer
     int64_t it = 0;
     for (int64_t g = gs; g < ge; ++g, ++it) {
-      const int stage = static_cast<int>(it % kStages);
-      const uint32_t round = static_cast<uint32_t>(it / kStages);
+      const int stage = static_cast<int>(it % L::kStages);
+      const uint32_t round = static_cast<uint32_t>(it / L::kStages);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(&empty[stage], (round & 1u) ^ 1u, p.status, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -678,38 +754,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
         if (lane == 0) set_status(p.status, ISOQUANT_DEVERR_PAGE_RANGE);
         phys = 0;
       }
-      uint8_t *st = smem + static_cast<size_t>(stage) * kStageBytes;
-      if (lane == 0) mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(108 * ps));
+      uint8_t *st = smem + static_cast<size_t>(stage) * L::kStageBytes;
+      if (lane == 0) mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(L::kTxPerToken * ps));
       __syncwarp();
       const int64_t kblk = (static_cast<int64_t>(phys) * 2 + 0) * p.H + wk.h;
       const int64_t vblk = (static_cast<int64_t>(phys) * 2 + 1) * p.H + wk.h;
-#ifdef ISOQUANT_DENSE_STAGE
-      if (lane == 0) {
-        bulk_g2s(st + kStageKC, p.codes + kblk * kWords * ps, static_cast<uint32_t>(kWords * ps * 4), &full[stage]);
-      } else if (lane == 1) {
-        bulk_g2s(st + kStageVC, p.codes + vblk * kWords * ps, static_cast<uint32_t>(kWords * ps * 4), &full[stage]);
-      } else if (lane == 2 * kWords) {
-#else
-      if (lane < kWords) {
-        bulk_g2s(st + kStageKC + lane * kStrideK * 4, p.codes + (kblk * kWords + lane) * ps,
-                 static_cast<uint32_t>(ps * 4), &full[stage]);
-      } else if (lane < 2 * kWords) {
-        const int w = lane - kWords;
-        bulk_g2s(st + kStageVC + w * kStrideV * 4, p.codes + (vblk * kWords + w) * ps,
-                 static_cast<uint32_t>(ps * 4), &full[stage]);
-      } else if (lane == 2 * kWords) {
-#endif
-        bulk_g2s(st + kStageKN, p.norms + kblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
-      } else if (lane == 2 * kWords + 1) {
-        bulk_g2s(st + kStageVN, p.norms + vblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
+      // one bulk copy per code-word row of K and V, and the two norm rows
+      for (int c = lane; c < 2 * L::W + 2; c += 32) {
+        if (c < L::W) {
+          bulk_g2s(st + L::kStageKC + c * L::kStrideK * 4, p.codes + (kblk * L::W + c) * ps,
+                   static_cast<uint32_t>(ps * 4), &full[stage]);
+        } else if (c < 2 * L::W) {
+          const int w = c - L::W;
+          bulk_g2s(st + L::kStageVC + w * L::kStrideV * 4, p.codes + (vblk * L::W + w) * ps,
+                   static_cast<uint32_t>(ps * 4), &full[stage]);
+        } else if (c == 2 * L::W) {
+          bulk_g2s(st + L::kStageKN, p.norms + kblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
+        } else {
+          bulk_g2s(st + L::kStageVN, p.norms + vblk * ps, static_cast<uint32_t>(ps * 2), &full[stage]);
+        }
       }
       if (g + 1 < ge) wk.advance(p.seq_lens, p.B, p.H, ps);
     }
     // wait (bounded) for every copy still in flight before the CTA exits
     if (lane == 0) {
       const int64_t issued = it;
-      for (int64_t k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
-        mbar_wait(&full[k % kStages], static_cast<uint32_t>((k / kStages) & 1), p.status, nullptr);
+      for (int64_t k = (issued > L::kStages ? issued - L::kStages : 0); k < issued; ++k)
+        mbar_wait(&full[k % L::kStages], static_cast<uint32_t>((k / L::kStages) & 1), p.status, nullptr);
     }
     return;
   }
@@ -720,21 +791,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
   // dims this thread feeds to Q.K^T: pair k (k = 0..15) = coordinates
   // (kdim(k), kdim(k) + 1); pairs 0..14 come from words 3tq..3tq+2, pair 15
   // from word 12.
+  // (2 and 4 bits: pairs of words tq, tq + 4, ..., kPpw pairs per word)
   auto kdim = [&](int k) -> int {
-    return k < 15 ? 10 * (3 * tq + k / 5) + 2 * (k % 5) : 120 + 2 * tq;
+    if constexpr (BITS == 3) return k < 15 ? 10 * (3 * tq + k / 5) + 2 * (k % 5) : 120 + 2 * tq;
+    else return (tq + 4 * (k / L::kPpw)) * L::kCpw + 2 * (k % L::kPpw);
   };
   // dims this thread feeds to P.V (rows gid / gid+8 of each 16-dim tile):
   // word gid fully, half of word 8 + gid/2, code gid of word 12.
   const int par = gid & 1;
+  // 2 bits: word gid (even dims, then odd ones); 4 bits: words gid and
+  // 8 + gid (each: even dims, then odd ones)
   auto vdim = [&](int k) -> int {
-    if (k < 5) return 10 * gid + 2 * k;
-    if (k < 10) return 10 * gid + 2 * (k - 5) + 1;
-    if (k < 15) return 10 * (8 + (gid >> 1)) + par + 2 * (k - 10);
-    return 120 + gid;
+    if constexpr (BITS == 3) {
+      if (k < 5) return 10 * gid + 2 * k;
+      if (k < 10) return 10 * gid + 2 * (k - 5) + 1;
+      if (k < 15) return 10 * (8 + (gid >> 1)) + par + 2 * (k - 10);
+      return 120 + gid;
+    } else if constexpr (BITS == 2) {
+      return 16 * gid + (k < 8 ? 2 * k : 2 * (k - 8) + 1);
+    } else {
+      const int w = k < 8 ? gid : 8 + gid, kk = k & 7;
+      return 8 * w + (kk < 4 ? 2 * kk : 2 * (kk - 4) + 1);
+    }
   };
 
-  uint4 *sq = reinterpret_cast<uint4 *>(smem + kQFrag);
-  float *sq_scale = reinterpret_cast<float *>(smem + kQScale);
+  uint4 *sq = reinterpret_cast<uint4 *>(smem + L::kQFrag);
+  float *sq_scale = reinterpret_cast<float *>(smem + L::kQScale);
   float acc[8][4];
   float m_run = -INFINITY, l_run = 0.f, inv2e = 1.f;
   int lim = 0, lim_min = 0, lim_max = 0;
@@ -801,11 +883,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
     bool ok = true;
     if (lane == 0) ok = mbar_wait(&full[stage], phase, p.status, abort_flag);
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    const uint8_t *st = smem + static_cast<size_t>(stage) * kStageBytes;
-    const uint32_t *kc = reinterpret_cast<const uint32_t *>(st + kStageKC);
-    const uint32_t *vc = reinterpret_cast<const uint32_t *>(st + kStageVC);
-    const __half *kn = reinterpret_cast<const __half *>(st + kStageKN);
-    const __half *vn = reinterpret_cast<const __half *>(st + kStageVN);
+    const uint8_t *st = smem + static_cast<size_t>(stage) * L::kStageBytes;
+    const uint32_t *kc = reinterpret_cast<const uint32_t *>(st + L::kStageKC);
+    const uint32_t *vc = reinterpret_cast<const uint32_t *>(st + L::kStageVC);
+    const __half *kn = reinterpret_cast<const __half *>(st + L::kStageKN);
+    const __half *vn = reinterpret_cast<const __half *>(st + L::kStageVN);
 
     // each warp takes 64-token units: two 32-token halves whose independent
     // work interleaves, sharing one softmax reduction
@@ -819,19 +901,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
 
       // ---- scores: tile t = 4h + j, column n = token t0 + 32h + 4n + j.  The
       // k-chunk loop is outermost so that the 8 tiles' mma chains interleave.
-#ifdef ISOQUANT_DENSE_STAGE
-      const int rsK = ps, rsV = ps;
-#else
-      constexpr int rsK = kStrideK, rsV = kStrideV;
-#endif
-      uint4 kw[2][4];  // words 3tq, 3tq+1, 3tq+2 and 12 of tokens t0 + 32h + 4gid + {0..3}
+      constexpr int rsK = L::kStrideK, rsV = L::kStrideV;
+      uint4 kw[2][4];  // words 3tq, 3tq+1, 3tq+2 and 12 (or tq + 4i) of tokens t0 + 32h + 4gid + {0..3}
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t *kb = kc + t0 + 32 * h + 4 * gid;
-        kw[h][0] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 0) * rsK);
-        kw[h][1] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 1) * rsK);
-        kw[h][2] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 2) * rsK);
-        kw[h][3] = *reinterpret_cast<const uint4 *>(kb + 12 * rsK);
+        if constexpr (BITS == 3) {
+          kw[h][0] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 0) * rsK);
+          kw[h][1] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 1) * rsK);
+          kw[h][2] = *reinterpret_cast<const uint4 *>(kb + (3 * tq + 2) * rsK);
+          kw[h][3] = *reinterpret_cast<const uint4 *>(kb + 12 * rsK);
+        } else {
+#pragma unroll
+          for (int i = 0; i < L::kKWords; ++i) kw[h][i] = *reinterpret_cast<const uint4 *>(kb + (tq + 4 * i) * rsK);
+        }
       }
       const uint32_t sh12 = 6 * tq;
       float d[8][4];
@@ -842,8 +925,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
         const uint4 qa = sq[c * 32 + lane];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          const uint32_t b0 = k_pair(kw[t >> 2], t & 3, 2 * c, sh12, lane4);
-          const uint32_t b1 = k_pair(kw[t >> 2], t & 3, 2 * c + 1, sh12, lane4);
+          const uint32_t b0 = k_pair<BITS>(kw[t >> 2], t & 3, 2 * c, sh12, lane4, lutb);
+          const uint32_t b1 = k_pair<BITS>(kw[t >> 2], t & 3, 2 * c + 1, sh12, lane4, lutb);
           mma16816(d[t], qa.x, qa.y, qa.z, qa.w, b0, b1);
         }
       }
@@ -914,44 +997,84 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
       l_run += psum[0] + psum[1];
 
       // ---- P.V: O^T[16 dims x 8 rows] += V^T[16 dims x 16 tok] P^T
-      constexpr uint32_t M = 0x071C71C7u;  // even-indexed 3-bit fields
+      if constexpr (BITS == 3) {
+        constexpr uint32_t M = 0x071C71C7u;  // even-indexed 3-bit fields
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t *vb = vc + t0 + 32 * h + 8 * tq;
-        const uint4 va0 = *reinterpret_cast<const uint4 *>(vb + gid * rsV);
-        const uint4 va1 = *reinterpret_cast<const uint4 *>(vb + gid * rsV + 4);
-        const uint4 vb0 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * rsV);
-        const uint4 vb1 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * rsV + 4);
-        const uint4 vz0 = *reinterpret_cast<const uint4 *>(vb + 12 * rsV);
-        const uint4 vz1 = *reinterpret_cast<const uint4 *>(vb + 12 * rsV + 4);
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t *vb = vc + t0 + 32 * h + 8 * tq;
+          const uint4 va0 = *reinterpret_cast<const uint4 *>(vb + gid * rsV);
+          const uint4 va1 = *reinterpret_cast<const uint4 *>(vb + gid * rsV + 4);
+          const uint4 vb0 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * rsV);
+          const uint4 vb1 = *reinterpret_cast<const uint4 *>(vb + (8 + (gid >> 1)) * rsV + 4);
+          const uint4 vz0 = *reinterpret_cast<const uint4 *>(vb + 12 * rsV);
+          const uint4 vz1 = *reinterpret_cast<const uint4 *>(vb + 12 * rsV + 4);
 #pragma unroll
-        for (int kap = 0; kap < 2; ++kap) {
-          uint32_t va[2][16];
+          for (int kap = 0; kap < 2; ++kap) {
+            uint32_t va[2][16];
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int tp = 2 * kap + half;  // token pair (2tp, 2tp+1) of this thread's 8
-            const uint4 &A = tp < 2 ? va0 : va1;
-            const uint4 &Bv = tp < 2 ? vb0 : vb1;
-            const uint4 &Z = tp < 2 ? vz0 : vz1;
-            const int e0 = (tp & 1) * 2;
-            const uint32_t wa = u4_at(A, e0), wa1 = u4_at(A, e0 + 1);
-            const uint32_t wb = u4_at(Bv, e0), wb1 = u4_at(Bv, e0 + 1);
-            const uint32_t wz = u4_at(Z, e0), wz1 = u4_at(Z, e0 + 1);
-            // merge two tokens' words: 6-bit slot k = (code of tok a, code of tok b)
-            const uint32_t e_even = (wa & M) | ((wa1 << 3) & ~M);
-            const uint32_t e_odd = ((wa >> 3) & M) | (wa1 & ~M);
-            const uint32_t e_half = ((wb >> (3 * par)) & M) | ((wb1 << (3 - 3 * par)) & ~M);
-            word_pairs(e_even, lane4, va[half] + 0);
-            word_pairs(e_odd, lane4, va[half] + 5);
-            word_pairs(e_half, lane4, va[half] + 10);
-            const uint32_t z12 = (((wz >> (3 * gid)) & 7u) << 7) | (((wz1 >> (3 * gid)) & 7u) << 10);
-            va[half][15] = lut_at(z12 | lane4);
+            for (int half = 0; half < 2; ++half) {
+              const int tp = 2 * kap + half;  // token pair (2tp, 2tp+1) of this thread's 8
+              const uint4 &A = tp < 2 ? va0 : va1;
+              const uint4 &Bv = tp < 2 ? vb0 : vb1;
+              const uint4 &Z = tp < 2 ? vz0 : vz1;
+              const int e0 = (tp & 1) * 2;
+              const uint32_t wa = u4_at(A, e0), wa1 = u4_at(A, e0 + 1);
+              const uint32_t wb = u4_at(Bv, e0), wb1 = u4_at(Bv, e0 + 1);
+              const uint32_t wz = u4_at(Z, e0), wz1 = u4_at(Z, e0 + 1);
+              // merge two tokens' words: 6-bit slot k = (code of tok a, code of tok b)
+              const uint32_t e_even = (wa & M) | ((wa1 << 3) & ~M);
+              const uint32_t e_odd = ((wa >> 3) & M) | (wa1 & ~M);
+              const uint32_t e_half = ((wb >> (3 * par)) & M) | ((wb1 << (3 - 3 * par)) & ~M);
+              word_pairs(e_even, lane4, va[half] + 0);
+              word_pairs(e_odd, lane4, va[half] + 5);
+              word_pairs(e_half, lane4, va[half] + 10);
+              const uint32_t z12 = (((wz >> (3 * gid)) & 7u) << 7) | (((wz1 >> (3 * gid)) & 7u) << 10);
+              va[half][15] = lut_at(z12 | lane4);
+            }
+            const uint32_t b0 = pack_half2(pv[8 * h + 4 * kap + 0], pv[8 * h + 4 * kap + 1]);
+            const uint32_t b1 = pack_half2(pv[8 * h + 4 * kap + 2], pv[8 * h + 4 * kap + 3]);
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+              mma16816(acc[m], va[0][2 * m], va[0][2 * m + 1], va[1][2 * m], va[1][2 * m + 1], b0, b1);
           }
-          const uint32_t b0 = pack_half2(pv[8 * h + 4 * kap + 0], pv[8 * h + 4 * kap + 1]);
-          const uint32_t b1 = pack_half2(pv[8 * h + 4 * kap + 2], pv[8 * h + 4 * kap + 3]);
+        }
+      } else {
+        // 2 and 4 bits: the words of two tokens merge field by field, so
+        // that slot k of the even (odd) merge is the pair (code of token a,
+        // code of token b) of the word's field 2k (2k + 1)
+        constexpr uint32_t M = BITS == 2 ? 0x33333333u : 0x0F0F0F0Fu;  // even-indexed fields
 #pragma unroll
-          for (int m = 0; m < 8; ++m)
-            mma16816(acc[m], va[0][2 * m], va[0][2 * m + 1], va[1][2 * m], va[1][2 * m + 1], b0, b1);
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t *vb = vc + t0 + 32 * h + 8 * tq;
+          uint4 vw[L::kVWords][2];  // words gid (and 8 + gid) of the thread's 8 tokens
+#pragma unroll
+          for (int i = 0; i < L::kVWords; ++i) {
+            vw[i][0] = *reinterpret_cast<const uint4 *>(vb + (gid + 8 * i) * rsV);
+            vw[i][1] = *reinterpret_cast<const uint4 *>(vb + (gid + 8 * i) * rsV + 4);
+          }
+#pragma unroll
+          for (int kap = 0; kap < 2; ++kap) {
+            uint32_t va[2][16];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const int tp = 2 * kap + half;  // token pair (2tp, 2tp+1) of this thread's 8
+              const int e0 = (tp & 1) * 2;
+#pragma unroll
+              for (int i = 0; i < L::kVWords; ++i) {
+                const uint4 &A = tp < 2 ? vw[i][0] : vw[i][1];
+                const uint32_t wa = u4_at(A, e0), wb = u4_at(A, e0 + 1);
+                const uint32_t e_even = (wa & M) | ((wb << BITS) & ~M);
+                const uint32_t e_odd = ((wa >> BITS) & M) | (wb & ~M);
+                merged_pairs<BITS>(e_even, lane4, lutb, va[half] + 8 * i);
+                merged_pairs<BITS>(e_odd, lane4, lutb, va[half] + 8 * i + L::kPpw);
+              }
+            }
+            const uint32_t b0 = pack_half2(pv[8 * h + 4 * kap + 0], pv[8 * h + 4 * kap + 1]);
+            const uint32_t b1 = pack_half2(pv[8 * h + 4 * kap + 2], pv[8 * h + 4 * kap + 3]);
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+              mma16816(acc[m], va[0][2 * m], va[0][2 * m + 1], va[1][2 * m], va[1][2 * m + 1], b0, b1);
+          }
         }
       }
     }
@@ -960,7 +1083,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
       const int64_t pair = (static_cast<int64_t>(wk.rg) * p.B + wk.b) * p.H + wk.h;
       // every warp is done reading this stage: reuse it as merge scratch
       named_bar_sync(1, kConsumerWarps * 32);
-      uint8_t *scr = smem + static_cast<size_t>(stage) * kStageBytes;
+      uint8_t *scr = smem + static_cast<size_t>(stage) * L::kStageBytes;
       float *sm_o = reinterpret_cast<float *>(scr + kScratchO);
       float *sm_m = reinterpret_cast<float *>(scr + kScratchM);
       float *sm_l = reinterpret_cast<float *>(scr + kScratchL);
@@ -1014,7 +1137,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
-    if (++stage == kStages) {
+    if (++stage == L::kStages) {
       stage = 0;
       phase ^= 1u;
     }
@@ -2180,9 +2303,9 @@ struct TilePlan {
 };
 TilePlan tile_plan(const AttendShape &s, int num_sms) {
   TilePlan t{};
-  // 2- and 4-bit codes always run on the tcgen05 kernels (the mma.sync
-  // kernel's unpacking is 3-bit); 3-bit ones from 64 rows per KV head
-  if ((s.bits == 3 && s.rows < kTRows) || s.page_size < kTTok) return t;
+  // the tcgen05 kernels from 64 rows per KV head (and 64-token pages); the
+  // mma.sync kernel below that, at every code width
+  if (s.rows < kTRows || s.page_size < kTTok) return t;
   t.kind = s.rows >= kWideMinRows ? 2 : 1;
   t.rps = t.kind == 2 ? kWRows : kTRows;
   t.n_cta = t.kind == 2 ? num_sms : num_sms * kTCtasPerSm;
@@ -2205,10 +2328,7 @@ TilePlan use_tiles(const isoquant_ctx *ctx, const AttendShape &s, size_t ws_byte
 }  // namespace
 
 size_t attend_workspace_min_bytes(const AttendShape &s) {
-  if (s.bits != 3) {
-    const TilePlan t = tile_plan(s, s.n_cta / kCtasPerSm);
-    return t.kind != 0 ? t.bytes : kWsHeader;
-  }
+  // the mma.sync kernel's records (every shape can run on it)
   return kWsHeader + s.slots * kRecordFloats * sizeof(float);
 }
 
@@ -2221,9 +2341,16 @@ size_t attend_workspace_bytes(const AttendShape &s) {
 }
 
 namespace {
+// kernel attributes of one code width (the mma.sync and both tcgen05 kernels)
 template <int BITS>
-cudaError_t configure_tcgen05() {
-  cudaError_t e = cudaFuncSetAttribute(k_attend_tiles<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
+cudaError_t configure_width() {
+  cudaError_t e = cudaFuncSetAttribute(k_attend_partial<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DecLayout<BITS>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_attend_partial<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_attend_tiles<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_attend_tiles<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
@@ -2246,14 +2373,9 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
                                   cudaStream_t stream) {
   static int configured_device = -1;
   if (configured_device != ctx->device) {
-    cudaError_t e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_attend_partial, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    e = configure_tcgen05<3>();
-    if (e == cudaSuccess) e = configure_tcgen05<2>();
-    if (e == cudaSuccess) e = configure_tcgen05<4>();
+    cudaError_t e = configure_width<3>();
+    if (e == cudaSuccess) e = configure_width<2>();
+    if (e == cudaSuccess) e = configure_width<4>();
     if (e != cudaSuccess) return e;
     configured_device = ctx->device;
   }
@@ -2293,8 +2415,11 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
       default: return launch_tcgen05<3>(t.kind, p, stream);
     }
   }
-  if (p.bits != 3) return cudaErrorInvalidValue;  // the callers check shapes first
-  return launch_pdl(k_attend_partial, dim3(s.n_cta), dim3(kThreads), kSmemBytes, stream, p);
+  switch (p.bits) {
+    case 2: return launch_pdl(k_attend_partial<2>, dim3(s.n_cta), dim3(kThreads), DecLayout<2>::kSmemBytes, stream, p);
+    case 4: return launch_pdl(k_attend_partial<4>, dim3(s.n_cta), dim3(kThreads), DecLayout<4>::kSmemBytes, stream, p);
+    default: return launch_pdl(k_attend_partial<3>, dim3(s.n_cta), dim3(kThreads), DecLayout<3>::kSmemBytes, stream, p);
+  }
 }
 
 cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s, const int32_t *seq_lens,

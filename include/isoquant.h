@@ -106,9 +106,8 @@ int isoquant_init(isoquant_ctx **out, int num_kv_heads, int head_dim,
  * bits * (j % per_word) of word j / per_word) and ceil(128 / per_word)
  * words per vector (8, 13, 16) in the cache's code array instead of 13;
  * everything else as isoquant_init.  A context's width fixes the layout of
- * every cache used with it.  At 2 and 4 bits attention always runs on the
- * tensor-core kernels, which need pages of at least 64 tokens (otherwise
- * UNSUPPORTED) and the full workspace of isoquant_workspace_size.
+ * every cache used with it.  Attention picks its kernel by shape at every
+ * width (see isoquant_attend_decode).
  * Errors: as isoquant_init; UNSUPPORTED for another width. */
 int isoquant_init_bits(isoquant_ctx **out, int num_kv_heads, int head_dim,
                        const int8_t *signs, const float *quats, int bits);
@@ -169,7 +168,8 @@ int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
  * per KV head, pages of at least 64 tokens and the full workspace, the
  * partial step runs on tcgen05 tensor cores (streams of 64 rows, or of 128
  * rows from 128 rows up), each stream walking only the pages inside its
- * causal horizon.
+ * causal horizon; otherwise on the mma.sync kernel (8-row groups), at every
+ * code width and page size.
  *   q_rot:      device float [batch][nq][num_q_heads][128] (from rotate_q)
  *   page_table: device int32 [batch][max_pages]
  *   seq_lens:   device int32 [batch]; tokens 0..seq_lens[b]-1 are in the

@@ -3,8 +3,9 @@
 The codes and norms the library writes are the oracle's bit for bit
 (outside the 1e-6 boundary band), and attention over them matches the
 oracle's compressed-space attention on every row of sampled (sequence, KV
-head) pairs at decode, verification and prefill shapes (2- and 4-bit
-attention runs on the tcgen05 kernels at every shape).
+head) pairs at decode, verification and prefill shapes: below 64 query rows
+per KV head or with 32-token pages on the mma.sync kernel, from 64 rows on
+the tcgen05 kernels.
 """
 import numpy as np
 import pytest
@@ -22,6 +23,10 @@ def _state(csd, case, bits):
     from compressed_space_decode_b200.workload import DecodeState
     if case == "decode":
         wl = Workload(case, 3, 32, 8, [700, 65, 1], nq=1, page_size=256, seed=61)
+    elif case == "decode_p32":
+        wl = Workload(case, 2, 8, 2, [100, 37], nq=1, page_size=32, seed=66)
+    elif case == "verify_p32":
+        wl = Workload(case, 2, 32, 8, [300, 45], nq=16, page_size=32, causal=True, seed=67)
     elif case == "verify":
         wl = Workload(case, 2, 32, 8, [600, 130], nq=16, page_size=128, causal=True, seed=62)
     else:
@@ -39,7 +44,7 @@ def test_codebook_matches_oracle(cuda_lib, bits):
 
 
 @pytest.mark.parametrize("bits", [2, 4])
-@pytest.mark.parametrize("case", ["decode", "verify", "prefill"])
+@pytest.mark.parametrize("case", ["decode", "verify", "prefill", "decode_p32", "verify_p32"])
 def test_codes_and_attention_match_oracle(cuda_lib, bits, case):
     csd = cuda_lib
     st = _state(csd, case, bits)
@@ -69,19 +74,6 @@ def test_codes_and_attention_match_oracle(cuda_lib, bits, case):
         got = np.stack([out[b, i, hq].numpy() for (i, hq) in idx])
         err = rowwise_rel_err(got, ref)
         assert err.max() <= ATTN_TOL, (bits, case, b, err.max())
-
-
-def test_small_pages_are_unsupported_below_3_bits(cuda_lib):
-    from compressed_space_decode_b200.synthetic import Workload
-    from compressed_space_decode_b200.workload import DecodeState
-    csd = cuda_lib
-    wl = Workload("p32", 1, 8, 2, [100], nq=1, page_size=32, seed=64)
-    st = DecodeState(wl, bits=2)
-    q_rot = torch.zeros((1, 1, 8, D), dtype=torch.float32, device="cuda")
-    out = torch.empty_like(q_rot)
-    with pytest.raises(csd.IsoquantError) as e:
-        csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, _ws(csd, st), out)
-    assert e.value.status == -2
 
 
 @pytest.mark.parametrize("bits", [2, 4])
