@@ -1735,14 +1735,21 @@ constexpr int kWSoftWarps = 4 * kWParts;
 constexpr int kWTpt = kWTok / kWParts;  // tokens of a tile per softmax thread
 constexpr int kWDpt = kD / kWParts;     // Q~ dims / O columns per softmax thread
 // decoder warps: 4 (a thread decodes one token of K or V per tile) or 2 (a
-// thread decodes one token of K and of V), keeping registers in budget
+// thread decodes one token of K and of V).  At 4 bits a pair takes two
+// table lookups, and two decoder warps become the bound (a 8192-token
+// prefill: 3.2 ms with two, 2.1 with four); at 2 and 3 bits two keep the
+// registers in budget at no cost
 #ifndef ISOQUANT_WIDE_DEC
 #define ISOQUANT_WIDE_DEC 0
 #endif
-constexpr int kWDecWarps = ISOQUANT_WIDE_DEC ? ISOQUANT_WIDE_DEC : (kWParts == 2 ? 4 : 2);
-static_assert(kWDecWarps == 2 || kWDecWarps == 4, "two or four decoder warps");
-constexpr int kWMmaWarp = kWSoftWarps + kWDecWarps;
-constexpr int kWThreads = (kWMmaWarp + 1) * 32;
+template <int BITS>
+constexpr int wide_dec_warps() {
+  return ISOQUANT_WIDE_DEC ? ISOQUANT_WIDE_DEC : ((kWParts == 2 || BITS == 4) ? 4 : 2);
+}
+template <int BITS>
+constexpr int wide_threads() {
+  return (kWSoftWarps + wide_dec_warps<BITS>() + 1) * 32;  // softmax, decoder and MMA warps
+}
 // Tensor memory (512 columns, one CTA per SM): S buffers 0 and 1, O, then
 // the A operands of both products, fp16 pairs packed per 32-bit column
 // (row = lane): Q~ high and low parts (64 columns each) and two buffers of
@@ -1765,7 +1772,10 @@ constexpr int kWRed = kWVN + kWStages * kWTok * 4;    // per part: row maxima [2
 constexpr int kWBar = kWRed + 4 * kWParts * kWRows * 4;  // 2 kWStages + 8 mbarriers
 constexpr int kWMisc = kWBar + (2 * kWStages + 8) * 8;  // tensor-memory base, abort flag, MMA-issued flag
 constexpr int kWLoc = kWMisc + 16;                    // walk start + scan scratch
-constexpr int kWSmemBytes = kWLoc + (4 + kWThreads / 32) * 8;
+template <int BITS>
+constexpr int wide_smem_bytes() {
+  return kWLoc + (4 + wide_threads<BITS>() / 32) * 8;
+}
 static_assert(kWK % 128 == 0 && kWV % 128 == 0, "UMMA tile alignment");
 static_assert(kWBar % 8 == 0 && kWLoc % 8 == 0, "barrier alignment");
 
@@ -1810,7 +1820,11 @@ __device__ __forceinline__ void for_each_tile(const PartialParams &p, int64_t gs
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(kWThreads, 1) k_attend_wide(const PartialParams p) {
+__global__ void __launch_bounds__(wide_threads<BITS>(), 1) k_attend_wide(const PartialParams p) {
+  constexpr int kWDecWarps = wide_dec_warps<BITS>();
+  static_assert(kWDecWarps == 2 || kWDecWarps == 4, "two or four decoder warps");
+  constexpr int kWMmaWarp = kWSoftWarps + kWDecWarps;
+  constexpr int kWThreads = wide_threads<BITS>();
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kWBar);
@@ -2355,14 +2369,15 @@ cudaError_t configure_width() {
   e = cudaFuncSetAttribute(k_attend_tiles<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_attend_wide<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
+  e = cudaFuncSetAttribute(k_attend_wide<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, wide_smem_bytes<BITS>());
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(k_attend_wide<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
                               cudaSharedmemCarveoutMaxShared);
 }
 template <int BITS>
 cudaError_t launch_tcgen05(int kind, const PartialParams &p, cudaStream_t stream) {
-  if (kind == 2) return launch_pdl(k_attend_wide<BITS>, dim3(p.n_cta), dim3(kWThreads), kWSmemBytes, stream, p);
+  if (kind == 2)
+    return launch_pdl(k_attend_wide<BITS>, dim3(p.n_cta), dim3(wide_threads<BITS>()), wide_smem_bytes<BITS>(), stream, p);
   return launch_pdl(k_attend_tiles<BITS>, dim3(p.n_cta), dim3(kTThreads), kTSmemBytes, stream, p);
 }
 }  // namespace
