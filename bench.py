@@ -69,6 +69,18 @@ def source_hash(*names):
     return h.hexdigest()[:16]
 
 
+def stage_layout(tensors, align=256):
+    """Byte layout of one pinned staging row holding the given tensors back to
+    back: a list of (offset, bytes, dtype, shape) with every offset a multiple
+    of `align`, and the row's total size."""
+    layout, row_bytes = [], 0
+    for t in tensors:
+        n = t.numel() * t.element_size()
+        layout.append((row_bytes, n, t.dtype, t.shape))
+        row_bytes += (n + align - 1) // align * align
+    return layout, row_bytes
+
+
 def profiled_traffic(kernel_src, bytes_per_launch):
     """Per-launch DRAM bytes of the attention kernel from the committed ncu
     summary, scaled from the captured launch to this one by the algorithmic
@@ -244,10 +256,7 @@ def run_ours(args):
     # and cross to the device in one transfer, as a serving loop would stage them
     kd, vd = torch.empty_like(k_all[0]), torch.empty_like(v_all[0])
     qd, sd, ld = torch.empty_like(q_all[0]), torch.empty_like(slots_all[0]), torch.empty_like(lens_all[0])
-    layout, row_bytes = [], 0
-    for t in (kd, vd, qd, sd, ld):
-        layout.append((row_bytes, t.numel() * t.element_size(), t.dtype, t.shape))
-        row_bytes += (t.numel() * t.element_size() + 255) // 256 * 256
+    layout, row_bytes = stage_layout((kd, vd, qd, sd, ld))
     stage_d = torch.empty(row_bytes, dtype=torch.uint8, device=dev)
     kd, vd, qd, sd, ld = (stage_d[o:o + n].view(dt).view(shp) for o, n, dt, shp in layout)
     stage_h = torch.zeros((e2e_steps, row_bytes), dtype=torch.uint8).pin_memory()

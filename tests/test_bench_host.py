@@ -27,3 +27,22 @@ def test_causal_pairs_matches_brute_force(lens, nq):
 def test_causal_pairs_full_prefill_is_the_triangle():
     wl = Workload("t", 1, 32, 8, [32768], nq=32768, causal=True)
     assert bench.causal_pairs(wl) == 32768 * 32769 // 2
+
+
+def test_stage_layout_views_round_trip():
+    """The e2e staging row: aligned, non-overlapping slots whose views give
+    back each tensor bit for bit after one byte-level copy."""
+    import torch
+    import bench
+    ts = [torch.randn(3, 5, 7).to(torch.bfloat16), torch.arange(17, dtype=torch.int64),
+          torch.arange(5, dtype=torch.int32), torch.randn(2, 128)]
+    layout, row = bench.stage_layout(ts)
+    ends = [o + n for o, n, _, _ in layout]
+    assert all(o % 256 == 0 for o, _, _, _ in layout)
+    assert all(ends[i] <= layout[i + 1][0] for i in range(len(ts) - 1)) and ends[-1] <= row
+    stage = torch.zeros(row, dtype=torch.uint8)
+    for (o, n, dt, shp), t in zip(layout, ts):
+        stage[o:o + n].view(dt).view(shp).copy_(t)
+    copy = stage.clone()
+    for (o, n, dt, shp), t in zip(layout, ts):
+        assert torch.equal(copy[o:o + n].view(dt).view(shp), t)
