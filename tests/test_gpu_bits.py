@@ -27,6 +27,11 @@ def _state(csd, case, bits):
         wl = Workload(case, 2, 8, 2, [100, 37], nq=1, page_size=32, seed=66)
     elif case == "verify_p32":
         wl = Workload(case, 2, 32, 8, [300, 45], nq=16, page_size=32, causal=True, seed=67)
+    elif case == "decode_full":
+        # the decode bench's workload (B = 16, 32 q / 4 KV heads, 32768 tokens, shuffled pages); two
+        # sequences are checked against the oracle
+        import compressed_space_decode_b200.synthetic as syn
+        wl = syn.workloads()["gqa_b16_q32_kv4_L32768_paged"]
     elif case == "verify":
         wl = Workload(case, 2, 32, 8, [600, 130], nq=16, page_size=128, causal=True, seed=62)
     else:
@@ -44,7 +49,7 @@ def test_codebook_matches_oracle(cuda_lib, bits):
 
 
 @pytest.mark.parametrize("bits", [2, 4])
-@pytest.mark.parametrize("case", ["decode", "verify", "prefill", "decode_p32", "verify_p32"])
+@pytest.mark.parametrize("case", ["decode", "verify", "prefill", "decode_p32", "verify_p32", "decode_full"])
 def test_codes_and_attention_match_oracle(cuda_lib, bits, case):
     csd = cuda_lib
     st = _state(csd, case, bits)
@@ -61,7 +66,7 @@ def test_codes_and_attention_match_oracle(cuda_lib, bits, case):
     out = out.cpu()
     assert torch.isfinite(out).all()
     qc = q.float().cpu()
-    for b in range(st.B):
+    for b in (range(st.B) if case != "decode_full" else (3, 12)):
         L = st.seq_lens[b]
         h = (3 * b + 1) % st.H
         k, v = st.kv_tokens(b, 0, L)
