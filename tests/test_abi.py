@@ -66,3 +66,42 @@ def test_strerror_and_argument_errors(native):
     assert L.isoquant_init(ctypes.byref(h), 1, 128, signs.ctypes.data, zq.ctypes.data) == -1
     assert L.isoquant_compress_kv(None, None, None, None, 0, 1, None, None) == -1
     assert L.isoquant_attend_decode(None, None, None, 1, 1, 8, None, 1, None, 0, 0.0, None, 0, None, None) == -1
+
+
+def test_every_entry_rejects_a_null_context(native):
+    """Calls given no context (or no output pointer) return INVALID_ARG on
+    the host, before any CUDA call; width checks return UNSUPPORTED."""
+    L = native.lib()
+    sz = ctypes.c_size_t()
+    st = ctypes.c_uint32()
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 16)()
+    assert L.isoquant_codebook(None, None) == -1
+    assert L.isoquant_codebook_bits(3, None, th) == -1
+    assert L.isoquant_codebook_bits(5, lv, th) == -2
+    assert L.isoquant_codebook_bits(1, lv, th) == -2
+    assert L.isoquant_codebook_bits(2, lv, th) == 0 and L.isoquant_codebook_bits(4, lv, th) == 0
+    h = ctypes.c_void_p()
+    signs = np.ones((1, 128), np.int8)
+    quats = np.zeros((1, 32, 2, 4), np.float32)
+    quats[..., 0] = 1
+    assert L.isoquant_init_bits(ctypes.byref(h), 1, 128, signs.ctypes.data, quats.ctypes.data, 5) == -2
+    assert L.isoquant_init_bits(ctypes.byref(h), 1, 128, signs.ctypes.data, quats.ctypes.data, 1) == -2
+    nanq = quats.copy()
+    nanq[0, 5, 1, 2] = np.nan
+    assert L.isoquant_init_bits(ctypes.byref(h), 1, 128, signs.ctypes.data, nanq.ctypes.data, 3) == -1
+    assert L.isoquant_cache_bytes(None, 4, 256, ctypes.byref(sz), ctypes.byref(sz)) == -1
+    assert L.isoquant_rotate_q(None, None, 0, 1, 8, None, None) == -1
+    assert L.isoquant_decode_prep(None, None, None, None, 1, None, None, 0, 1, 8, None, None) == -1
+    assert L.isoquant_workspace_size(None, 1, 1, 8, ctypes.byref(sz)) == -1
+    assert L.isoquant_step_workspace_size(None, 1, 1, 8, ctypes.byref(sz)) == -1
+    assert L.isoquant_attend_partial(None, None, None, 1, 1, 8, None, 1, None, 0, 0.0, None, 0, None) == -1
+    assert L.isoquant_attend_combine(None, 1, 1, 8, None, 256, None, 0, None, None) == -1
+    assert L.isoquant_attend_decode_static(None, None, None, 1, 1, 8, None, 1, None, 0, 0.0, None, None) == -1
+    assert L.isoquant_decode_step(None, None, None, None, 1, None, None, 0, 1, 1, 8, None, 1, None, 0, 0.0,
+                                  None, 0, None, None) == -1
+    assert L.isoquant_get_status(None, ctypes.byref(st), None) == -1
+    assert L.isoquant_selftest_wait(None, 1000, None, None) == -1
+    assert L.isoquant_last_launch_count(None) == 0
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert native.strerror(code)

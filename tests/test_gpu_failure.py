@@ -48,3 +48,57 @@ def test_selftest_wait_rejects_unbounded_limits(cuda_lib):
     for bad in (0, 10_000_000_001):
         with pytest.raises(cuda_lib.IsoquantError):
             cuda_lib.isoquant_selftest_wait(ctx, bad)
+
+
+def test_argument_errors_with_a_live_context(cuda_lib):
+    """Checks that need a context: each bad argument returns its status from
+    the host, launches nothing and leaves the status word clear; the same
+    context then serves a correct call."""
+    import ctypes
+    from compressed_space_decode_b200.synthetic import Workload
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    L = csd.lib()
+    st = DecodeState(Workload("args", 2, 16, 4, [300, 40], nq=1, page_size=64, seed=72))
+    ctx = st.ctx.handle
+    s0 = csd._stream(None)
+    q = st.queries(0)
+    n_rows = q.shape[0] * q.shape[1]
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    spare = torch.empty(q_rot.numel() + 4, dtype=torch.float32, device="cuda")
+    off4 = ctypes.c_void_p(spare.data_ptr() + 4)  # 4 bytes past a 16-byte boundary
+    p = csd._ptr
+    dt = csd._dtype(q)
+    # rotate_q: misaligned output, unknown dtype, q heads not a multiple of the KV heads
+    assert L.isoquant_rotate_q(ctx, p(q), dt, n_rows, st.Hq, off4, s0) == -6
+    assert L.isoquant_rotate_q(ctx, p(q), 99, n_rows, st.Hq, p(q_rot), s0) == -2
+    assert L.isoquant_rotate_q(ctx, p(q), dt, n_rows, st.Hq + 1, p(q_rot), s0) == -1
+    assert L.isoquant_last_launch_count(ctx) == 0
+    csd.isoquant_rotate_q(st.ctx, q.reshape(-1, st.Hq, D), q_rot.view(-1, st.Hq, D))
+    ws = _ws(csd, st)
+    out = torch.empty_like(q_rot)
+    cs = st.cache.c_struct()
+    B, nq, Hq, maxp = st.B, 1, st.Hq, st.page_table.shape[1]
+
+    def attend(cache_struct=cs, ws_ptr=None, ws_bytes=None, out_ptr=None, scale=0.0):
+        return L.isoquant_attend_decode(ctx, ctypes.byref(cache_struct), p(q_rot), B, nq, Hq, p(st.page_table), maxp,
+                                        p(st.seq_lens_dev), 0, scale, ws_ptr if ws_ptr is not None else p(ws),
+                                        ws.numel() * 4 if ws_bytes is None else ws_bytes,
+                                        out_ptr if out_ptr is not None else p(out), s0)
+    assert attend(ws_bytes=64) == -4                      # workspace too small
+    assert attend(ws_ptr=ctypes.c_void_p(ws.data_ptr() + 4)) == -6
+    assert attend(out_ptr=off4) == -6
+    assert attend(scale=-1.0) == -1
+    bad = csd._Cache(st.cache.codes.data_ptr(), st.cache.norms.data_ptr(), st.cache.num_pages, 48)
+    assert attend(cache_struct=bad) == -2                 # page size 48
+    none = csd._Cache(0, st.cache.norms.data_ptr(), st.cache.num_pages, st.ps)
+    assert attend(cache_struct=none) == -1
+    assert L.isoquant_last_launch_count(ctx) == 0
+    torch.cuda.synchronize()
+    assert csd.isoquant_get_status(st.ctx) == 0
+    assert attend() == 0
+    torch.cuda.synchronize()
+    assert csd.isoquant_get_status(st.ctx) == 0
+    out_c, qc = out.cpu(), q.float().cpu()
+    for b in range(st.B):
+        check_pair(st, b, b % st.H, qc, out_c)
