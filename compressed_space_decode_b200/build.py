@@ -47,5 +47,6 @@ def build(force=False, verbose=False, extra=()):
 
 
 if __name__ == "__main__":
-    extra = ["-Xptxas", "-v"] if "-v" in sys.argv else []
+    # -v: register and shared-memory report; --nvtx: NVTX ranges around the C-ABI calls
+    extra = (["-Xptxas", "-v"] if "-v" in sys.argv else []) + (["-DISOQUANT_NVTX"] if "--nvtx" in sys.argv else [])
     print(build(force=True, verbose=True, extra=extra))

@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "isoquant_internal.cuh"
+#include "trace.cuh"
 
 namespace isoquant {
 
@@ -201,6 +202,7 @@ int isoquant_init(isoquant_ctx **out, int num_kv_heads, int head_dim, const int8
 
 int isoquant_init_bits(isoquant_ctx **out, int num_kv_heads, int head_dim, const int8_t *signs, const float *quats,
                        int bits) {
+  ISOQUANT_TRACE("isoquant_init_bits");
   if (out == nullptr || signs == nullptr || quats == nullptr || num_kv_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
   *out = nullptr;
   if (head_dim != kD || bits < 2 || bits > 4) return ISOQUANT_ERR_UNSUPPORTED;
@@ -228,6 +230,7 @@ int isoquant_init_bits(isoquant_ctx **out, int num_kv_heads, int head_dim, const
 }
 
 void isoquant_destroy(isoquant_ctx *ctx) {
+  ISOQUANT_TRACE("isoquant_destroy");
   if (ctx == nullptr) return;
   int prev = -1;
   cudaGetDevice(&prev);
@@ -251,6 +254,7 @@ int isoquant_cache_bytes(const isoquant_ctx *ctx, int num_pages, int page_size, 
 
 int isoquant_compress_kv(isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v, int dtype,
                          int n_tok, const int64_t *slot_mapping, void *stream) {
+  ISOQUANT_TRACE("isoquant_compress_kv");
   if (ctx == nullptr || n_tok < 0) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 0;
   int st = check_cache(cache);
@@ -269,6 +273,7 @@ int isoquant_compress_kv(isoquant_ctx *ctx, const isoquant_cache *cache, const v
 
 int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows, int num_q_heads, float *q_rot,
                       void *stream) {
+  ISOQUANT_TRACE("isoquant_rotate_q");
   if (ctx == nullptr || n_rows < 0 || num_q_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 0;
   if (num_q_heads % ctx->num_kv_heads != 0) return ISOQUANT_ERR_INVALID_ARG;
@@ -286,6 +291,7 @@ int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows, i
 int isoquant_decode_prep(isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v, int n_tok,
                          const int64_t *slot_mapping, const void *q, int dtype, int n_rows, int num_q_heads,
                          float *q_rot, void *stream) {
+  ISOQUANT_TRACE("isoquant_decode_prep");
   if (ctx == nullptr || n_tok < 0 || n_rows < 0 || num_q_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 0;
   int st = check_cache(cache);
@@ -328,6 +334,7 @@ int isoquant_decode_step(isoquant_ctx *ctx, const isoquant_cache *cache, const v
                          const int64_t *slot_mapping, const void *q, int dtype, int batch, int nq, int num_q_heads,
                          const int32_t *page_table, int max_pages, const int32_t *seq_lens, int causal,
                          float scale, void *workspace, size_t ws_bytes, float *out, void *stream) {
+  ISOQUANT_TRACE("isoquant_decode_step");
   if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 0;
   size_t need = 0;
@@ -371,6 +378,7 @@ int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq, int num_
 int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache, const float *q_rot, int batch, int nq,
                             int num_q_heads, const int32_t *page_table, int max_pages, const int32_t *seq_lens,
                             int causal, float scale, void *workspace, size_t ws_bytes, void *stream) {
+  ISOQUANT_TRACE("isoquant_attend_partial");
   if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 0;
   int st = check_cache(cache);
@@ -395,6 +403,7 @@ int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache, cons
 
 int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq, int num_q_heads, const int32_t *seq_lens,
                             int page_size, const void *workspace, size_t ws_bytes, float *out, void *stream) {
+  ISOQUANT_TRACE("isoquant_attend_combine");
   if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 0;
   if (!valid_page_size(page_size)) return ISOQUANT_ERR_UNSUPPORTED;
@@ -414,6 +423,7 @@ int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq, int num_q_head
 int isoquant_attend_decode(isoquant_ctx *ctx, const isoquant_cache *cache, const float *q_rot, int batch, int nq,
                            int num_q_heads, const int32_t *page_table, int max_pages, const int32_t *seq_lens,
                            int causal, float scale, void *workspace, size_t ws_bytes, float *out, void *stream) {
+  ISOQUANT_TRACE("isoquant_attend_decode");
   if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   if (out == nullptr && batch > 0) return ISOQUANT_ERR_INVALID_ARG;
   if (out != nullptr && !aligned(out, 16)) return ISOQUANT_ERR_ALIGNMENT;
@@ -428,6 +438,7 @@ int isoquant_attend_decode(isoquant_ctx *ctx, const isoquant_cache *cache, const
 }
 
 int isoquant_get_status(isoquant_ctx *ctx, uint32_t *status, void *stream) {
+  ISOQUANT_TRACE("isoquant_get_status");
   if (ctx == nullptr || status == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t host = 0;
@@ -442,6 +453,7 @@ int isoquant_get_status(isoquant_ctx *ctx, uint32_t *status, void *stream) {
 int isoquant_last_launch_count(const isoquant_ctx *ctx) { return ctx ? ctx->last_launches : 0; }
 
 int isoquant_selftest_wait(isoquant_ctx *ctx, uint64_t limit_ns, uint64_t *elapsed_ns, void *stream) {
+  ISOQUANT_TRACE("isoquant_selftest_wait");
   if (ctx == nullptr || limit_ns == 0 || limit_ns > kSelftestMaxNs) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 1;
   return launch_wait_selftest(ctx, limit_ns, elapsed_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess

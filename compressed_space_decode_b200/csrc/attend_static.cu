@@ -24,6 +24,7 @@
 #include <mutex>
 
 #include "isoquant_internal.cuh"
+#include "trace.cuh"
 
 namespace isoquant {
 namespace {
@@ -57,6 +58,7 @@ extern "C" int isoquant_attend_decode_static(isoquant_ctx *ctx, const isoquant_c
                                              int batch, int nq, int num_q_heads, const int32_t *page_table,
                                              int max_pages, const int32_t *seq_lens, int causal, float scale,
                                              float *out, void *stream) {
+  ISOQUANT_TRACE("isoquant_attend_decode_static");
   if (ctx == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   ctx->last_launches = 0;
   if (num_q_heads < 1 || nq < 1 || batch < 0 || num_q_heads % ctx->num_kv_heads != 0)

@@ -105,3 +105,19 @@ def test_every_entry_rejects_a_null_context(native):
     assert L.isoquant_last_launch_count(None) == 0
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert native.strerror(code)
+
+
+def test_nvtx_build_compiles(tmp_path):
+    """The optional NVTX-traced build (-DISOQUANT_NVTX) of the C-ABI unit
+    compiles and pulls in the NVTX ranges."""
+    import shutil
+    import subprocess
+    nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+    if not os.path.exists(nvcc) and shutil.which("nvcc") is None:
+        pytest.skip("no nvcc")
+    obj = tmp_path / "api_nvtx.o"
+    subprocess.check_call([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-Xcompiler",
+                           "-fPIC", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include"), "-DISOQUANT_NVTX",
+                           "-c", "-o", str(obj), os.path.join(ROOT, "compressed_space_decode_b200", "csrc", "api.cu")])
+    syms = subprocess.run(["nm", str(obj)], capture_output=True, text=True).stdout
+    assert "nvtx" in syms.lower()
