@@ -681,14 +681,16 @@ def run_prefill(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=500)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gpus", type=int, default=1, help="GPUs (ranks) of the run; N > 1 under torchrun, one shard per rank")
+    ap.add_argument("--steps", type=int, default=5000, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=20, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
+                    help="ours: the CUDA library; reference: the fp64 oracle on the host")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="decode workload name, prefill_attend_* for causal prefill, prefill_32768_kv8_layers48 for compression")
+    ap.add_argument("--e2e-steps", type=int, default=500, help="steps of the end-to-end (host buffers) measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="time budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--bits", type=int, default=3, choices=[2, 3, 4],
                     help="code width of the decode workload (3: the method's; 2 and 4: other widths)")
     args = ap.parse_args()
