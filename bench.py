@@ -241,9 +241,35 @@ def run_ours(args):
     units = multi.sum_over_ranks(units_local, device=dev)
     value = units / (ms / 1e3)
 
+    # the attention call alone, repeated for >= --attn-seconds so that the
+    # roofline rests on thousands of launches and the clock sampler sees
+    # them: CUDA events around every call on the launching stream (median),
+    # over the cache as the timed loop left it (larger than L2)
+    lens_last = lens_all[n_total - 1]
+    n_attn = max(200, int(math.ceil(args.attn_seconds * 1e3 / max(attn_avg_ms, 1e-3))))
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_attn)]
+    attn_launches = 0
+    multi.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    for ea, eb in attn_ev:
+        ea.record(stream)
+        csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, lens_last, ws, out, causal=wl.causal,
+                                   stream=stream)
+        attn_launches += csd.isoquant_last_launch_count(st.ctx)
+        eb.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks_attn = sampler.stop()
+    multi.barrier()
+    loop_ms = sorted(ea.elapsed_time(eb) for ea, eb in attn_ev)
+    attn_med_ms = loop_ms[len(loop_ms) // 2]
+
     # roofline of the attention kernel: algorithmic bytes per launch / duration
-    bytes_per_launch = bytes_per_token_head * units_local / args.steps
-    achieved = bytes_per_launch / (attn_avg_ms / 1e3) / 1e9
+    bytes_per_launch = bytes_per_token_head * int(lens_last.sum().item()) * H
+    bytes_in_step = bytes_per_token_head * units_local / args.steps
+    achieved = bytes_per_launch / (attn_med_ms / 1e3) / 1e9
+    achieved_in_step = bytes_in_step / (attn_avg_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
     # the profiled traffic is that of the 3-bit mma.sync kernel
     traffic = None  # set below once the kernel is known
@@ -296,7 +322,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds, bits=args.bits)
+        cpu = cpu_baseline(wl, budget_s=args.cpu_seconds, bits=args.bits, st=st, dev=dev)
     # the library's kernel choice: mma.sync below 64 query rows per KV head
     # (or with pages under 64 tokens), tcgen05 from there
     rows = wl.nq * (Hq // H)
@@ -330,10 +356,21 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": f"isoquant_attend_decode ({partial_kernel} + k_attend_combine)",
                      "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
-                     "bytes_per_launch": bytes_per_launch, "avg_launch_ms": attn_avg_ms,
+                     "bytes_per_launch": bytes_per_launch, "avg_launch_ms": attn_med_ms,
+                     "launches_timed": n_attn, "launch_ms_p10_p90": [loop_ms[len(loop_ms) // 10],
+                                                                     loop_ms[(9 * len(loop_ms)) // 10]],
+                     "loop": f"{n_attn} attention calls back to back, CUDA events around each (median); "
+                             f"clocks sampled over the loop",
+                     "clocks": clocks_attn,
+                     "achieved_in_step": achieved_in_step, "in_step_launches_timed": len(attn_ms),
                      "frac_of_8TBps": achieved / 8000.0},
         "gpu_launches": kernel_launches,
-        "clocks": clocks,
+        # the timed steps are often too short for nvidia-smi to sample (it
+        # polls every 50 ms); then the clocks of the attention loop that
+        # follows them on the same GPU stand in, and say so
+        "clocks": clocks if clocks.get("samples", 0) > 0 else
+        dict(clocks_attn, note="sampled over the attention-only loop right after the timed steps "
+                               "(the timed steps ended before the first sample)"),
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
@@ -342,7 +379,8 @@ def run_ours(args):
 
 def oracle_sample(wl, b, h, bits=3):
     """Oracle state for one (sequence, KV head) of workload `wl`: its own
-    codes of the context, the appended token and the step's query rows.
+    codes of the context, the appended token and the step's query rows, and
+    how many context coordinates lie within 1e-6 of a decision threshold.
     Inputs come from the seeded generators only."""
     import oracle
     from compressed_space_decode_b200 import synthetic
@@ -351,12 +389,14 @@ def oracle_sample(wl, b, h, bits=3):
     k, v = synthetic.workload_kv_tokens(wl, b, 0, L + 1, device="cuda")
     signs, quats = synthetic.rotation_params(wl.seed, wl.kv_heads)
     s, qt = signs[h].numpy(), quats[h].numpy()
-    kc, kn, _, _ = oracle.compress(s, qt, k[:L, h].double().cpu().numpy(), bits=bits)
-    vc, vn, _, _ = oracle.compress(s, qt, v[:L, h].double().cpu().numpy(), bits=bits)
+    kc, kn, zk, _ = oracle.compress(s, qt, k[:L, h].double().cpu().numpy(), want_z=True, bits=bits)
+    vc, vn, zv, _ = oracle.compress(s, qt, v[:L, h].double().cpu().numpy(), want_z=True, bits=bits)
+    near = [int(oracle.near_boundary(z, 1e-6, bits=bits).sum()) for z in (zk, zv)]
     newk = k[L:L + 1, h].double().cpu().numpy()
     newv = v[L:L + 1, h].double().cpu().numpy()
     q = synthetic.workload_queries(wl, 0, device="cuda")[b, 0, h * G:(h + 1) * G].double().cpu().numpy()
-    return dict(s=s, qt=qt, kc=kc, kn=kn, vc=vc, vn=vn, newk=newk, newv=newv, q=q, L=L, G=G, bits=bits)
+    return dict(s=s, qt=qt, kc=kc, kn=kn, vc=vc, vn=vn, newk=newk, newv=newv, q=q, L=L, G=G, bits=bits, b=b, h=h,
+                near=near)
 
 
 def oracle_step(o):
@@ -375,18 +415,117 @@ def oracle_step(o):
     return oracle.attend(o["s"], o["qt"], o["q"], kc, kn, vc, vn, [o["L"] + 1] * R, bits=o["bits"])
 
 
-def cpu_baseline(wl, budget_s=12.0, bits=3):
+def host_cores():
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_worker(job):
+    """One host process of the all-core oracle leg: wait for the common
+    start, then run whole oracle decode steps until the budget is spent."""
+    sample, start_at, budget_s, max_steps = job
+    while time.time() < start_at:
+        time.sleep(0.001)
+    n, t0 = 0, time.perf_counter()
+    while n < max_steps and (budget_s is None or time.perf_counter() - t0 < budget_s):
+        oracle_step(sample)
+        n += 1
+    return n, time.perf_counter() - t0
+
+
+class OraclePool:
+    """`cores` spawned host processes, each running the oracle's decode step
+    on the sample (processes, not threads: the oracle is single-threaded C
+    behind ctypes; spawned, not forked, since the parent holds a CUDA
+    context)."""
+
+    def __init__(self, sample, cores):
+        import multiprocessing as mp
+        self.sample, self.cores = sample, cores
+        self.pool = mp.get_context("spawn").Pool(cores)
+
+    def run(self, budget_s=None, steps=1):
+        start_at = time.time() + 0.5
+        res = self.pool.map(_oracle_worker, [(self.sample, start_at, budget_s, steps if budget_s is None else 1 << 40)]
+                            * self.cores, chunksize=1)
+        return sum(r[0] for r in res), max(r[1] for r in res)
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def parity_sample(st, o, dev):
+    """The oracle sample's (sequence, KV head) against the GPU path: its
+    context's codes and norms as the library wrote them (mismatches, and
+    coordinates within 1e-6 of a threshold), and one attention call over the
+    same L + 1 tokens with the sample's query rows (max row-normwise error)."""
+    import numpy as np
+    import torch
+
+    import compressed_space_decode_b200 as csd
+    import oracle
+    from compressed_space_decode_b200 import synthetic
+    b, h, L, G, bits = o["b"], o["h"], o["L"], o["G"], o["bits"]
+    res = {"pair": f"sequence {b}, KV head {h}", "vectors": 2 * L, "coords": 2 * L * 128,
+           "near_boundary_1e-6": sum(o["near"])}
+    mism_codes = mism_norms = 0
+    for kv, (oc, on) in enumerate(((o["kc"], o["kn"]), (o["vc"], o["vn"]))):
+        gc, gn = st.gather(b, h, kv, 0, L)
+        gc = gc.numpy().astype(np.uint32)
+        gn = gn.numpy().astype(np.uint16)
+        diff = (gc != oc).any(axis=1)
+        if diff.any():
+            mism_codes += int((oracle.unpack(gc[diff], bits=bits) != oracle.unpack(oc[diff], bits=bits)).sum())
+        mism_norms += int((gn != on).sum())
+    res["code_mismatches"] = mism_codes
+    res["norm_mismatches"] = mism_norms
+    wl = st.wl
+    q = synthetic.workload_queries(wl, 0, device=dev)[b:b + 1].contiguous()
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    csd.isoquant_rotate_q(st.ctx, q.view(-1, st.Hq, 128), q_rot.view(-1, st.Hq, 128))
+    out = torch.empty_like(q_rot)
+    lens = torch.tensor([L + 1], dtype=torch.int32, device=dev)
+    ws = csd.alloc_workspace(st.ctx, 1, 1, st.Hq, device=dev)
+    csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table[b:b + 1].contiguous(), lens, ws, out)
+    torch.cuda.synchronize(dev)
+    got = out[0, 0, h * G:(h + 1) * G].double().cpu().numpy()
+    ref = oracle_step(o)
+    err = np.abs(got - ref).max(axis=1) / np.abs(ref).max(axis=1)
+    res["max_row_rel_err"] = float(err.max())
+    res["tolerance"] = 2e-3
+    return res
+
+
+def cpu_baseline(wl, budget_s=12.0, bits=3, st=None, dev=None):
     """The fp64 oracle, as it stands, on the host cores: a bounded sample of
-    the same decode step (whole (sequence, KV head) units, repeated)."""
+    the same decode step (one (sequence, KV head) unit, repeated), on one
+    core and on every core (one spawned process per core), plus the sample's
+    parity against the GPU path."""
     o = oracle_sample(wl, 0, 0, bits)
     units, t0 = 0, time.perf_counter()
     while time.perf_counter() - t0 < budget_s:
         oracle_step(o)
         units += o["L"] + 1
     dt = time.perf_counter() - t0
-    return {"value": units / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+    one = {"value": units / dt, "unit": UNIT, "cores": 1,
+           "sample": f"{units // (o['L'] + 1)} steps in {dt:.1f} s"}
+    cores = host_cores()
+    pool = OraclePool(o, cores)
+    pool.run(steps=1)  # start-up, untimed
+    n, dt_all = pool.run(budget_s=budget_s)
+    pool.close()
+    line = {"value": n * (o["L"] + 1) / dt_all, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"sequence 0, KV head 0 of the workload (context {o['L'] + 1}, {o['G']} query rows): "
-                      f"compress the appended token + attend, repeated {units // (o['L'] + 1)}x in {dt:.1f} s"}
+                      f"compress the appended token + attend; {cores} host processes ran {n} steps in "
+                      f"{dt_all:.1f} s",
+            "single_core": one}
+    if st is not None:
+        line["parity_sample"] = parity_sample(st, o, dev)
+    return line
 
 
 # ---------------------------------------------------------- reference arm
@@ -423,16 +562,16 @@ def run_reference(args):
         }))
         return
     o = oracle_sample(wl, 0, 0, args.bits)
-    for _ in range(args.warmup):
-        oracle_step(o)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(o)
-    dt = time.perf_counter() - t0
-    units = args.steps * (o["L"] + 1)
+    cores = host_cores()
+    pool = OraclePool(o, cores)
+    pool.run(steps=args.warmup)
+    # each step: every host process runs one oracle decode step
+    _, dt = pool.run(steps=args.steps)  # the slowest process's own time
+    pool.close()
+    units = args.steps * cores * (o["L"] + 1)
     value = units / dt
-    sample = (f"each step: sequence 0, KV head 0 of {wl.name} (context {o['L'] + 1}, {o['G']} query rows), "
-              f"compress the appended token + attend")
+    sample = (f"each step: {cores} host processes each run sequence 0, KV head 0 of {wl.name} (context "
+              f"{o['L'] + 1}, {o['G']} query rows): compress the appended token + attend")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -440,7 +579,7 @@ def run_reference(args):
         "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.q_heads, "kv_heads": wl.kv_heads,
                    "head_dim": 128, "context_start": wl.seq_lens[0], "page_size": wl.page_size,
                    "code_bits": args.bits},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -689,7 +828,10 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="decode workload name, prefill_attend_* for causal prefill, prefill_32768_kv8_layers48 for compression")
     ap.add_argument("--e2e-steps", type=int, default=500, help="steps of the end-to-end (host buffers) measurement")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="time budget of the CPU-oracle baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="time budget of each CPU-oracle baseline leg (one core, then all cores)")
+    ap.add_argument("--attn-seconds", type=float, default=1.0,
+                    help="length of the attention-only loop behind the roofline figure")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--bits", type=int, default=3, choices=[2, 3, 4],
                     help="code width of the decode workload (3: the method's; 2 and 4: other widths)")

@@ -25,6 +25,7 @@ _DTYPES = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
 DEVERR_WAIT_TIMEOUT = 1
 DEVERR_PAGE_RANGE = 2
 DEVERR_SLOT_RANGE = 4
+DEVERR_PLAN_MISMATCH = 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libisoquant.so")
@@ -36,6 +37,7 @@ SYMBOLS = [
     "isoquant_attend_partial", "isoquant_attend_combine", "isoquant_get_status", "isoquant_last_launch_count",
     "isoquant_attend_decode_static", "isoquant_decode_prep", "isoquant_step_workspace_size",
     "isoquant_decode_step", "isoquant_init_bits", "isoquant_codebook_bits", "isoquant_selftest_wait",
+    "isoquant_workspace_size_paged", "isoquant_debug_export_z",
 ]
 
 
@@ -71,6 +73,7 @@ def lib():
             "isoquant_compress_kv": ([vp, cp, vp, vp, i32, i32, vp, vp], i32),
             "isoquant_rotate_q": ([vp, vp, i32, i32, i32, vp, vp], i32),
             "isoquant_workspace_size": ([vp, i32, i32, i32, ctypes.POINTER(sz)], i32),
+            "isoquant_workspace_size_paged": ([vp, i32, i32, i32, i32, ctypes.POINTER(sz)], i32),
             "isoquant_attend_decode": ([vp, cp, vp, i32, i32, i32, vp, i32, vp, i32, ctypes.c_float, vp, sz, vp, vp],
                                        i32),
             "isoquant_attend_partial": ([vp, cp, vp, i32, i32, i32, vp, i32, vp, i32, ctypes.c_float, vp, sz, vp],
@@ -85,6 +88,7 @@ def lib():
             "isoquant_decode_step": ([vp, cp, vp, vp, i32, vp, vp, i32, i32, i32, i32, vp, i32, vp, i32,
                                       ctypes.c_float, vp, sz, vp, vp], i32),
             "isoquant_selftest_wait": ([vp, ctypes.c_uint64, vp, vp], i32),
+            "isoquant_debug_export_z": ([vp, vp, i32, i32, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -264,8 +268,15 @@ def isoquant_workspace_size(ctx, batch, nq, num_q_heads):
     return n.value
 
 
-def alloc_workspace(ctx, batch, nq, num_q_heads, device="cuda"):
-    n = isoquant_workspace_size(ctx, batch, nq, num_q_heads)
+def isoquant_workspace_size_paged(ctx, batch, nq, num_q_heads, page_size):
+    n = ctypes.c_size_t()
+    _check(lib().isoquant_workspace_size_paged(ctx.handle, batch, nq, num_q_heads, page_size, ctypes.byref(n)),
+           "isoquant_workspace_size_paged")
+    return n.value
+
+
+def alloc_workspace(ctx, batch, nq, num_q_heads, device="cuda", page_size=256):
+    n = isoquant_workspace_size_paged(ctx, batch, nq, num_q_heads, page_size)
     return torch.empty(((n + 15) // 16) * 4, dtype=torch.int32, device=device)
 
 
@@ -336,6 +347,14 @@ def isoquant_selftest_wait(ctx, limit_ns, elapsed=None, stream=None):
         ptr = _ptr(elapsed)
     _check(lib().isoquant_selftest_wait(ctx.handle, int(limit_ns), ptr, _stream(stream)),
            "isoquant_selftest_wait")
+
+
+def isoquant_debug_export_z(ctx, x, z, stream=None):
+    """x: [n_tok][H][128] (fp32/bf16/fp16, device); z float32 same shape:
+    the compress kernels' fp32 z = sqrt(128) (R x) / ||x|| (debug only)."""
+    assert x.is_contiguous() and z.is_contiguous() and z.dtype == torch.float32 and z.shape == x.shape
+    _check(lib().isoquant_debug_export_z(ctx.handle, _ptr(x), _dtype(x), x.shape[0], _ptr(z), _stream(stream)),
+           "isoquant_debug_export_z")
 
 
 def isoquant_last_launch_count(ctx):

@@ -3,6 +3,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -114,6 +115,13 @@ int make_shape(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, int 
                AttendShape *s) {
   if (batch < 0 || nq < 1 || num_q_heads < 1) return ISOQUANT_ERR_INVALID_ARG;
   if (num_q_heads % ctx->num_kv_heads != 0) return ISOQUANT_ERR_INVALID_ARG;
+  // the kernels index rows, row groups x sequences and output rows in 32
+  // bits: refuse shapes that would overflow them
+  const int64_t rows = static_cast<int64_t>(nq) * (num_q_heads / ctx->num_kv_heads);
+  const int64_t units = ((rows + 7) / 8) * static_cast<int64_t>(batch);
+  const int64_t out_rows = static_cast<int64_t>(batch) * nq * num_q_heads;
+  if (rows >= INT32_MAX || units >= INT32_MAX || units * ctx->num_kv_heads >= INT32_MAX || out_rows >= INT32_MAX)
+    return ISOQUANT_ERR_INVALID_ARG;
   s->batch = batch;
   s->nq = nq;
   s->q_heads = num_q_heads;
@@ -141,6 +149,14 @@ int attend_workspace_min(const isoquant_ctx *ctx, int batch, int nq, int num_q_h
 }
 
 namespace {
+
+// The library launches on the device that is current; it must be the one
+// the context's parameters live on.
+int check_device(const isoquant_ctx *ctx) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ISOQUANT_ERR_CUDA;
+  return dev == ctx->device ? ISOQUANT_OK : ISOQUANT_ERR_INVALID_ARG;
+}
 
 int check_cache(const isoquant_cache *cache) {
   if (cache == nullptr || cache->codes == nullptr || cache->norms == nullptr) return ISOQUANT_ERR_INVALID_ARG;
@@ -265,6 +281,8 @@ int isoquant_compress_kv(isoquant_ctx *ctx, const isoquant_cache *cache, const v
   if (k == nullptr || v == nullptr || slot_mapping == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   const uintptr_t need = eb == 4 ? 16 : 8;
   if (!aligned(k, need) || !aligned(v, need) || !aligned(slot_mapping, 8)) return ISOQUANT_ERR_ALIGNMENT;
+  st = check_device(ctx);
+  if (st != ISOQUANT_OK) return st;
   cudaError_t e = launch_compress(ctx, cache, k, v, dtype, n_tok, slot_mapping, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
   ctx->last_launches = 1;
@@ -282,8 +300,26 @@ int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows, i
   if (n_rows == 0) return ISOQUANT_OK;
   if (q == nullptr || q_rot == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   if (!aligned(q, eb == 4 ? 16 : 8) || !aligned(q_rot, 16)) return ISOQUANT_ERR_ALIGNMENT;
+  const int dst = check_device(ctx);
+  if (dst != ISOQUANT_OK) return dst;
   cudaError_t e = launch_rotate_q(ctx, q, dtype, n_rows, num_q_heads, q_rot, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
+  ctx->last_launches = 1;
+  return ISOQUANT_OK;
+}
+
+int isoquant_debug_export_z(isoquant_ctx *ctx, const void *x, int dtype, int n_tok, float *z, void *stream) {
+  ISOQUANT_TRACE("isoquant_debug_export_z");
+  if (ctx == nullptr || n_tok < 0) return ISOQUANT_ERR_INVALID_ARG;
+  ctx->last_launches = 0;
+  if (dtype_bytes(dtype) == 0) return ISOQUANT_ERR_UNSUPPORTED;
+  if (n_tok == 0) return ISOQUANT_OK;
+  if (x == nullptr || z == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(z, 16)) return ISOQUANT_ERR_ALIGNMENT;
+  const int st = check_device(ctx);
+  if (st != ISOQUANT_OK) return st;
+  if (launch_export_z(ctx, x, dtype, n_tok, z, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ISOQUANT_ERR_CUDA;
   ctx->last_launches = 1;
   return ISOQUANT_OK;
 }
@@ -309,6 +345,8 @@ int isoquant_decode_prep(isoquant_ctx *ctx, const isoquant_cache *cache, const v
     if (!aligned(q, need) || !aligned(q_rot, 16)) return ISOQUANT_ERR_ALIGNMENT;
   }
   if (n_tok == 0 && n_rows == 0) return ISOQUANT_OK;
+  st = check_device(ctx);
+  if (st != ISOQUANT_OK) return st;
   cudaError_t e = launch_decode_prep(ctx, cache, k, v, n_tok, slot_mapping, q, dtype, n_rows, num_q_heads, q_rot,
                                      static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
@@ -367,9 +405,15 @@ int isoquant_decode_step(isoquant_ctx *ctx, const isoquant_cache *cache, const v
 }
 
 int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, size_t *bytes) {
+  return isoquant_workspace_size_paged(ctx, batch, nq, num_q_heads, 256, bytes);
+}
+
+int isoquant_workspace_size_paged(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, int page_size,
+                                  size_t *bytes) {
   if (ctx == nullptr || bytes == nullptr) return ISOQUANT_ERR_INVALID_ARG;
+  if (!valid_page_size(page_size)) return ISOQUANT_ERR_UNSUPPORTED;
   AttendShape s;
-  int st = make_shape(ctx, batch, nq, num_q_heads, 256, 0, &s);
+  int st = make_shape(ctx, batch, nq, num_q_heads, page_size, 0, &s);
   if (st != ISOQUANT_OK) return st;
   *bytes = attend_workspace_bytes(s);
   return ISOQUANT_OK;
@@ -394,6 +438,11 @@ int isoquant_attend_partial(isoquant_ctx *ctx, const isoquant_cache *cache, cons
   if (!aligned(workspace, 16) || !aligned(q_rot, 4) || !aligned(page_table, 4) || !aligned(seq_lens, 4))
     return ISOQUANT_ERR_ALIGNMENT;
   if (ws_bytes < attend_workspace_min_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
+  // a sequence's pages of all KV heads (plus the tcgen05 kernels' work-free
+  // pages, at most 16 per head) are counted in 32 bits
+  if ((static_cast<int64_t>(max_pages) + 16) * ctx->num_kv_heads >= INT32_MAX) return ISOQUANT_ERR_INVALID_ARG;
+  st = check_device(ctx);
+  if (st != ISOQUANT_OK) return st;
   cudaError_t e = launch_attend_partial(ctx, cache, s, q_rot, page_table, max_pages, seq_lens, scale, workspace,
                                         ws_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
@@ -414,6 +463,8 @@ int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq, int num_q_head
   if (seq_lens == nullptr || workspace == nullptr || out == nullptr) return ISOQUANT_ERR_INVALID_ARG;
   if (!aligned(workspace, 16) || !aligned(out, 16) || !aligned(seq_lens, 4)) return ISOQUANT_ERR_ALIGNMENT;
   if (ws_bytes < attend_workspace_min_bytes(s)) return ISOQUANT_ERR_WORKSPACE;
+  st = check_device(ctx);
+  if (st != ISOQUANT_OK) return st;
   cudaError_t e = launch_attend_combine(ctx, s, seq_lens, workspace, ws_bytes, out, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return ISOQUANT_ERR_CUDA;
   ctx->last_launches = 1;

@@ -27,6 +27,7 @@
 #include <cuda_fp16.h>
 
 #include <cmath>
+#include <mutex>
 
 #include "isoquant_internal.cuh"
 
@@ -111,6 +112,8 @@ struct PartialParams {
   int n_cta;
   int64_t *prefix;  // tcgen05 kernels: pages before each (stream, sequence) unit
   int vpages;       // tcgen05 kernels: work-free pages that follow each (unit, head) block
+  uint32_t *plan;   // first word of the workspace header: receives plan_tag
+  uint32_t plan_tag;
 };
 
 struct CombineParams {
@@ -122,6 +125,9 @@ struct CombineParams {
   int rps;  // query rows per stream: 8 (mma.sync kernel), 64 or 128 (tcgen05 kernels)
   const int64_t *prefix;  // null for the mma.sync kernel
   int vpages;             // as in PartialParams
+  uint32_t *status;
+  const uint32_t *plan;   // the tag the partial kernel wrote
+  uint32_t plan_tag;      // the tag of the plan this combine expects
 };
 
 // ------------------------------------------------------------------ PTX
@@ -297,7 +303,8 @@ __device__ __forceinline__ int unit_horizon(const PartialParams &p, int rps, int
 // pages is followed by vpages work-free ones, so that the split balances
 // work rather than pages (a causal prefill's early streams are one or two
 // tiles long).  (Units and the pages of one unit are counted in 32 bits:
-// the host keeps streams * batch and max_pages * kv_heads below 2^31.)
+// make_shape and isoquant_attend_partial refuse shapes where row groups x
+// sequences x KV heads or (max_pages + 16) x KV heads reach 2^31 - 1.)
 __device__ __forceinline__ int64_t unit_pages(const PartialParams &p, int rps, int u) {
   const int rg = u / p.B, b = u - rg * p.B;
   const int np = pages_of(unit_horizon(p, rps, rg, b), p.page_size);
@@ -399,12 +406,21 @@ __device__ void tile_locate(const PartialParams &p, int rps, int64_t *scratch, i
 // so that 32 lanes with 32 different indices hit 32 different banks.
 __shared__ __align__(16) uint32_t s_lut[64 * 32];
 
+// x >> SH for SH >= 0, x << -SH otherwise (SH a compile-time constant).
+// (Shifting by multiplication on the FMA pipe instead, to unload the
+// half-rate ALU pipe, was measured slower: the high-word multiplies stalled
+// instruction dispatch.)
+template <int SH>
+__device__ __forceinline__ uint32_t shifted(uint32_t x) {
+  static_assert(SH > -32 && SH < 32, "shift range");
+  if constexpr (SH < 0) return x << (-SH);
+  else return x >> SH;
+}
 // Byte offset of entry ((x >> (SH + 7)) & 63) for this lane: the entry index
 // lands in bits 7..12 and the lane's bank in bits 2..6, so one AND-OR forms it.
 template <int SH>
 __device__ __forceinline__ uint32_t lut_off(uint32_t x, uint32_t lane4) {
-  const uint32_t y = (SH >= 0) ? (x >> (SH >= 0 ? SH : 0)) : (x << (SH < 0 ? -SH : 0));
-  return (y & 0x1F80u) | lane4;
+  return (shifted<SH>(x) & 0x1F80u) | lane4;
 }
 __device__ __forceinline__ uint32_t lut_at(uint32_t off) {
   return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(s_lut) + off);
@@ -479,8 +495,7 @@ __device__ __forceinline__ uint32_t k_pair_c(const uint4 (&kw)[4], int j, uint32
 // bit 2 * BITS * (k mod P); the table has 2^(2 BITS) entries.
 template <int SH, uint32_t MASK>
 __device__ __forceinline__ uint32_t lut_off_m(uint32_t x, uint32_t lane4) {
-  const uint32_t y = (SH >= 0) ? (x >> (SH >= 0 ? SH : 0)) : (x << (SH < 0 ? -SH : 0));
-  return (y & MASK) | lane4;
+  return (shifted<SH>(x) & MASK) | lane4;
 }
 __device__ __forceinline__ uint32_t lut_at2(const char *lut, uint32_t off) {
   return *reinterpret_cast<const uint32_t *>(lut + off);
@@ -491,16 +506,25 @@ __device__ __forceinline__ uint32_t k_pair_w(const uint4 (&kw)[4], int j, uint32
   constexpr uint32_t kMask = ((1u << (2 * BITS)) - 1u) << 7;
   return lut_at2(lut, lut_off_m<2 * BITS * (K % kPpw) - 7, kMask>(u4_at(kw[K / kPpw], j), lane4));
 }
+// Slot K of a merged word, looked up
+template <int BITS, uint32_t MASK, int K>
+__device__ __forceinline__ uint32_t merged_pair(uint32_t e, uint32_t lane4, const char *lut) {
+  return lut_at2(lut, lut_off_m<2 * BITS * K - 7, MASK>(e, lane4));
+}
 // The kPpw 2*BITS-bit slots of a merged word, looked up in order
 template <int BITS>
 __device__ __forceinline__ void merged_pairs(uint32_t e, uint32_t lane4, const char *lut, uint32_t *out) {
   constexpr int kPpw = 16 / BITS;
   constexpr uint32_t kMask = ((1u << (2 * BITS)) - 1u) << 7;
-#pragma unroll
-  for (int k = 0; k < kPpw; ++k) {
-    const int sh = 2 * BITS * k - 7;
-    const uint32_t y = sh >= 0 ? (e >> sh) : (e << -sh);
-    out[k] = lut_at2(lut, (y & kMask) | lane4);
+  out[0] = merged_pair<BITS, kMask, 0>(e, lane4, lut);
+  out[1] = merged_pair<BITS, kMask, 1>(e, lane4, lut);
+  out[2] = merged_pair<BITS, kMask, 2>(e, lane4, lut);
+  out[3] = merged_pair<BITS, kMask, 3>(e, lane4, lut);
+  if constexpr (kPpw > 4) {
+    out[4] = merged_pair<BITS, kMask, 4>(e, lane4, lut);
+    out[5] = merged_pair<BITS, kMask, 5>(e, lane4, lut);
+    out[6] = merged_pair<BITS, kMask, 6>(e, lane4, lut);
+    out[7] = merged_pair<BITS, kMask, 7>(e, lane4, lut);
   }
 }
 template <int BITS>
@@ -667,6 +691,14 @@ __device__ __forceinline__ void merge_rows(const float *records, int64_t pair, i
   }
 }
 
+// The partial kernel of a call records which plan (kernel, rows per stream,
+// streams, CTAs) laid out the records, so that a combine launched with
+// another plan (a different workspace size passed to the two halves) sees
+// the mismatch instead of merging the wrong records.
+__device__ __forceinline__ void write_plan_tag(const PartialParams &p) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.plan = p.plan_tag;
+}
+
 // ------------------------------------------------------------ partial kernel
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const PartialParams p) {
@@ -704,6 +736,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
   // the set-up above touches only shared memory; global memory from here on
   pdl_trigger();
   pdl_wait();
+  write_plan_tag(p);
   // CTA's page range [gs, ge) and where it starts
   if (warp == 0) {
     const int64_t pb = pages_before(p.seq_lens, p.B, ps, lane);
@@ -1022,8 +1055,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
               const uint32_t wb = u4_at(Bv, e0), wb1 = u4_at(Bv, e0 + 1);
               const uint32_t wz = u4_at(Z, e0), wz1 = u4_at(Z, e0 + 1);
               // merge two tokens' words: 6-bit slot k = (code of tok a, code of tok b)
-              const uint32_t e_even = (wa & M) | ((wa1 << 3) & ~M);
-              const uint32_t e_odd = ((wa >> 3) & M) | (wa1 & ~M);
+              const uint32_t e_even = (wa & M) | (shifted<-3>(wa1) & ~M);
+              const uint32_t e_odd = (shifted<3>(wa) & M) | (wa1 & ~M);
               const uint32_t e_half = ((wb >> (3 * par)) & M) | ((wb1 << (3 - 3 * par)) & ~M);
               word_pairs(e_even, lane4, va[half] + 0);
               word_pairs(e_odd, lane4, va[half] + 5);
@@ -1063,8 +1096,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
               for (int i = 0; i < L::kVWords; ++i) {
                 const uint4 &A = tp < 2 ? vw[i][0] : vw[i][1];
                 const uint32_t wa = u4_at(A, e0), wb = u4_at(A, e0 + 1);
-                const uint32_t e_even = (wa & M) | ((wb << BITS) & ~M);
-                const uint32_t e_odd = ((wa >> BITS) & M) | (wb & ~M);
+                const uint32_t e_even = (wa & M) | (shifted<-BITS>(wb) & ~M);
+                const uint32_t e_odd = (shifted<BITS>(wa) & M) | (wb & ~M);
                 merged_pairs<BITS>(e_even, lane4, lutb, va[half] + 8 * i);
                 merged_pairs<BITS>(e_odd, lane4, lutb, va[half] + 8 * i + L::kPpw);
               }
@@ -1387,6 +1420,7 @@ __global__ void __launch_bounds__(kTThreads, kTCtasPerSm) k_attend_tiles(const P
   }
   pdl_trigger();
   pdl_wait();
+  write_plan_tag(p);
   __shared__ int64_t tloc[4 + kTThreads / 32];
   tile_locate<kTThreads>(p, kTRows, tloc + 4, tloc);
   tc_fence_after();
@@ -1862,6 +1896,7 @@ __global__ void __launch_bounds__(wide_threads<BITS>(), 1) k_attend_wide(const P
   }
   pdl_trigger();
   pdl_wait();
+  write_plan_tag(p);
   tile_locate<kWThreads>(p, kWRows, loc + 4, loc);
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -2249,6 +2284,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const uint32_t grp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const bool plan_ok = __ldcg(p.plan) == p.plan_tag;
   const uint32_t per_bi = static_cast<uint32_t>(p.Hq / NR);
   const uint32_t n_groups = static_cast<uint32_t>(p.B) * p.nq * per_bi;
   if (grp_id >= n_groups) return;
@@ -2268,6 +2304,14 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
     dsts[k] = p.out + (static_cast<int64_t>(bi) * p.Hq + hq0 + k) * kD + 4 * lane;
   }
 
+  if (!plan_ok) {
+    // the records were laid out by another plan (the two halves were given
+    // different workspace sizes): flag it and output zeros, merge nothing
+    if (lane == 0) set_status(p.status, ISOQUANT_DEVERR_PLAN_MISMATCH);
+#pragma unroll
+    for (int k = 0; k < NR; ++k) *reinterpret_cast<float4 *>(dsts[k]) = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
   int np;
   int64_t g0, total;
   if (p.prefix != nullptr) {
@@ -2334,24 +2378,42 @@ TilePlan tile_plan(const AttendShape &s, int num_sms) {
   t.bytes = t.prefix_off + (static_cast<size_t>(t.streams) * s.batch + 1) * sizeof(int64_t);
   return t;
 }
+// the mma.sync kernel's records (every shape can run on it)
+size_t mma_bytes(const AttendShape &s) { return kWsHeader + s.slots * kRecordFloats * sizeof(float); }
+// The plan a call runs: the tcgen05 kernel its shape selects when that
+// kernel's records fit the workspace, else the mma.sync kernel.
 TilePlan use_tiles(const isoquant_ctx *ctx, const AttendShape &s, size_t ws_bytes) {
   TilePlan t = tile_plan(s, ctx->num_sms);
   if (t.kind != 0 && t.bytes > ws_bytes) t.kind = 0;
   return t;
 }
+// Tag of a plan, written to the workspace header by the partial kernel and
+// checked by the combine kernel.
+uint32_t plan_tag(const AttendShape &s, const TilePlan &t, int n_cta, int rg) {
+  uint64_t h = 0x9E3779B97F4A7C15ull;
+  const int64_t f[] = {t.kind, t.kind ? t.rps : 8, rg, n_cta, t.vpages, s.batch, s.nq, s.q_heads, s.kv_heads,
+                       s.page_size};
+  for (int64_t v : f) {
+    h ^= static_cast<uint64_t>(v) + 0x632BE59BD9B4E019ull + (h << 6) + (h >> 2);
+  }
+  return static_cast<uint32_t>(h ^ (h >> 32)) | 1u;
+}
 }  // namespace
 
 size_t attend_workspace_min_bytes(const AttendShape &s) {
-  // the mma.sync kernel's records (every shape can run on it)
-  return kWsHeader + s.slots * kRecordFloats * sizeof(float);
+  // the smaller of the two plans: any workspace of at least this size runs
+  // one of them
+  const size_t mma = mma_bytes(s);
+  const TilePlan t = tile_plan(s, s.n_cta / kCtasPerSm);
+  return t.kind != 0 && t.bytes < mma ? t.bytes : mma;
 }
 
 size_t attend_workspace_bytes(const AttendShape &s) {
-  // room for the tcgen05 kernels' records and unit prefix too, when the
-  // shape can use them
-  const size_t mma = attend_workspace_min_bytes(s);
+  // the records of the kernel the shape runs on: the tcgen05 plan from 64
+  // query rows per KV head (pages of 64 tokens or more), else the mma.sync
+  // kernel's
   const TilePlan t = tile_plan(s, s.n_cta / kCtasPerSm);
-  return t.kind != 0 && t.bytes > mma ? t.bytes : mma;
+  return t.kind != 0 ? t.bytes : mma_bytes(s);
 }
 
 namespace {
@@ -2380,20 +2442,30 @@ cudaError_t launch_tcgen05(int kind, const PartialParams &p, cudaStream_t stream
     return launch_pdl(k_attend_wide<BITS>, dim3(p.n_cta), dim3(wide_threads<BITS>()), wide_smem_bytes<BITS>(), stream, p);
   return launch_pdl(k_attend_tiles<BITS>, dim3(p.n_cta), dim3(kTThreads), kTSmemBytes, stream, p);
 }
+
+// Kernel attributes are per device: set them once on each device (the one
+// current at the call, which the entry points check is the context's).
+constexpr int kMaxConfigDevices = 64;
+std::mutex g_config_mutex;
+bool g_configured[kMaxConfigDevices] = {};
+cudaError_t configure_device(int device) {
+  if (device < 0 || device >= kMaxConfigDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_config_mutex);
+  if (g_configured[device]) return cudaSuccess;
+  cudaError_t e = configure_width<3>();
+  if (e == cudaSuccess) e = configure_width<2>();
+  if (e == cudaSuccess) e = configure_width<4>();
+  if (e == cudaSuccess) g_configured[device] = true;
+  return e;
+}
 }  // namespace
 
 cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache *cache, const AttendShape &s,
                                   const float *q_rot, const int32_t *page_table, int max_pages,
                                   const int32_t *seq_lens, float scale, void *ws, size_t ws_bytes,
                                   cudaStream_t stream) {
-  static int configured_device = -1;
-  if (configured_device != ctx->device) {
-    cudaError_t e = configure_width<3>();
-    if (e == cudaSuccess) e = configure_width<2>();
-    if (e == cudaSuccess) e = configure_width<4>();
-    if (e != cudaSuccess) return e;
-    configured_device = ctx->device;
-  }
+  cudaError_t ce = configure_device(ctx->device);
+  if (ce != cudaSuccess) return ce;
   PartialParams p{};
   p.codes = cache->codes;
   p.norms = cache->norms;
@@ -2418,12 +2490,16 @@ cudaError_t launch_attend_partial(const isoquant_ctx *ctx, const isoquant_cache 
   p.status = ctx->status;
   p.n_cta = s.n_cta;
   p.prefix = nullptr;
+  p.plan = static_cast<uint32_t *>(ws);
   const TilePlan t = use_tiles(ctx, s, ws_bytes);
   if (t.kind != 0) {
     p.RG = t.streams;
     p.n_cta = t.n_cta;
     p.vpages = t.vpages;
     p.prefix = reinterpret_cast<int64_t *>(static_cast<char *>(ws) + t.prefix_off);
+  }
+  p.plan_tag = plan_tag(s, t, p.n_cta, p.RG);
+  if (t.kind != 0) {
     switch (p.bits) {
       case 2: return launch_tcgen05<2>(t.kind, p, stream);
       case 4: return launch_tcgen05<4>(t.kind, p, stream);
@@ -2454,6 +2530,8 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
   p.n_cta = s.n_cta;
   p.rps = 8;
   p.prefix = nullptr;
+  p.status = ctx->status;
+  p.plan = static_cast<const uint32_t *>(ws);
   const TilePlan t = use_tiles(ctx, s, ws_bytes);
   if (t.kind != 0) {
     p.RG = t.streams;
@@ -2462,6 +2540,7 @@ cudaError_t launch_attend_combine(const isoquant_ctx *ctx, const AttendShape &s,
     p.vpages = t.vpages;
     p.prefix = reinterpret_cast<const int64_t *>(static_cast<const char *>(ws) + t.prefix_off);
   }
+  p.plan_tag = plan_tag(s, t, p.n_cta, p.RG);
   // rows per warp: one while there are few rows (decode: a row's merge has
   // many split records, and more warps overlap more of them); with many
   // rows (prefill: one or two records each), the largest of 8, 4, 2 that

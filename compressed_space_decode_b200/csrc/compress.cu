@@ -15,10 +15,12 @@ namespace isoquant {
 namespace {
 
 // Coordinates whose fp32 z lies closer than this to a threshold are
-// re-derived in fp64.  The fp32 rotation error in z is below 1e-6 (7
-// butterfly stages plus a 4-term product, each rounding at 2^-24 of
-// quantities bounded by sqrt(128) |x| / n), so every code decided on the
-// fast path is the code of the exact z.
+// re-derived in fp64.  The fp32 rotation error in z (7 butterfly stages, a
+// 4-term product and 1/n, each rounding at 2^-24 of quantities bounded by
+// sqrt(128) |x| / n) measures about 1e-6 at most (isoquant_debug_export_z
+// against the exact z: 1.04e-6 for fp32 inputs, 7e-7 for bf16/fp16 ones),
+// a tenth of this band, so every code decided on the fast path is the code
+// of the exact z.
 constexpr float kRecheckBand = 1e-5f;
 
 __device__ __forceinline__ void load4(const float *p, float (&x)[4]) {
@@ -184,6 +186,59 @@ __device__ __forceinline__ void pack_store_wide(uint64_t cbits, int q, bool stor
   }
 }
 
+// The fp32 fast path of one lane group's vector, shared by the compress
+// kernels and the z export: the squared norm (exact squares of bf16/fp16
+// inputs, a 7-level tree: 4 in the lane, 3 across the group), 1/n from the
+// hardware reciprocal square root plus one Newton step (~1e-7), the signs
+// and the unnormalised WHT in place, then z of coordinate 16q + 4k + r as
+// (row r of SO(4) block 4q + k) . x / n.  sqrt(128) of the normalised Hn
+// cancels against the sqrt(128) of z = sqrt(128) * y / n.
+struct FastNorm {
+  float ssf, n32, inv;
+};
+__device__ __forceinline__ FastNorm fast_norm(const float (&x)[16]) {
+  float sq[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) sq[i] = x[i] * x[i];
+#pragma unroll
+  for (int s = 8; s >= 1; s >>= 1)
+#pragma unroll
+    for (int i = 0; i < s; ++i) sq[i] += sq[i + s];
+  float ssf = sq[0];
+  ssf += __shfl_xor_sync(0xffffffffu, ssf, 1);
+  ssf += __shfl_xor_sync(0xffffffffu, ssf, 2);
+  ssf += __shfl_xor_sync(0xffffffffu, ssf, 4);
+  FastNorm f;
+  f.ssf = ssf;
+  f.n32 = sqrtf(ssf);
+  const float rs = rsqrtf(ssf);
+  f.inv = rs * (1.5f - 0.5f * ssf * rs * rs);
+  return f;
+}
+__device__ __forceinline__ void fast_signs_wht(float (&x)[16], uint32_t sbits, int q) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(__float_as_uint(x[i]) ^ (((sbits >> i) & 1u) << 31));
+  wht128_wide(x, q);
+}
+__device__ __forceinline__ float fast_z(const float (&mrow)[4][16], const float (&x)[16], int k, int r, float inv) {
+  const float yr = fmaf(mrow[k][4 * r + 3], x[4 * k + 3],
+                        fmaf(mrow[k][4 * r + 2], x[4 * k + 2],
+                             fmaf(mrow[k][4 * r + 1], x[4 * k + 1], mrow[k][4 * r] * x[4 * k])));
+  return yr * inv;
+}
+// The lane's sign bits (coordinates 16q..16q+15) and SO(4) blocks 4q..4q+3.
+__device__ __forceinline__ void lane_blocks(const HeadParams &hp, int q, uint32_t &sbits, float (&mrow)[4][16]) {
+  sbits = (hp.sign_bits[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 row = reinterpret_cast<const float4 *>(hp.m32[4 * q + k])[r];
+      mrow[k][4 * r] = row.x; mrow[k][4 * r + 1] = row.y; mrow[k][4 * r + 2] = row.z; mrow[k][4 * r + 3] = row.w;
+    }
+  }
+}
+
 // The fp64 path for one vector, by the whole warp (lane l: coordinates
 // 4l..4l+3): norm, rotation and codes all in fp64.  Used for the few vectors
 // whose fp16 norm rounding or codes the fp32 fast path cannot decide.
@@ -256,16 +311,9 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
   const int grp = lane >> 3, q = lane & 7;
 
   // this lane's sign bits and SO(4) blocks 4q..4q+3, for the whole strip
-  const uint32_t sbits = (hp.sign_bits[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+  uint32_t sbits;
   float mrow[4][16];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float4 row = reinterpret_cast<const float4 *>(hp.m32[4 * q + k])[r];
-      mrow[k][4 * r] = row.x; mrow[k][4 * r + 1] = row.y; mrow[k][4 * r + 2] = row.z; mrow[k][4 * r + 3] = row.w;
-    }
-  }
+  lane_blocks(hp, q, sbits, mrow);
   // the positive thresholds (the codebook is symmetric; the middle one is 0)
   float tp[kHalf - 1];
 #pragma unroll
@@ -293,18 +341,8 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
     // (4 levels in the lane, 3 across the group) is within 7 * 2^-24
     // relative; the fp16 norm is decided in fp32 unless n lies within 1e-6
     // (relative) of a rounding midpoint, or is huge, tiny or not finite
-    float sq[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) sq[i] = x[i] * x[i];
-#pragma unroll
-    for (int s = 8; s >= 1; s >>= 1)
-#pragma unroll
-      for (int i = 0; i < s; ++i) sq[i] += sq[i + s];
-    float ssf = sq[0];
-    ssf += __shfl_xor_sync(0xffffffffu, ssf, 1);
-    ssf += __shfl_xor_sync(0xffffffffu, ssf, 2);
-    ssf += __shfl_xor_sync(0xffffffffu, ssf, 4);
-    const float n32 = sqrtf(ssf);
+    const FastNorm fn = fast_norm(x);
+    const float ssf = fn.ssf, n32 = fn.n32;
     const __half h32 = __float2half_rn(fminf(n32, 65504.f));
     const float hv = __half2float(h32);
     const uint16_t hb = __half_as_ushort(h32);
@@ -312,15 +350,10 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
     const float dn = hb > 0 ? __half2float(__ushort_as_half(static_cast<uint16_t>(hb - 1))) : 0.f;
     const float mid = n32 >= hv ? 0.5f * (hv + up) : 0.5f * (hv + dn);
     bool slow = !(ssf > 1e-30f && n32 < 65000.f && fabsf(n32 - mid) > 1e-6f * n32);
-    // 1/n: hardware reciprocal square root plus one Newton step (~1e-7)
-    const float rs = rsqrtf(ssf);
-    const float inv = rs * (1.5f - 0.5f * ssf * rs * rs);
+    const float inv = fn.inv;
 
-    // z = (B H D x) / n; sqrt(128) of the normalised Hn cancels against the
-    // sqrt(128) of z = sqrt(128) * y / n.
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(__float_as_uint(x[i]) ^ (((sbits >> i) & 1u) << 31));
-    wht128_wide(x, q);
+    // z = (B H D x) / n
+    fast_signs_wht(x, sbits, q);
     // codes from |z| and the positive thresholds (the codebook is
     // symmetric): z > 0 -> half + #{|z| > t}, otherwise half - 1 - #{|z| >= t}
     uint64_t cbits = 0;
@@ -329,10 +362,7 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
     for (int k = 0; k < 4; ++k) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        const float yr = fmaf(mrow[k][4 * r + 3], x[4 * k + 3],
-                              fmaf(mrow[k][4 * r + 2], x[4 * k + 2],
-                                   fmaf(mrow[k][4 * r + 1], x[4 * k + 1], mrow[k][4 * r] * x[4 * k])));
-        const float z = yr * inv;
+        const float z = fast_z(mrow, x, k, r, inv);
         const float a = fabsf(z);
         uint32_t gt = 0, ge = 0;
         bool nr = a < kRecheckBand;
@@ -391,6 +421,45 @@ __global__ void __launch_bounds__(256, 2) k_compress(const CompressArgs g) {
   pdl_trigger();
   pdl_wait();
   compress_warp<T, BITS>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), threadIdx.x & 31);
+}
+
+// Debug export of the fast path's fp32 z: the same lane-group layout and the
+// same helpers as compress_warp, one vector per lane group, every
+// coordinate's z (fp32, before any fp64 re-check) written to
+// z[(t * H + h) * 128 + j].
+template <typename T>
+__global__ void __launch_bounds__(256) k_export_z(const HeadParams *params, const T *x, int n_tok, int H,
+                                                  float *z) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, grp = lane >> 3, q = lane & 7;
+  const int64_t vec = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + grp;
+  // whole warps exit together (the helpers shuffle within the group)
+  if ((vec & ~int64_t(3)) >= static_cast<int64_t>(n_tok) * H) return;
+  const bool live = vec < static_cast<int64_t>(n_tok) * H;
+  const int h = live ? static_cast<int>(vec % H) : 0;
+  uint32_t sbits;
+  float mrow[4][16];
+  lane_blocks(params[h], q, sbits, mrow);
+  float v[16];
+  if (live) {
+    load16(x + vec * kD + 16 * q, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+  }
+  const FastNorm fn = fast_norm(v);
+  fast_signs_wht(v, sbits, q);
+  float out[16];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) out[4 * k + r] = fn.ssf > 0.f ? fast_z(mrow, v, k, r, fn.inv) : 0.f;
+  if (live) {
+    float4 *dst = reinterpret_cast<float4 *>(z + vec * kD + 16 * q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_float4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+  }
 }
 
 struct RotateArgs {
@@ -540,6 +609,27 @@ cudaError_t launch_rotate_q(const isoquant_ctx *ctx, const void *q, int dtype, i
     case ISOQUANT_F32: return launch_pdl(k_rotate_q<float>, grid, block, 0, stream, g);
     case ISOQUANT_BF16: return launch_pdl(k_rotate_q<__nv_bfloat16>, grid, block, 0, stream, g);
     default: return launch_pdl(k_rotate_q<__half>, grid, block, 0, stream, g);
+  }
+}
+
+cudaError_t launch_export_z(const isoquant_ctx *ctx, const void *x, int dtype, int n_tok, float *z,
+                            cudaStream_t stream) {
+  const int64_t warps = (static_cast<int64_t>(n_tok) * ctx->num_kv_heads + 3) / 4;
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  const int H = ctx->num_kv_heads;
+  switch (dtype) {
+    case ISOQUANT_F32:
+      return launch_pdl(k_export_z<float>, grid, block, 0, stream, ctx->params, static_cast<const float *>(x), n_tok,
+                        H, z);
+    case ISOQUANT_BF16:
+      return launch_pdl(k_export_z<__nv_bfloat16>, grid, block, 0, stream, ctx->params,
+                        static_cast<const __nv_bfloat16 *>(x), n_tok, H, z);
+    default:
+      return launch_pdl(k_export_z<__half>, grid, block, 0, stream, ctx->params, static_cast<const __half *>(x),
+                        n_tok, H, z);
   }
 }
 

@@ -67,6 +67,8 @@ cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache
                             cudaStream_t stream);
 cudaError_t launch_rotate_q(const isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
                             int num_q_heads, float *q_rot, cudaStream_t stream);
+cudaError_t launch_export_z(const isoquant_ctx *ctx, const void *x, int dtype, int n_tok, float *z,
+                            cudaStream_t stream);
 cudaError_t launch_decode_prep(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k,
                                const void *v, int n_tok, const int64_t *slot_mapping, const void *q,
                                int dtype, int n_rows, int num_q_heads, float *q_rot, cudaStream_t stream);
@@ -80,8 +82,9 @@ struct AttendShape {
 constexpr size_t kWsHeader = 256;
 constexpr size_t kRecordFloats = 8 * 2 + 8 * kD;  // (m,l) x 8 rows, o[8][128]
 
-// Workspace sizes: the full size (room for either attention kernel's
-// records) and the minimum any call accepts (the mma.sync kernel's).
+// Workspace sizes: the records of the kernel the shape runs on with an
+// ample workspace, and the minimum any call accepts (the smaller of the
+// tcgen05 plan and the mma.sync records).
 size_t attend_workspace_bytes(const AttendShape &s);
 size_t attend_workspace_min_bytes(const AttendShape &s);
 int attend_workspace_min(const isoquant_ctx *ctx, int batch, int nq, int num_q_heads, size_t *bytes);

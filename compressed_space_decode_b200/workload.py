@@ -77,7 +77,7 @@ class DecodeState:
         return (pages * self.ps + t % self.ps).to(self.device)
 
     def workspace(self, nq=None):
-        return alloc_workspace(self.ctx, self.B, nq or self.wl.nq, self.Hq, device=self.device)
+        return alloc_workspace(self.ctx, self.B, nq or self.wl.nq, self.Hq, device=self.device, page_size=self.ps)
 
     # ----------------------------------------------------- canonical views
     def gather(self, b, h, kv, t0, t1):

@@ -62,6 +62,8 @@ typedef enum {
 #define ISOQUANT_DEVERR_WAIT_TIMEOUT 1u   /* a bounded pipeline wait expired */
 #define ISOQUANT_DEVERR_PAGE_RANGE 2u     /* page_table entry outside [0, num_pages) */
 #define ISOQUANT_DEVERR_SLOT_RANGE 4u     /* slot_mapping entry outside the cache */
+#define ISOQUANT_DEVERR_PLAN_MISMATCH 8u  /* attend_combine given another workspace size than
+                                             attend_partial: records not merged, zeros written */
 
 typedef enum {
   ISOQUANT_F32 = 0,
@@ -131,7 +133,12 @@ int isoquant_codebook_bits(int bits, float *levels, float *thresholds);
 int isoquant_cache_bytes(const isoquant_ctx *ctx, int num_pages, int page_size,
                          size_t *code_bytes, size_t *norm_bytes);
 
-/* Rotate, quantize, pack and append K and V vectors into the paged cache.
+/* Rotate, quantize, pack and append K and V vectors into the paged cache
+ * (RotaryQuant, Abstract: each KV vector is isotropized by the
+ * Walsh-Hadamard transform and the block-diagonal SO(4) rotations, then
+ * scalar-quantized to 3 bits; the quantizer -- per-vector fp16 norm,
+ * Lloyd-Max levels, ten codes per word -- is the one stated at the top of
+ * this file, where the pages leave it open).
  *   k, v:  device [n_tok][num_kv_heads][128] of `dtype` (F32, BF16, F16),
  *          contiguous, 8-byte aligned.
  *   slot_mapping: device int64 [n_tok], slot = page * page_size + offset;
@@ -143,21 +150,38 @@ int isoquant_compress_kv(isoquant_ctx *ctx, const isoquant_cache *cache,
                          const void *k, const void *v, int dtype, int n_tok,
                          const int64_t *slot_mapping, void *stream);
 
-/* q_rot = R q for every row: q device [n_rows][num_q_heads][128] of dtype,
- * q_rot device float [n_rows][num_q_heads][128].  Query head h uses the
- * rotation of KV head h / (num_q_heads / num_kv_heads). */
+/* q_rot = R q for every row (RotaryQuant, Abstract: scores are formed in the
+ * rotated space, so the query takes the same R = B Hn D as the keys of its
+ * head; <R q, R k> = <q, k> because R is orthogonal).
+ *   q:     device [n_rows][num_q_heads][128] of dtype (F32, BF16, F16),
+ *          contiguous, 8-byte aligned (16 for F32);
+ *   q_rot: device float [n_rows][num_q_heads][128], 16-byte aligned,
+ *          caller-owned.
+ * Query head h uses the rotation of KV head h / (num_q_heads /
+ * num_kv_heads).  Errors: INVALID_ARG (null, n_rows < 0, num_q_heads not a
+ * multiple of num_kv_heads), UNSUPPORTED (dtype), ALIGNMENT, CUDA. */
 int isoquant_rotate_q(isoquant_ctx *ctx, const void *q, int dtype, int n_rows,
                       int num_q_heads, float *q_rot, void *stream);
 
 /* Workspace bytes isoquant_attend_decode (and the partial/combine pair)
- * needs for this shape: a 256-byte header and one partial record of
- * (16 + 8 * 128) floats per slot, a slot per CTA plus one per
- * (row group, sequence, KV head) pair; with 64 or more query rows per KV
- * head (nq * num_q_heads / num_kv_heads), room for the tensor-core
- * kernels' records and their work prefix too.  A smaller workspace that
- * still holds the first part runs the mma.sync kernel. */
+ * needs for this shape with pages of 64 tokens or more: a 256-byte header,
+ * then the partial records of (16 + 8 * 128) floats of the kernel the shape
+ * runs on.  Below 64 query rows per KV head (nq * num_q_heads /
+ * num_kv_heads) that is the mma.sync kernel: a record per CTA plus one per
+ * (8-row group, sequence, KV head).  From 64 rows it is a tcgen05 kernel:
+ * 8 or 16 records per (CTA or 64/128-row stream, sequence, KV head) slot
+ * and its work prefix.  A workspace too small for the tcgen05 plan but
+ * large enough for the mma.sync records runs the mma.sync kernel; calls
+ * accept any workspace that holds one of the two. */
 int isoquant_workspace_size(const isoquant_ctx *ctx, int batch, int nq,
                             int num_q_heads, size_t *bytes);
+
+/* isoquant_workspace_size for a given page size (32, 64, 128 or 256):
+ * caches of 32-token pages always run the mma.sync kernel, whose records a
+ * long prefill needs more room for.  Errors: INVALID_ARG, UNSUPPORTED. */
+int isoquant_workspace_size_paged(const isoquant_ctx *ctx, int batch, int nq,
+                                  int num_q_heads, int page_size,
+                                  size_t *bytes);
 
 /* Split-context decode attention over the packed cache, then the merge of
  * the splits with R^-1 applied once per output row (RotaryQuant, Abstract:
@@ -260,6 +284,22 @@ int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq,
                             int num_q_heads, const int32_t *seq_lens,
                             int page_size, const void *workspace,
                             size_t ws_bytes, float *out, void *stream);
+
+/* Debug export of the normalised rotated coordinates z that
+ * isoquant_compress_kv quantizes: z_j = sqrt(128) * (R x)_j / ||x||_2, the
+ * Walsh-Hadamard transform then the SO(4) blocks (RotaryQuant, Abstract),
+ * as the compress kernels compute it on their fp32 fast path, before any
+ * fp64 re-check (coordinates within 1e-5 of a decision threshold and norms
+ * near an fp16 rounding midpoint are redone in fp64 when compressing).
+ * Lets a test measure the fp32 error of z against an exact reference.  Not
+ * on the decode path.
+ *   x: device [n_tok][num_kv_heads][128] of dtype (F32, BF16, F16),
+ *      contiguous, 16-byte aligned;
+ *   z: device float [n_tok][num_kv_heads][128], 16-byte aligned,
+ *      caller-owned; a zero vector exports zeros.
+ * Errors: INVALID_ARG, UNSUPPORTED (dtype), ALIGNMENT, CUDA. */
+int isoquant_debug_export_z(isoquant_ctx *ctx, const void *x, int dtype,
+                            int n_tok, float *z, void *stream);
 
 /* Copy the device status word to *status and clear it (synchronises the
  * stream).  0 means no device-side error since the last call. */

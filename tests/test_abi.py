@@ -102,6 +102,8 @@ def test_every_entry_rejects_a_null_context(native):
                                   None, 0, None, None) == -1
     assert L.isoquant_get_status(None, ctypes.byref(st), None) == -1
     assert L.isoquant_selftest_wait(None, 1000, None, None) == -1
+    assert L.isoquant_debug_export_z(None, None, 1, 1, None, None) == -1
+    assert L.isoquant_workspace_size_paged(None, 1, 1, 8, 256, ctypes.byref(sz)) == -1
     assert L.isoquant_last_launch_count(None) == 0
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert native.strerror(code)

@@ -102,3 +102,83 @@ def test_argument_errors_with_a_live_context(cuda_lib):
     out_c, qc = out.cpu(), q.float().cpu()
     for b in range(st.B):
         check_pair(st, b, b % st.H, qc, out_c)
+
+
+def test_combine_with_another_plan_is_flagged(cuda_lib):
+    """The partial half writes the tag of its plan into the workspace
+    header.  A combine given another workspace size (so another kernel's
+    record layout) sees the mismatch: it merges nothing, writes zeros and
+    raises DEVERR_PLAN_MISMATCH; with matching sizes the halves agree with
+    the one-call entry."""
+    from compressed_space_decode_b200.synthetic import Workload
+    from compressed_space_decode_b200.workload import DecodeState
+    csd = cuda_lib
+    # 16 positions x 4 heads = 64 rows per KV head: the tcgen05 plan with the
+    # full workspace, the mma.sync plan with the minimum one
+    st = DecodeState(Workload("plan", 3, 16, 4, [700, 300, 65], nq=16, page_size=64, causal=True, seed=73))
+    q = st.queries(0)
+    q_rot = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    csd.isoquant_rotate_q(st.ctx, q.reshape(-1, st.Hq, D), q_rot.view(-1, st.Hq, D))
+    ws = _ws(csd, st)
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pairs = ((16 * st.G + 7) // 8) * st.B * st.H
+    small = (256 + (2 * n_sms + pairs) * 4160)
+    assert small < ws.numel() * 4
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    csd.isoquant_attend_partial(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, ws, causal=True)
+    # combine told the workspace is the small one: the mma.sync layout
+    csd.isoquant_attend_combine(st.ctx, st.B, 16, st.Hq, st.seq_lens_dev, st.ps, ws[:small // 4], out)
+    torch.cuda.synchronize()
+    assert csd.isoquant_get_status(st.ctx) == csd.DEVERR_PLAN_MISMATCH
+    assert torch.all(out == 0)
+    # matching sizes: no flag, and the same output as the one-call entry
+    csd.isoquant_attend_partial(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, ws, causal=True)
+    csd.isoquant_attend_combine(st.ctx, st.B, 16, st.Hq, st.seq_lens_dev, st.ps, ws, out)
+    ref = torch.empty_like(out)
+    csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, st.seq_lens_dev, _ws(csd, st), ref,
+                               causal=True)
+    torch.cuda.synchronize()
+    assert csd.isoquant_get_status(st.ctx) == 0
+    assert torch.equal(out, ref)
+
+
+def test_oversized_shapes_are_refused(cuda_lib):
+    """Shapes whose row or unit counts would overflow the kernels' 32-bit
+    indexing are refused on the host (INVALID_ARG), before any launch."""
+    import ctypes
+    from compressed_space_decode_b200 import synthetic
+    csd = cuda_lib
+    L = csd.lib()
+    signs, quats = synthetic.rotation_params(9, 8)
+    ctx = csd.isoquant_init(signs, quats)
+    sz = ctypes.c_size_t()
+    # 2^31 query rows per KV head (nq * G)
+    assert L.isoquant_workspace_size(ctx.handle, 1, 1 << 28, 64, ctypes.byref(sz)) == -1
+    # 2^28 row groups x 16 sequences x 8 KV heads
+    assert L.isoquant_workspace_size(ctx.handle, 16, 1 << 28, 64, ctypes.byref(sz)) == -1
+    # a modest shape still works
+    assert L.isoquant_workspace_size(ctx.handle, 16, 1, 64, ctypes.byref(sz)) == 0
+
+
+def test_workspace_sized_by_the_kernel_that_runs(cuda_lib):
+    """isoquant_workspace_size reports the records of the kernel the shape
+    runs on: the mma.sync records below 64 query rows per KV head, the
+    tcgen05 plan (16 or 8 records per CTA and per stream, plus the unit
+    prefix) from there, and the mma.sync records again for 32-token pages."""
+    from compressed_space_decode_b200 import synthetic
+    csd = cuda_lib
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rec = 4160
+    signs, quats = synthetic.rotation_params(10, 8)
+    ctx = csd.isoquant_init(signs, quats)
+    # decode, 16 sequences, 8 rows per KV head
+    assert csd.isoquant_workspace_size(ctx, 16, 1, 64) == 256 + (2 * n_sms + 16 * 8) * rec
+    # verification, 8 sequences, 16 positions x 4 heads = 64 rows: one 64-row stream
+    tiles = 256 + (2 * n_sms + 1 * 8 * 8) * 8 * rec + (1 * 8 + 1) * 8
+    assert csd.isoquant_workspace_size(ctx, 8, 16, 32) == tiles
+    # causal prefill of 4096 positions, 32 q heads: 128-row streams
+    streams = 4096 * 4 // 128
+    wide = 256 + (n_sms + streams * 8) * 16 * rec + (streams + 1) * 8
+    assert csd.isoquant_workspace_size(ctx, 1, 4096, 32) == wide
+    # 32-token pages: the mma.sync records whatever the rows
+    assert csd.isoquant_workspace_size_paged(ctx, 8, 16, 32, 32) == 256 + (2 * n_sms + 8 * 8 * 8) * rec

@@ -21,7 +21,7 @@ D = 128
 
 def _ws(csd, st):
     # NaN-filled so that reading a record nobody wrote shows up as NaN
-    return csd.alloc_workspace(st.ctx, st.B, st.wl.nq, st.Hq).fill_(0x7FC00000)
+    return csd.alloc_workspace(st.ctx, st.B, st.wl.nq, st.Hq, page_size=st.ps).fill_(0x7FC00000)
 
 
 def run_attend(csd, st, step=0, scale=0.0, q=None):

@@ -6,12 +6,17 @@ all device memory, or a decode loop that must avoid cudaMalloc's device-wide
 synchronisation).  Its split records live in a fixed array inside the
 library.  It must give the same output as isoquant_attend_decode, call
 after call: the array keeps the previous call's records, so a second call
-with different inputs checks that nothing stale leaks through.
+with different inputs checks that nothing stale leaks through.  Both entry
+points pick their kernel by the shape and the room for its records (the
+16 MiB array holds the tcgen05 plan of the verification shape here), so the
+two outputs are identical bit for bit, which also pins the kernel the static
+path chose; each workload is checked against the oracle as well.
 """
 import pytest
 import torch
 
 from tests.parity import ATTN_TOL, rowwise_rel_err
+from tests.test_gpu_parity import check_pair
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +48,11 @@ def test_static_entry_matches_workspace_entry_twice(cuda_lib):
             assert csd.isoquant_get_status(st.ctx) == 0
             err = rowwise_rel_err(got.cpu().numpy(), ref.cpu().numpy())
             assert err.max() <= ATTN_TOL, (name, step, err.max())
+            # same kernel and plan as the workspace entry: identical output
+            assert torch.equal(got, ref), (name, step)
+        # the last call's output against the oracle on one sampled pair
+        q = st.queries(steps[-1]).float().cpu()
+        check_pair(st, st.B - 1, st.H - 1, q, got.cpu())
 
 
 def test_static_entry_rejects_oversized_shapes(cuda_lib):
