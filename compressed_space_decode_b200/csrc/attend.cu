@@ -82,12 +82,20 @@ struct DecLayout {
   static constexpr int kBarriers = kQScale + 8 * 4;
   // abort flag (+0), CTA range and walk start (+8..+47)
   static constexpr int kLocate = kBarriers + 2 * kStages * 8;
-  static constexpr int kSmemBytes = kLocate + 64;
+  // Pair table, entry i = half2(C[i mod 2^BITS], C[i >> BITS]), one copy
+  // per lane (entry i of lane l at byte 128 i + 4 l: 32 lanes with 32
+  // different entries hit 32 different banks).  At 2 and 3 bits it sits in
+  // this dynamic area at an address aligned to its span (2 KB, 8 KB), so an
+  // entry's shared address is one AND-OR of the code bits with
+  // (table base | 4 lane): no add per lookup.  The 4-bit table (32 KB) stays
+  // a static array addressed from its base.
+  static constexpr bool kAbsLut = BITS != 4;
+  static constexpr int kLutSpan = (1 << (2 * BITS)) * 128;
+  static constexpr int kLutArea = kLocate + 64;
+  static constexpr int kSmemBytes = kAbsLut ? kLutArea + 2 * kLutSpan : kLocate + 64;
   // bytes a page's copies bring per token: K and V words, K and V norms
   static constexpr int kTxPerToken = 8 * W + 4;
-  // pair table of the 2- and 4-bit kernels (the 3-bit one uses s_lut):
-  // entry i = half2(C[i mod 2^BITS], C[i >> BITS]), one copy per lane
-  static constexpr int kLutWords = BITS == 3 ? 4 : (1 << (2 * BITS)) * 32;
+  static constexpr int kLutWords = kAbsLut ? 4 : (1 << (2 * BITS)) * 32;
   static_assert(kScratchE + 8 * 4 <= kStageBytes, "merge scratch must fit in one stage");
   static_assert(kStageBytes % 16 == 0, "stage alignment");
 };
@@ -425,13 +433,20 @@ __device__ __forceinline__ uint32_t lut_off(uint32_t x, uint32_t lane4) {
 __device__ __forceinline__ uint32_t lut_at(uint32_t off) {
   return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const char *>(s_lut) + off);
 }
+// A table entry at a shared-window address (the decode kernel's aligned table).
+__device__ __forceinline__ uint32_t plut(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
 // five adjacent-code pairs (2k, 2k+1), k = 0..4, of a packed word
+// (lane4: the aligned table's base | 4 lane)
 __device__ __forceinline__ void word_pairs(uint32_t w, uint32_t lane4, uint32_t *out) {
-  out[0] = lut_at(lut_off<-7>(w, lane4));
-  out[1] = lut_at(lut_off<-1>(w, lane4));
-  out[2] = lut_at(lut_off<5>(w, lane4));
-  out[3] = lut_at(lut_off<11>(w, lane4));
-  out[4] = lut_at(lut_off<17>(w, lane4));
+  out[0] = plut(lut_off<-7>(w, lane4));
+  out[1] = plut(lut_off<-1>(w, lane4));
+  out[2] = plut(lut_off<5>(w, lane4));
+  out[3] = plut(lut_off<11>(w, lane4));
+  out[4] = plut(lut_off<17>(w, lane4));
 }
 
 // The tcgen05 kernels' decode tables, one copy per lane: BITS = 3: entry i =
@@ -485,9 +500,9 @@ __device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
 template <int K>
 __device__ __forceinline__ uint32_t k_pair_c(const uint4 (&kw)[4], int j, uint32_t sh12, uint32_t lane4) {
   if constexpr (K < 15) {
-    return lut_at(lut_off<6 * (K % 5) - 7>(u4_at(kw[K / 5], j), lane4));
+    return plut(lut_off<6 * (K % 5) - 7>(u4_at(kw[K / 5], j), lane4));
   } else {
-    return lut_at((((u4_at(kw[3], j) << 7) >> sh12) & 0x1F80u) | lane4);
+    return plut((((u4_at(kw[3], j) << 7) >> sh12) & 0x1F80u) | lane4);
   }
 }
 // 2 and 4 bits: pair k (0..15) is pair k mod P (P = pairs per word) of word
@@ -497,19 +512,23 @@ template <int SH, uint32_t MASK>
 __device__ __forceinline__ uint32_t lut_off_m(uint32_t x, uint32_t lane4) {
   return (shifted<SH>(x) & MASK) | lane4;
 }
+// 2 bits: off is a shared-window address (aligned table | 4 lane); 4 bits: a
+// byte offset into the static table `lut`
+template <int BITS>
 __device__ __forceinline__ uint32_t lut_at2(const char *lut, uint32_t off) {
-  return *reinterpret_cast<const uint32_t *>(lut + off);
+  if constexpr (BITS == 4) return *reinterpret_cast<const uint32_t *>(lut + off);
+  else return plut(off);
 }
 template <int BITS, int K>
 __device__ __forceinline__ uint32_t k_pair_w(const uint4 (&kw)[4], int j, uint32_t lane4, const char *lut) {
   constexpr int kPpw = 16 / BITS;
   constexpr uint32_t kMask = ((1u << (2 * BITS)) - 1u) << 7;
-  return lut_at2(lut, lut_off_m<2 * BITS * (K % kPpw) - 7, kMask>(u4_at(kw[K / kPpw], j), lane4));
+  return lut_at2<BITS>(lut, lut_off_m<2 * BITS * (K % kPpw) - 7, kMask>(u4_at(kw[K / kPpw], j), lane4));
 }
 // Slot K of a merged word, looked up
 template <int BITS, uint32_t MASK, int K>
 __device__ __forceinline__ uint32_t merged_pair(uint32_t e, uint32_t lane4, const char *lut) {
-  return lut_at2(lut, lut_off_m<2 * BITS * K - 7, MASK>(e, lane4));
+  return lut_at2<BITS>(lut, lut_off_m<2 * BITS * K - 7, MASK>(e, lane4));
 }
 // The kPpw 2*BITS-bit slots of a merged word, looked up in order
 template <int BITS>
@@ -713,11 +732,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
   int64_t *loc = reinterpret_cast<int64_t *>(smem + L::kLocate + 8);
   const int ps = p.page_size;
 
-  if constexpr (BITS == 3) {
-    for (int e = tid; e < 64 * 32; e += kThreads) {
+  uint32_t lut_lane = static_cast<uint32_t>(lane) * 4u;  // table base | 4 lane (4 bits: 4 lane)
+  if constexpr (L::kAbsLut) {
+    const uint32_t base = (smem_addr(smem + L::kLutArea) + L::kLutSpan - 1) & ~static_cast<uint32_t>(L::kLutSpan - 1);
+    for (int e = tid; e < L::kLutSpan / 4; e += kThreads) {
       const int idx = e >> 5;
-      s_lut[e] = pack_half2(p.level[idx & 7], p.level[idx >> 3]);
+      const uint32_t v = pack_half2(p.level[idx & ((1 << BITS) - 1)], p.level[idx >> BITS]);
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(base + 4u * e), "r"(v) : "memory");
     }
+    lut_lane |= base;
   } else {
     for (int e = tid; e < L::kLutWords; e += kThreads) {
       const int idx = e >> 5;
@@ -819,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
   }
 
   // -------------------------------------------------------------- consumers
-  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+  const uint32_t lane4 = lut_lane;
 
   // dims this thread feeds to Q.K^T: pair k (k = 0..15) = coordinates
   // (kdim(k), kdim(k) + 1); pairs 0..14 come from words 3tq..3tq+2, pair 15
@@ -1062,7 +1085,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
               word_pairs(e_odd, lane4, va[half] + 5);
               word_pairs(e_half, lane4, va[half] + 10);
               const uint32_t z12 = (((wz >> (3 * gid)) & 7u) << 7) | (((wz1 >> (3 * gid)) & 7u) << 10);
-              va[half][15] = lut_at(z12 | lane4);
+              va[half][15] = plut(z12 | lane4);
             }
             const uint32_t b0 = pack_half2(pv[8 * h + 4 * kap + 0], pv[8 * h + 4 * kap + 1]);
             const uint32_t b1 = pack_half2(pv[8 * h + 4 * kap + 2], pv[8 * h + 4 * kap + 3]);
