@@ -168,7 +168,10 @@ def run_ours(args):
 
     wl = multi.shard_workload(synthetic.workloads()[args.workload], rank, world)
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    growth = args.warmup + args.steps + e2e_steps + 2
+    # tokens each step appends per sequence: one for decode; a causal chunk
+    # of nq query positions (verification) appends its nq tokens
+    adv = wl.nq if wl.causal else 1
+    growth = (args.warmup + args.steps + e2e_steps + 2) * adv
     st = DecodeState(wl, growth=growth, device=dev, bits=args.bits)
     bytes_per_token_head = 2 * (csd.WORDS_FOR[args.bits] * 4 + 2)
     B, H, Hq, nq = st.B, st.H, st.Hq, wl.nq
@@ -177,15 +180,20 @@ def run_ours(args):
     # per-step inputs, generated up front (device-resident for the kernel metric)
     n_total = args.warmup + args.steps
     lens0 = list(st.seq_lens)
-    k_all = torch.empty((n_total, B, H, 128), dtype=torch.bfloat16, device=dev)
+    # step s appends tokens lens0[b] + s adv + a (a < adv) of every sequence b,
+    # ordered (a, b) like their slots
+    k_all = torch.empty((n_total, adv, B, H, 128), dtype=torch.bfloat16, device=dev)
     v_all = torch.empty_like(k_all)
     for b in range(B):
-        k, v = st.kv_tokens(b, lens0[b], lens0[b] + n_total)
-        k_all[:, b] = k
-        v_all[:, b] = v
+        k, v = st.kv_tokens(b, lens0[b], lens0[b] + n_total * adv)
+        k_all[:, :, b] = k.view(n_total, adv, H, 128)
+        v_all[:, :, b] = v.view(n_total, adv, H, 128)
+    k_all = k_all.view(n_total, adv * B, H, 128)
+    v_all = v_all.view(n_total, adv * B, H, 128)
     q_all = synthetic.gaussian(wl.seed, 20_000_000, (n_total, B * nq, Hq, 128), device=dev, dtype=torch.bfloat16)
-    slots_all = st.slot_matrix(lens0, n_total)
-    lens_all = torch.tensor([[L + s + 1 for L in lens0] for s in range(n_total)], dtype=torch.int32, device=dev)
+    slots_all = st.slot_matrix(lens0, n_total * adv).view(n_total, adv * B)
+    lens_all = torch.tensor([[L + (s + 1) * adv for L in lens0] for s in range(n_total)], dtype=torch.int32,
+                            device=dev)
     q_rot = torch.empty((B, nq, Hq, 128), dtype=torch.float32, device=dev)
     out = torch.empty_like(q_rot)
     ws = csd.alloc_workspace(st.ctx, B, nq, Hq, device=dev)
@@ -276,8 +284,8 @@ def run_ours(args):
 
     # end to end through the public API from pinned host buffers
     attn_events = None
-    st.seq_lens = [L + n_total for L in lens0]
-    base = n_total
+    st.seq_lens = [L + n_total * adv for L in lens0]
+    base = n_total * adv
     # a step's inputs (k | v | q | slots | lens) sit in one pinned staging row
     # and cross to the device in one transfer, as a serving loop would stage them
     kd, vd = torch.empty_like(k_all[0]), torch.empty_like(v_all[0])
@@ -287,14 +295,14 @@ def run_ours(args):
     kd, vd, qd, sd, ld = (stage_d[o:o + n].view(dt).view(shp) for o, n, dt, shp in layout)
     stage_h = torch.zeros((e2e_steps, row_bytes), dtype=torch.uint8).pin_memory()
     host_views = [[stage_h[s, o:o + n].view(dt).view(shp) for o, n, dt, shp in layout] for s in range(e2e_steps)]
-    lens_e2e = [[L + base + s + 1 for L in lens0] for s in range(e2e_steps)]
+    lens_e2e = [[L + base + (s + 1) * adv for L in lens0] for s in range(e2e_steps)]
     for b in range(B):
-        k, v = st.kv_tokens(b, lens0[b] + base, lens0[b] + base + e2e_steps)
-        k, v = k.cpu(), v.cpu()
+        k, v = st.kv_tokens(b, lens0[b] + base, lens0[b] + base + e2e_steps * adv)
+        k, v = k.cpu().view(e2e_steps, adv, H, 128), v.cpu().view(e2e_steps, adv, H, 128)
         for s in range(e2e_steps):
-            host_views[s][0][b] = k[s]
-            host_views[s][1][b] = v[s]
-    slots_h = st.slot_matrix([L + base for L in lens0], e2e_steps).cpu()
+            host_views[s][0].view(adv, B, H, 128)[:, b] = k[s]
+            host_views[s][1].view(adv, B, H, 128)[:, b] = v[s]
+    slots_h = st.slot_matrix([L + base for L in lens0], e2e_steps * adv).view(e2e_steps, adv * B).cpu()
     for s in range(e2e_steps):
         host_views[s][2].copy_(q_all[s].cpu())
         host_views[s][3].copy_(slots_h[s])
@@ -347,7 +355,7 @@ def run_ours(args):
         "data": "synthetic (seeded bf16 Student-t(4) K/V, log-uniform channel scales, x20 outliers)",
         "config": {"workload": wl.name.split("@")[0], "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
                    "context_start": lens0[0], "page_size": st.ps, "page_table": "shuffled",
-                   "step": "decode_prep (append 1 token/seq + rotate q, one launch) + attend_decode (split-K attention + combine); programmatic launches",
+                   "step": f"decode_prep (append {adv} token(s)/seq + rotate q, one launch) + attend_decode (split-K attention + combine); programmatic launches",
                    "l2": f"packed cache {bytes_per_launch / 1e6:.0f} MB > 126 MB L2; no flush",
                    "parallelism": f"dp{world} (independent shards)", "code_bits": args.bits,
                    "bytes_per_kv_token_head": bytes_per_token_head},
