@@ -191,7 +191,7 @@ def run_ours(args):
     k_all = k_all.view(n_total, adv * B, H, 128)
     v_all = v_all.view(n_total, adv * B, H, 128)
     q_all = synthetic.gaussian(wl.seed, 20_000_000, (n_total, B * nq, Hq, 128), device=dev, dtype=torch.bfloat16)
-    slots_all = st.slot_matrix(lens0, n_total * adv).view(n_total, adv * B)
+    slots_all = st.slot_matrix(lens0, n_total * adv).reshape(n_total, adv * B)
     lens_all = torch.tensor([[L + (s + 1) * adv for L in lens0] for s in range(n_total)], dtype=torch.int32,
                             device=dev)
     q_rot = torch.empty((B, nq, Hq, 128), dtype=torch.float32, device=dev)
@@ -302,7 +302,7 @@ def run_ours(args):
         for s in range(e2e_steps):
             host_views[s][0].view(adv, B, H, 128)[:, b] = k[s]
             host_views[s][1].view(adv, B, H, 128)[:, b] = v[s]
-    slots_h = st.slot_matrix([L + base for L in lens0], e2e_steps * adv).view(e2e_steps, adv * B).cpu()
+    slots_h = st.slot_matrix([L + base for L in lens0], e2e_steps * adv).reshape(e2e_steps, adv * B).cpu()
     for s in range(e2e_steps):
         host_views[s][2].copy_(q_all[s].cpu())
         host_views[s][3].copy_(slots_h[s])
@@ -385,31 +385,38 @@ def run_ours(args):
     print(json.dumps(line))
 
 
-def oracle_sample(wl, b, h, bits=3):
+def oracle_sample(wl, b, h, bits=3, device="cuda"):
     """Oracle state for one (sequence, KV head) of workload `wl`: its own
-    codes of the context, the appended token and the step's query rows, and
-    how many context coordinates lie within 1e-6 of a decision threshold.
-    Inputs come from the seeded generators only."""
+    codes of the context, the tokens a step appends (one, or the nq of a
+    causal chunk) and the step's query rows (every position of the chunk,
+    each seeing the tokens up to its own), and how many context coordinates
+    lie within 1e-6 of a decision threshold.  Inputs come from the seeded
+    generators only."""
     import oracle
     from compressed_space_decode_b200 import synthetic
     L = wl.seq_lens[b]
     G = wl.group
-    k, v = synthetic.workload_kv_tokens(wl, b, 0, L + 1, device="cuda")
+    adv = wl.nq if wl.causal else 1
+    k, v = synthetic.workload_kv_tokens(wl, b, 0, L + adv, device=device)
     signs, quats = synthetic.rotation_params(wl.seed, wl.kv_heads)
     s, qt = signs[h].numpy(), quats[h].numpy()
     kc, kn, zk, _ = oracle.compress(s, qt, k[:L, h].double().cpu().numpy(), want_z=True, bits=bits)
     vc, vn, zv, _ = oracle.compress(s, qt, v[:L, h].double().cpu().numpy(), want_z=True, bits=bits)
     near = [int(oracle.near_boundary(z, 1e-6, bits=bits).sum()) for z in (zk, zv)]
-    newk = k[L:L + 1, h].double().cpu().numpy()
-    newv = v[L:L + 1, h].double().cpu().numpy()
-    q = synthetic.workload_queries(wl, 0, device="cuda")[b, 0, h * G:(h + 1) * G].double().cpu().numpy()
+    newk = k[L:L + adv, h].double().cpu().numpy()
+    newv = v[L:L + adv, h].double().cpu().numpy()
+    nq = adv
+    q = synthetic.workload_queries(wl, 0, device=device)[b, :nq, h * G:(h + 1) * G]
+    q = q.reshape(nq * G, 128).double().cpu().numpy()  # rows (position, head)
+    lims = [L + i + 1 for i in range(nq) for _ in range(G)]
     return dict(s=s, qt=qt, kc=kc, kn=kn, vc=vc, vn=vn, newk=newk, newv=newv, q=q, L=L, G=G, bits=bits, b=b, h=h,
-                near=near)
+                near=near, adv=adv, nq=nq, lims=lims, causal=bool(wl.causal))
 
 
 def oracle_step(o):
-    """One decode step of the oracle for one (sequence, KV head): compress
-    the appended K/V token, then attend over L+1 tokens."""
+    """One step of the oracle for one (sequence, KV head): compress the
+    appended K/V tokens, then attend (position i of the step's chunk over the
+    first L + i + 1 tokens)."""
     import numpy as np
 
     import oracle
@@ -419,8 +426,7 @@ def oracle_step(o):
     kn = np.concatenate([o["kn"], kn1])
     vc = np.concatenate([o["vc"], vc1])
     vn = np.concatenate([o["vn"], vn1])
-    R = o["q"].shape[0]
-    return oracle.attend(o["s"], o["qt"], o["q"], kc, kn, vc, vn, [o["L"] + 1] * R, bits=o["bits"])
+    return oracle.attend(o["s"], o["qt"], o["q"], kc, kn, vc, vn, o["lims"], bits=o["bits"])
 
 
 def host_cores():
@@ -492,15 +498,17 @@ def parity_sample(st, o, dev):
     res["code_mismatches"] = mism_codes
     res["norm_mismatches"] = mism_norms
     wl = st.wl
-    q = synthetic.workload_queries(wl, 0, device=dev)[b:b + 1].contiguous()
+    nq = o["nq"]
+    q = synthetic.workload_queries(wl, 0, device=dev)[b:b + 1, :nq].contiguous()
     q_rot = torch.empty(q.shape, dtype=torch.float32, device=dev)
     csd.isoquant_rotate_q(st.ctx, q.view(-1, st.Hq, 128), q_rot.view(-1, st.Hq, 128))
     out = torch.empty_like(q_rot)
-    lens = torch.tensor([L + 1], dtype=torch.int32, device=dev)
-    ws = csd.alloc_workspace(st.ctx, 1, 1, st.Hq, device=dev)
-    csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table[b:b + 1].contiguous(), lens, ws, out)
+    lens = torch.tensor([L + o["adv"]], dtype=torch.int32, device=dev)
+    ws = csd.alloc_workspace(st.ctx, 1, nq, st.Hq, page_size=st.ps, device=dev)
+    csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table[b:b + 1].contiguous(), lens, ws, out,
+                               causal=o["causal"])
     torch.cuda.synchronize(dev)
-    got = out[0, 0, h * G:(h + 1) * G].double().cpu().numpy()
+    got = out[0, :, h * G:(h + 1) * G].reshape(nq * G, 128).double().cpu().numpy()
     ref = oracle_step(o)
     err = np.abs(got - ref).max(axis=1) / np.abs(ref).max(axis=1)
     res["max_row_rel_err"] = float(err.max())
@@ -517,19 +525,19 @@ def cpu_baseline(wl, budget_s=12.0, bits=3, st=None, dev=None):
     units, t0 = 0, time.perf_counter()
     while time.perf_counter() - t0 < budget_s:
         oracle_step(o)
-        units += o["L"] + 1
+        units += o["L"] + o["adv"]
     dt = time.perf_counter() - t0
     one = {"value": units / dt, "unit": UNIT, "cores": 1,
-           "sample": f"{units // (o['L'] + 1)} steps in {dt:.1f} s"}
+           "sample": f"{units // (o['L'] + o['adv'])} steps in {dt:.1f} s"}
     cores = host_cores()
     pool = OraclePool(o, cores)
     pool.run(steps=1)  # start-up, untimed
     n, dt_all = pool.run(budget_s=budget_s)
     pool.close()
-    line = {"value": n * (o["L"] + 1) / dt_all, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"sequence 0, KV head 0 of the workload (context {o['L'] + 1}, {o['G']} query rows): "
-                      f"compress the appended token + attend; {cores} host processes ran {n} steps in "
-                      f"{dt_all:.1f} s",
+    line = {"value": n * (o["L"] + o["adv"]) / dt_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"sequence 0, KV head 0 of the workload (context {o['L'] + o['adv']}, {len(o['lims'])} "
+                      f"query rows): compress the {o['adv']} appended token(s) + attend; {cores} host processes "
+                      f"ran {n} steps in {dt_all:.1f} s",
             "single_core": one}
     if st is not None:
         line["parity_sample"] = parity_sample(st, o, dev)
@@ -576,10 +584,11 @@ def run_reference(args):
     # each step: every host process runs one oracle decode step
     _, dt = pool.run(steps=args.steps)  # the slowest process's own time
     pool.close()
-    units = args.steps * cores * (o["L"] + 1)
+    units = args.steps * cores * (o["L"] + o["adv"])
     value = units / dt
     sample = (f"each step: {cores} host processes each run sequence 0, KV head 0 of {wl.name} (context "
-              f"{o['L'] + 1}, {o['G']} query rows): compress the appended token + attend")
+              f"{o['L'] + o['adv']}, {len(o['lims'])} query rows): compress the {o['adv']} appended token(s) "
+              f"+ attend")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",

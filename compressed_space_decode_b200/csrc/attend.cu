@@ -953,9 +953,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
           if (wk.j * ps + tin >= lim || tin >= ps) x[i] = -INFINITY;
         }
       }
-      float mx = x[0];
+      // row maximum as a tree (depth 4, not a 15-long chain)
+      float mt[8];
 #pragma unroll
-      for (int i = 1; i < 16; ++i) mx = fmaxf(mx, x[i]);
+      for (int i = 0; i < 8; ++i) mt[i] = fmaxf(x[i], x[i + 8]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mt[i] = fmaxf(mt[i], mt[i + 4]);
+      float mx = fmaxf(fmaxf(mt[0], mt[2]), fmaxf(mt[1], mt[3]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float m_new = fmaxf(m_run, mx);
@@ -971,12 +975,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
         m_run = m_new;
       }
       const float mm = (m_run == -INFINITY) ? 0.f : m_run * inv2e;
-      float pv[16], psum[2] = {0.f, 0.f};
+      float pv[16], psum[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains
       if (!tail) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float pr = ex2(fmaf(x[i], inv2e, -mm));
-          psum[i & 1] += pr;
+          psum[i & 3] += pr;
           pv[i] = pr * nv[i];
         }
       } else {
@@ -984,11 +988,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_attend_partial(const P
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float pr = ex2(fmaf(x[i], inv2e, -mm));
-          psum[i & 1] += pr;
+          psum[i & 3] += pr;
           pv[i] = pr > 0.f ? pr * nv[i] : 0.f;
         }
       }
-      l_run += psum[0] + psum[1];
+      l_run += (psum[0] + psum[1]) + (psum[2] + psum[3]);
 
       // ---- P.V: O^T[16 dims x 8 rows] += V^T[16 dims x 16 tok] P^T
       if constexpr (BITS == 3) {

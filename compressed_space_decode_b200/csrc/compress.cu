@@ -94,6 +94,55 @@ struct CompressArgs {
 // per-vector work (norm rounding, packing) is shared by 8 lanes instead of
 // 32.
 
+// A lane's 16 inputs as loaded (the raw 16-bit words, or fp32 values), so
+// that the next vector's loads can be issued before the current one is done.
+template <typename T>
+struct Raw16 {
+  uint4 w[2];
+};
+template <>
+struct Raw16<float> {
+  float4 w[4];
+};
+__device__ __forceinline__ void load16_raw(const float *p, Raw16<float> &r) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r.w[i] = reinterpret_cast<const float4 *>(p)[i];
+}
+template <typename T>
+__device__ __forceinline__ void load16_raw(const T *p, Raw16<T> &r) {
+  r.w[0] = reinterpret_cast<const uint4 *>(p)[0];
+  r.w[1] = reinterpret_cast<const uint4 *>(p)[1];
+}
+__device__ __forceinline__ void unpack16(const Raw16<float> &r, float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[4 * i] = r.w[i].x; x[4 * i + 1] = r.w[i].y; x[4 * i + 2] = r.w[i].z; x[4 * i + 3] = r.w[i].w;
+  }
+}
+__device__ __forceinline__ void unpack16(const Raw16<__nv_bfloat16> &r, float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t w[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+      x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  }
+}
+__device__ __forceinline__ void unpack16(const Raw16<__half> &r, float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t w[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
+      x[8 * i + 2 * k] = f.x;
+      x[8 * i + 2 * k + 1] = f.y;
+    }
+  }
+}
+
 __device__ __forceinline__ void load16(const float *p, float (&x)[16]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -321,17 +370,29 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
 
   const int t_begin = static_cast<int>(sidx) * g.strip;
   const int t_end = min(t_begin + g.strip, n_tok);
+  // the inputs and slot of the group's next vector are loaded one iteration
+  // ahead, so that their latency overlaps the current vector's rotation
+  Raw16<T> nraw{};
+  int64_t nslot = -1;
+  if (t_begin + grp < t_end) {
+    nslot = g.slots[t_begin + grp];
+    load16_raw(src + (static_cast<int64_t>(t_begin + grp) * H + h) * kD + 16 * q, nraw);
+  }
   for (int tb = t_begin; tb < t_end; tb += 4) {
     const int t = tb + grp;
     const bool live = t < t_end;
     float x[16];
     int64_t slot = -1;
     if (live) {
-      slot = g.slots[t];
-      load16(src + (static_cast<int64_t>(t) * H + h) * kD + 16 * q, x);
+      slot = nslot;
+      unpack16(nraw, x);
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i) x[i] = 0.f;
+    }
+    if (t + 4 < t_end) {
+      nslot = g.slots[t + 4];
+      load16_raw(src + (static_cast<int64_t>(t + 4) * H + h) * kD + 16 * q, nraw);
     }
     const int64_t page = slot >> ps_shift;
     const bool valid = live && slot >= 0 && page < g.num_pages;
@@ -364,17 +425,19 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
       for (int r = 0; r < 4; ++r) {
         const float z = fast_z(mrow, x, k, r, inv);
         const float a = fabsf(z);
-        uint32_t gt = 0, ge = 0;
-        bool nr = a < kRecheckBand;
+        // strict comparisons only: |z| equal to a threshold (or z = 0) is
+        // within the re-check band, so the fp64 path decides it and the tie
+        // rule of the fast path does not matter
+        uint32_t gt = 0;
+        float dm = a;  // distance to the nearest threshold (0 included)
 #pragma unroll
         for (int i = 0; i < kHalf - 1; ++i) {
           gt += a > tp[i] ? 1u : 0u;
-          ge += a >= tp[i] ? 1u : 0u;
-          nr |= fabsf(a - tp[i]) < kRecheckBand;
+          dm = fminf(dm, fabsf(a - tp[i]));
         }
-        const uint32_t c = z > 0.f ? kHalf + gt : kHalf - 1 - ge;
+        const uint32_t c = z > 0.f ? kHalf + gt : kHalf - 1 - gt;
         cbits |= static_cast<uint64_t>(c) << (BITS * (4 * k + r));
-        near |= nr;
+        near |= dm < kRecheckBand;
       }
     }
     // the group's verdict: any lane near a threshold sends the vector to
@@ -415,9 +478,16 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
   }
 }
 
-// warps per compress block; blockIdx.y selects K or V
+// warps per compress block; blockIdx.y selects K or V.  Four-warp blocks,
+// three per SM (bulk compression of 32768 x 8 vectors per layer: 0.218 ms
+// per layer against 0.261 ms with eight-warp blocks, two per SM).
+#ifndef ISOQUANT_COMPRESS_WARPS
+#define ISOQUANT_COMPRESS_WARPS 4
+#endif
+constexpr int kCompressWarps = ISOQUANT_COMPRESS_WARPS;  // warps per k_compress block
+constexpr int kCompressBlocksPerSm = kCompressWarps == 8 ? 2 : 3;
 template <typename T, int BITS>
-__global__ void __launch_bounds__(256, 2) k_compress(const CompressArgs g) {
+__global__ void __launch_bounds__(kCompressWarps * 32, kCompressBlocksPerSm) k_compress(const CompressArgs g) {
   pdl_trigger();
   pdl_wait();
   compress_warp<T, BITS>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), threadIdx.x & 31);
@@ -541,10 +611,10 @@ CompressArgs compress_args(const isoquant_ctx *ctx, const isoquant_cache *cache,
 }
 
 // compress blocks per K/V half (8 warps each, one strip per warp)
-int64_t compress_blocks(const isoquant_ctx *ctx, int n_tok) {
+int64_t compress_blocks(const isoquant_ctx *ctx, int n_tok, int warps_per_block) {
   const int strip = strip_tokens(n_tok);
   const int64_t warps = static_cast<int64_t>((n_tok + strip - 1) / strip) * ctx->num_kv_heads;
-  return (warps + 7) / 8;
+  return (warps + warps_per_block - 1) / warps_per_block;
 }
 
 RotateArgs rotate_args(const isoquant_ctx *ctx, const void *q, int n_rows, int num_q_heads, float *q_rot) {
@@ -587,11 +657,11 @@ cudaError_t launch_prep_t(int dtype, dim3 grid, dim3 block, cudaStream_t stream,
 cudaError_t launch_compress(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k,
                             const void *v, int dtype, int n_tok, const int64_t *slot_mapping,
                             cudaStream_t stream) {
-  const int64_t blocks = compress_blocks(ctx, n_tok);
+  const int64_t blocks = compress_blocks(ctx, n_tok, kCompressWarps);
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
   const CompressArgs g = compress_args(ctx, cache, k, v, n_tok, slot_mapping);
-  const dim3 grid(static_cast<unsigned>(blocks), 2), block(256);
+  const dim3 grid(static_cast<unsigned>(blocks), 2), block(kCompressWarps * 32);
   switch (ctx->codebook.bits) {
     case 2: return launch_compress_t<2>(dtype, grid, block, stream, g);
     case 4: return launch_compress_t<4>(dtype, grid, block, stream, g);
@@ -636,7 +706,7 @@ cudaError_t launch_export_z(const isoquant_ctx *ctx, const void *x, int dtype, i
 cudaError_t launch_decode_prep(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v,
                                int n_tok, const int64_t *slot_mapping, const void *q, int dtype, int n_rows,
                                int num_q_heads, float *q_rot, cudaStream_t stream) {
-  const int64_t nbc = compress_blocks(ctx, n_tok);
+  const int64_t nbc = compress_blocks(ctx, n_tok, 8);
   const int64_t nbr = rotate_blocks(n_rows, num_q_heads);
   const int64_t blocks = 2 * nbc + nbr;
   if (blocks == 0) return cudaSuccess;

@@ -46,3 +46,24 @@ def test_stage_layout_views_round_trip():
     copy = stage.clone()
     for (o, n, dt, shp), t in zip(layout, ts):
         assert torch.equal(copy[o:o + n].view(dt).view(shp), t)
+
+
+@pytest.mark.parametrize("causal,nq", [(False, 1), (True, 5)])
+def test_oracle_step_rows_see_their_prefix(causal, nq):
+    """The CPU-baseline sample of a step: with a causal chunk of nq appended
+    tokens, position i's rows attend over the first L + i + 1 tokens, so each
+    row equals the oracle's attention over that prefix alone."""
+    import numpy as np
+    import oracle
+    wl = Workload("t", 2, 4, 2, [70, 45], nq=nq, page_size=64, causal=causal, seed=5)
+    o = bench.oracle_sample(wl, 1, 1, device="cpu")
+    assert o["adv"] == (nq if causal else 1) and o["q"].shape == (nq * wl.group, 128)
+    out = bench.oracle_step(o)
+    kc1, kn1, _, _ = oracle.compress(o["s"], o["qt"], o["newk"])
+    vc1, vn1, _, _ = oracle.compress(o["s"], o["qt"], o["newv"])
+    kc, kn = np.concatenate([o["kc"], kc1]), np.concatenate([o["kn"], kn1])
+    vc, vn = np.concatenate([o["vc"], vc1]), np.concatenate([o["vn"], vn1])
+    for r in range(out.shape[0]):
+        n = 45 + r // wl.group + 1
+        ref = oracle.attend(o["s"], o["qt"], o["q"][r:r + 1], kc[:n], kn[:n], vc[:n], vn[:n], [n])
+        assert np.allclose(out[r], ref[0], rtol=0, atol=1e-12 * np.abs(ref).max())
