@@ -2,10 +2,10 @@
 //
 // RotaryQuant, Abstract: a Walsh-Hadamard transform followed by
 // block-diagonal SO(4) rotations isotropizes each head vector before 3-bit
-// scalar quantization.  A warp rotates one d = 128 vector at a time, lane l
-// holding coordinates 4l..4l+3: the two smallest WHT strides stay inside the
-// lane, the other five are warp shuffles, and SO(4) block l is lane l's own
-// 4x4 product, so the whole rotation stays in registers.
+// scalar quantization.  The compress kernels give each vector 8 lanes in two
+// layouts (below); the query rotation and the fp64 path give it a warp, lane
+// l holding coordinates 4l..4l+3 (two WHT strides inside the lane, five warp
+// shuffles, SO(4) block l as the lane's own 4x4 product).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -85,119 +85,168 @@ struct CompressArgs {
   uint32_t *status;
 };
 
-// ------------------------------------------------------------ wide layout
+// ------------------------------------------------------------ two layouts
 // A warp compresses four vectors of one head at a time: lane group
-// g = lane / 8 holds one vector, its lane q = lane % 8 holding coordinates
-// 16q..16q+15.  Four WHT strides (1..8) stay inside the lane and three
-// (16, 32, 64) cross lanes of the group, the lane's four SO(4) blocks
-// 4q..4q+3 stay in registers for the warp's whole strip of tokens, and the
-// per-vector work (norm rounding, packing) is shared by 8 lanes instead of
-// 32.
+// g = lane / 8 holds one vector and its lane q = lane % 8 a sixteenth of it,
+// in one of two layouts:
+//   layout A (loads, signs, norm, WHT strides 16, 32 and 64): coordinates
+//     16m + 2q and 16m + 2q + 1 for m = 0..7, as a[m] = (the two);
+//   layout B (WHT strides 1, 2, 4 and 8, the SO(4) blocks, the codes):
+//     coordinates 16q .. 16q + 15, as b[k] = (16q + 2k, 16q + 2k + 1).
+// Each layout keeps its WHT strides inside the lane, so the transform needs
+// no shuffles: the change of layout goes through a shared-memory tile per
+// warp, and the lane's four SO(4) blocks 4q .. 4q + 3 stay in registers for
+// the warp's whole strip of tokens.  Pairs of coordinates go through the
+// packed fp32 instructions (two independent IEEE operations each).
 
-// A lane's 16 inputs as loaded (the raw 16-bit words, or fp32 values), so
-// that the next vector's loads can be issued before the current one is done.
+// Shared tile of one warp: per vector 8 rows (m) of 16 floats, rows 20
+// floats apart and vectors 176 apart, so that neither the 8-byte stores of
+// layout A nor the 16-byte loads of layout B meet a bank conflict.
+constexpr int kTileRow = 20;
+constexpr int kTileVec = 8 * kTileRow + 16;
+constexpr int kTileFloats = 4 * kTileVec;
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
+
+// One layout-A lane's 16 inputs as loaded: a 32-bit word per pair of 16-bit
+// values, or the fp32 pair.
 template <typename T>
-struct Raw16 {
-  uint4 w[2];
+struct RawA {
+  uint32_t w[8];
 };
 template <>
-struct Raw16<float> {
-  float4 w[4];
+struct RawA<float> {
+  float2 w[8];
 };
-__device__ __forceinline__ void load16_raw(const float *p, Raw16<float> &r) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) r.w[i] = reinterpret_cast<const float4 *>(p)[i];
-}
 template <typename T>
-__device__ __forceinline__ void load16_raw(const T *p, Raw16<T> &r) {
-  r.w[0] = reinterpret_cast<const uint4 *>(p)[0];
-  r.w[1] = reinterpret_cast<const uint4 *>(p)[1];
-}
-__device__ __forceinline__ void unpack16(const Raw16<float> &r, float (&x)[16]) {
+__device__ __forceinline__ void load_a(const T *vec, int q, RawA<T> &r) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[4 * i] = r.w[i].x; x[4 * i + 1] = r.w[i].y; x[4 * i + 2] = r.w[i].z; x[4 * i + 3] = r.w[i].w;
+  for (int m = 0; m < 8; ++m) r.w[m] = *reinterpret_cast<const uint32_t *>(vec + 16 * m + 2 * q);
+}
+__device__ __forceinline__ void load_a(const float *vec, int q, RawA<float> &r) {
+#pragma unroll
+  for (int m = 0; m < 8; ++m) r.w[m] = *reinterpret_cast<const float2 *>(vec + 16 * m + 2 * q);
+}
+// Unpack to fp32 with the signs D applied (sgn[m]: bit 15 and bit 31 flip
+// coordinate 16m + 2q and 16m + 2q + 1).
+__device__ __forceinline__ void unpack_a(const RawA<__nv_bfloat16> &r, const uint32_t (&sgn)[8], float2 (&a)[8]) {
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const uint32_t w = r.w[m] ^ sgn[m];
+    a[m] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
   }
 }
-__device__ __forceinline__ void unpack16(const Raw16<__nv_bfloat16> &r, float (&x)[16]) {
+__device__ __forceinline__ void unpack_a(const RawA<__half> &r, const uint32_t (&sgn)[8], float2 (&a)[8]) {
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint32_t w[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      x[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
-      x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
+  for (int m = 0; m < 8; ++m) {
+    const uint32_t w = r.w[m] ^ sgn[m];
+    a[m] = __half22float2(*reinterpret_cast<const __half2 *>(&w));
   }
 }
-__device__ __forceinline__ void unpack16(const Raw16<__half> &r, float (&x)[16]) {
+__device__ __forceinline__ void unpack_a(const RawA<float> &r, const uint32_t (&sgn)[8], float2 (&a)[8]) {
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint32_t w[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
-      x[8 * i + 2 * k] = f.x;
-      x[8 * i + 2 * k + 1] = f.y;
-    }
-  }
+  for (int m = 0; m < 8; ++m)
+    a[m] = make_float2(__uint_as_float(__float_as_uint(r.w[m].x) ^ (sgn[m] << 16)),
+                       __uint_as_float(__float_as_uint(r.w[m].y) ^ (sgn[m] & 0x80000000u)));
 }
-
-__device__ __forceinline__ void load16(const float *p, float (&x)[16]) {
+// sum of the lane's 16 squares (signs do not matter): pairs, then a tree
+__device__ __forceinline__ float lane_squares(const float2 (&a)[8]) {
+  float2 s[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float4 v = reinterpret_cast<const float4 *>(p)[i];
-    x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
-  }
+  for (int i = 0; i < 4; ++i) s[i] = __ffma2_rn(a[2 * i + 1], a[2 * i + 1], __fmul2_rn(a[2 * i], a[2 * i]));
+  const float2 t = add2(add2(s[0], s[1]), add2(s[2], s[3]));
+  return t.x + t.y;
 }
-__device__ __forceinline__ void load16(const __nv_bfloat16 *p, float (&x)[16]) {
+// The lane's strip constants: the sign masks of its layout-A coordinates and
+// its SO(4) blocks 4q + k as column pairs, mc[k][r][j] = (M[r][2j], M[r][2j + 1]).
+struct LaneConsts {
+  uint32_t sgn[8];
+  float2 mc[4][4][2];
+};
+__device__ __forceinline__ void lane_consts(const HeadParams &hp, int q, LaneConsts &c) {
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint4 u = reinterpret_cast<const uint4 *>(p)[i];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      x[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
-      x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
+  for (int m = 0; m < 8; ++m) {
+    const int j = 16 * m + 2 * q;  // even: both coordinates in one sign word
+    const uint32_t bits = (hp.sign_bits[j >> 5] >> (j & 31)) & 3u;
+    c.sgn[m] = ((bits & 1u) << 15) | ((bits >> 1) << 31);
   }
-}
-__device__ __forceinline__ void load16(const __half *p, float (&x)[16]) {
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint4 u = reinterpret_cast<const uint4 *>(p)[i];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  for (int k = 0; k < 4; ++k) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
-      x[8 * i + 2 * k] = f.x;
-      x[8 * i + 2 * k + 1] = f.y;
+    for (int r = 0; r < 4; ++r) {
+      const float4 row = reinterpret_cast<const float4 *>(hp.m32[4 * q + k])[r];
+      c.mc[k][r][0] = make_float2(row.x, row.y);
+      c.mc[k][r][1] = make_float2(row.z, row.w);
     }
   }
 }
 
-// Sylvester WHT (unnormalised) of 128 values held 16 per lane by the 8 lanes
-// of a group, lane q holding elements 16q..16q+15 (q = lane & 7).  The lower
-// index of each butterfly keeps a+b, the upper one a-b.
-__device__ __forceinline__ void wht128_wide(float (&v)[16], int q) {
+__device__ __forceinline__ float group_sum(float s) {
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 4);
+  return s;
+}
+// min of three (one instruction on sm_100)
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// The rotation of one lane group's vector, a in layout A with the signs D
+// applied: the unnormalised Sylvester WHT (its sqrt(128) cancels against the
+// one of z = sqrt(128) y / n) and the SO(4) blocks, leaving y[i] =
+// coordinate 16q + i of B H D x.  The lower index of each butterfly keeps
+// a + b, the upper one a - b.  `tile` is the warp's shared tile; every lane
+// of the warp calls this together.
+__device__ __forceinline__ void rotate_two_layouts(float2 (&a)[8], const LaneConsts &c, float *tile, int grp, int q,
+                                                   float (&y)[16]) {
+  // strides 16, 32, 64: bits 0, 1, 2 of m
 #pragma unroll
-  for (int s = 1; s < 16; s <<= 1) {
+  for (int s = 1; s < 8; s <<= 1) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i & s) continue;
-      const float a = v[i], b = v[i + s];
-      v[i] = a + b;
-      v[i + s] = a - b;
+    for (int m = 0; m < 8; ++m) {
+      if (m & s) continue;
+      const float2 u = a[m], v = a[m + s];
+      a[m] = add2(u, v);
+      a[m + s] = sub2(u, v);
     }
   }
+  // layout A -> layout B: row m of the vector's tile holds 16m .. 16m + 15
+  float *tv = tile + grp * kTileVec;
+  __syncwarp();
 #pragma unroll
-  for (int m = 1; m < 8; m <<= 1) {
-    // lower lane: v + p; upper lane: p - v
-    const float sgn = (q & m) ? -1.f : 1.f;
+  for (int m = 0; m < 8; ++m) *reinterpret_cast<float2 *>(tv + m * kTileRow + 2 * q) = a[m];
+  __syncwarp();
+  float2 b[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float p = __shfl_xor_sync(0xffffffffu, v[i], m);
-      v[i] = fmaf(sgn, v[i], p);
+  for (int j = 0; j < 4; ++j) {
+    const float4 v = *reinterpret_cast<const float4 *>(tv + q * kTileRow + 4 * j);
+    b[2 * j] = make_float2(v.x, v.y);
+    b[2 * j + 1] = make_float2(v.z, v.w);
+  }
+  // stride 1 inside each pair; strides 2, 4, 8 between pairs
+#pragma unroll
+  for (int k = 0; k < 8; ++k) b[k] = make_float2(b[k].x + b[k].y, b[k].x - b[k].y);
+#pragma unroll
+  for (int s = 1; s < 8; s <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k & s) continue;
+      const float2 u = b[k], v = b[k + s];
+      b[k] = add2(u, v);
+      b[k + s] = sub2(u, v);
+    }
+  }
+  // SO(4) block 4q + k on coordinates 16q + 4k .. 16q + 4k + 3 = b[2k], b[2k + 1]
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float2 t = __ffma2_rn(c.mc[k][r][1], b[2 * k + 1], __fmul2_rn(c.mc[k][r][0], b[2 * k]));
+      y[4 * k + r] = t.x + t.y;
     }
   }
 }
@@ -235,58 +284,6 @@ __device__ __forceinline__ void pack_store_wide(uint64_t cbits, int q, bool stor
   }
 }
 
-// The fp32 fast path of one lane group's vector, shared by the compress
-// kernels and the z export: the squared norm (exact squares of bf16/fp16
-// inputs, a 7-level tree: 4 in the lane, 3 across the group), 1/n from the
-// hardware reciprocal square root plus one Newton step (~1e-7), the signs
-// and the unnormalised WHT in place, then z of coordinate 16q + 4k + r as
-// (row r of SO(4) block 4q + k) . x / n.  sqrt(128) of the normalised Hn
-// cancels against the sqrt(128) of z = sqrt(128) * y / n.
-struct FastNorm {
-  float ssf, n32, inv;
-};
-__device__ __forceinline__ FastNorm fast_norm(const float (&x)[16]) {
-  float sq[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) sq[i] = x[i] * x[i];
-#pragma unroll
-  for (int s = 8; s >= 1; s >>= 1)
-#pragma unroll
-    for (int i = 0; i < s; ++i) sq[i] += sq[i + s];
-  float ssf = sq[0];
-  ssf += __shfl_xor_sync(0xffffffffu, ssf, 1);
-  ssf += __shfl_xor_sync(0xffffffffu, ssf, 2);
-  ssf += __shfl_xor_sync(0xffffffffu, ssf, 4);
-  FastNorm f;
-  f.ssf = ssf;
-  f.n32 = sqrtf(ssf);
-  const float rs = rsqrtf(ssf);
-  f.inv = rs * (1.5f - 0.5f * ssf * rs * rs);
-  return f;
-}
-__device__ __forceinline__ void fast_signs_wht(float (&x)[16], uint32_t sbits, int q) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(__float_as_uint(x[i]) ^ (((sbits >> i) & 1u) << 31));
-  wht128_wide(x, q);
-}
-__device__ __forceinline__ float fast_z(const float (&mrow)[4][16], const float (&x)[16], int k, int r, float inv) {
-  const float yr = fmaf(mrow[k][4 * r + 3], x[4 * k + 3],
-                        fmaf(mrow[k][4 * r + 2], x[4 * k + 2],
-                             fmaf(mrow[k][4 * r + 1], x[4 * k + 1], mrow[k][4 * r] * x[4 * k])));
-  return yr * inv;
-}
-// The lane's sign bits (coordinates 16q..16q+15) and SO(4) blocks 4q..4q+3.
-__device__ __forceinline__ void lane_blocks(const HeadParams &hp, int q, uint32_t &sbits, float (&mrow)[4][16]) {
-  sbits = (hp.sign_bits[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float4 row = reinterpret_cast<const float4 *>(hp.m32[4 * q + k])[r];
-      mrow[k][4 * r] = row.x; mrow[k][4 * r + 1] = row.y; mrow[k][4 * r + 2] = row.z; mrow[k][4 * r + 3] = row.w;
-    }
-  }
-}
 
 // The fp64 path for one vector, by the whole warp (lane l: coordinates
 // 4l..4l+3): norm, rotation and codes all in fp64.  Used for the few vectors
@@ -343,11 +340,15 @@ __device__ void compress_one_fp64(const HeadParams &hp, const Codebook &cb, cons
   if (lane == 0) norms[(block << ps_shift) + off] = n16;
 }
 
+
 // Warp w of the K (kv = 0) or V (kv = 1) half: rotate, quantize and pack
 // tokens strip * (w / H) .. + strip - 1 of head w % H, four at a time.
+// `tile` is the warp's shared tile (kTileFloats floats).
 template <typename T, int BITS>
-__device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uint32_t w, int lane) {
+__device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uint32_t w, int lane, float *tile) {
   constexpr int kHalf = 1 << (BITS - 1);  // codes below kHalf are the negative levels
+  constexpr int kPos = kHalf - 1;         // positive thresholds (the middle one is 0)
+  constexpr uint32_t kAll = (1u << BITS) - 1u;
   constexpr int kW = words_for(BITS);
   const int H = g.H, n_tok = g.n_tok, ps_shift = g.ps_shift;
   const uint32_t strips = (static_cast<uint32_t>(n_tok) + g.strip - 1) / g.strip;
@@ -359,40 +360,39 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
   const T *__restrict__ src = static_cast<const T *>(kv ? g.vin : g.kin);
   const int grp = lane >> 3, q = lane & 7;
 
-  // this lane's sign bits and SO(4) blocks 4q..4q+3, for the whole strip
-  uint32_t sbits;
-  float mrow[4][16];
-  lane_blocks(hp, q, sbits, mrow);
-  // the positive thresholds (the codebook is symmetric; the middle one is 0)
-  float tp[kHalf - 1];
+  // this lane's sign masks and SO(4) blocks 4q..4q+3, for the whole strip
+  LaneConsts lc;
+  lane_consts(hp, q, lc);
+  // the positive thresholds (the codebook is symmetric)
+  float tp[kPos];
 #pragma unroll
-  for (int i = 0; i < kHalf - 1; ++i) tp[i] = cb.threshold[kHalf + i];
+  for (int i = 0; i < kPos; ++i) tp[i] = cb.threshold[kHalf + i];
 
   const int t_begin = static_cast<int>(sidx) * g.strip;
   const int t_end = min(t_begin + g.strip, n_tok);
   // the inputs and slot of the group's next vector are loaded one iteration
   // ahead, so that their latency overlaps the current vector's rotation
-  Raw16<T> nraw{};
+  RawA<T> nraw{};
   int64_t nslot = -1;
   if (t_begin + grp < t_end) {
     nslot = g.slots[t_begin + grp];
-    load16_raw(src + (static_cast<int64_t>(t_begin + grp) * H + h) * kD + 16 * q, nraw);
+    load_a(src + (static_cast<int64_t>(t_begin + grp) * H + h) * kD, q, nraw);
   }
   for (int tb = t_begin; tb < t_end; tb += 4) {
     const int t = tb + grp;
     const bool live = t < t_end;
-    float x[16];
+    float2 a[8];
     int64_t slot = -1;
     if (live) {
       slot = nslot;
-      unpack16(nraw, x);
+      unpack_a(nraw, lc.sgn, a);
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = 0.f;
+      for (int m = 0; m < 8; ++m) a[m] = make_float2(0.f, 0.f);
     }
     if (t + 4 < t_end) {
       nslot = g.slots[t + 4];
-      load16_raw(src + (static_cast<int64_t>(t + 4) * H + h) * kD + 16 * q, nraw);
+      load_a(src + (static_cast<int64_t>(t + 4) * H + h) * kD, q, nraw);
     }
     const int64_t page = slot >> ps_shift;
     const bool valid = live && slot >= 0 && page < g.num_pages;
@@ -402,8 +402,8 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
     // (4 levels in the lane, 3 across the group) is within 7 * 2^-24
     // relative; the fp16 norm is decided in fp32 unless n lies within 1e-6
     // (relative) of a rounding midpoint, or is huge, tiny or not finite
-    const FastNorm fn = fast_norm(x);
-    const float ssf = fn.ssf, n32 = fn.n32;
+    const float ssf = group_sum(lane_squares(a));
+    const float n32 = sqrtf(ssf);
     const __half h32 = __float2half_rn(fminf(n32, 65504.f));
     const float hv = __half2float(h32);
     const uint16_t hb = __half_as_ushort(h32);
@@ -411,35 +411,42 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
     const float dn = hb > 0 ? __half2float(__ushort_as_half(static_cast<uint16_t>(hb - 1))) : 0.f;
     const float mid = n32 >= hv ? 0.5f * (hv + up) : 0.5f * (hv + dn);
     bool slow = !(ssf > 1e-30f && n32 < 65000.f && fabsf(n32 - mid) > 1e-6f * n32);
-    const float inv = fn.inv;
 
-    // z = (B H D x) / n
-    fast_signs_wht(x, sbits, q);
-    // codes from |z| and the positive thresholds (the codebook is
-    // symmetric): z > 0 -> half + #{|z| > t}, otherwise half - 1 - #{|z| >= t}
+    float y[16];
+    rotate_two_layouts(a, lc, tile, grp, q, y);
+    // codes: z = y / n against the thresholds t, decided as |y| against
+    // t * n; neg = #{t : |y| < t * n} (the sign bits of the differences),
+    // so the code is neg for y < 0 and 2^BITS - 1 - neg for y > 0.  A
+    // coordinate within kRecheckBand of a threshold (0 included) in z units
+    // sends the vector to the fp64 path, so the fast path's comparisons
+    // (and its ties) only decide codes that the exact z decides the same way.
+    float thr[kPos];
+#pragma unroll
+    for (int i = 0; i < kPos; ++i) thr[i] = tp[i] * n32;
+    const float band = kRecheckBand * n32;
     uint64_t cbits = 0;
-    bool near = false;
+    float dmin = band;  // distance of the nearest coordinate to a threshold, capped
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int i = 0; i < 16; ++i) {
+      const float av = fabsf(y[i]);
+      uint32_t neg = 0;
+      float r[kPos];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float z = fast_z(mrow, x, k, r, inv);
-        const float a = fabsf(z);
-        // strict comparisons only: |z| equal to a threshold (or z = 0) is
-        // within the re-check band, so the fp64 path decides it and the tie
-        // rule of the fast path does not matter
-        uint32_t gt = 0;
-        float dm = a;  // distance to the nearest threshold (0 included)
+      for (int j = 0; j < kPos; ++j) {
+        r[j] = av - thr[j];
+        neg += __float_as_uint(r[j]) >> 31;
+      }
+      const uint32_t c = neg ^ (kAll & ~static_cast<uint32_t>(__float_as_int(y[i]) >> 31));
+      cbits |= static_cast<uint64_t>(c) << (BITS * i);
+      if constexpr (kPos == 1) {
+        dmin = fmin3(dmin, fabsf(r[0]), av);
+      } else {
 #pragma unroll
-        for (int i = 0; i < kHalf - 1; ++i) {
-          gt += a > tp[i] ? 1u : 0u;
-          dm = fminf(dm, fabsf(a - tp[i]));
-        }
-        const uint32_t c = z > 0.f ? kHalf + gt : kHalf - 1 - gt;
-        cbits |= static_cast<uint64_t>(c) << (BITS * (4 * k + r));
-        near |= dm < kRecheckBand;
+        for (int j = 0; j + 1 < kPos; j += 2) dmin = fmin3(dmin, fabsf(r[j]), fabsf(r[j + 1]));
+        dmin = fmin3(dmin, fabsf(r[kPos - 1]), av);
       }
     }
+    const bool near = dmin < band;
     // the group's verdict: any lane near a threshold sends the vector to
     // the fp64 path
     const uint32_t gmask = 0xFFu << (8 * grp);
@@ -473,14 +480,13 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
       const int64_t sl = __shfl_sync(0xffffffffu, slot, src_lane);
       const int64_t pg = sl >> ps_shift;
       compress_one_fp64<T, BITS>(hp, cb, src + (static_cast<int64_t>(tv) * H + h) * kD, g.codes, g.norms,
-                           (pg * 2 + kv) * H + h, static_cast<int>(sl & ((1 << ps_shift) - 1)), ps_shift, lane);
+                                 (pg * 2 + kv) * H + h, static_cast<int>(sl & ((1 << ps_shift) - 1)), ps_shift,
+                                 lane);
     }
   }
 }
 
-// warps per compress block; blockIdx.y selects K or V.  Four-warp blocks,
-// three per SM (bulk compression of 32768 x 8 vectors per layer: 0.218 ms
-// per layer against 0.261 ms with eight-warp blocks, two per SM).
+// warps per compress block; blockIdx.y selects K or V.
 #ifndef ISOQUANT_COMPRESS_WARPS
 #define ISOQUANT_COMPRESS_WARPS 4
 #endif
@@ -488,47 +494,56 @@ constexpr int kCompressWarps = ISOQUANT_COMPRESS_WARPS;  // warps per k_compress
 constexpr int kCompressBlocksPerSm = kCompressWarps == 8 ? 2 : 3;
 template <typename T, int BITS>
 __global__ void __launch_bounds__(kCompressWarps * 32, kCompressBlocksPerSm) k_compress(const CompressArgs g) {
+  __shared__ __align__(16) float tile[kCompressWarps][kTileFloats];
   pdl_trigger();
   pdl_wait();
-  compress_warp<T, BITS>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), threadIdx.x & 31);
+  const int warp = threadIdx.x >> 5;
+  compress_warp<T, BITS>(g, blockIdx.y, blockIdx.x * (blockDim.x >> 5) + warp, threadIdx.x & 31, tile[warp]);
 }
 
-// Debug export of the fast path's fp32 z: the same lane-group layout and the
-// same helpers as compress_warp, one vector per lane group, every
-// coordinate's z (fp32, before any fp64 re-check) written to
+// Debug export of the fast path's fp32 z: the same lane-group layouts and
+// the same helpers as compress_warp, one vector per lane group, every
+// coordinate's z = y / n (fp32, before any fp64 re-check; the compress
+// kernel compares |y| with t * n instead) written to
 // z[(t * H + h) * 128 + j].
 template <typename T>
 __global__ void __launch_bounds__(256) k_export_z(const HeadParams *params, const T *x, int n_tok, int H,
                                                   float *z) {
+  __shared__ __align__(16) float tile[8][kTileFloats];
   pdl_trigger();
   pdl_wait();
-  const int lane = threadIdx.x & 31, grp = lane >> 3, q = lane & 7;
-  const int64_t vec = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + grp;
+  const int lane = threadIdx.x & 31, grp = lane >> 3, q = lane & 7, warp = threadIdx.x >> 5;
+  const int64_t vec = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp) * 4 + grp;
   // whole warps exit together (the helpers shuffle within the group)
   if ((vec & ~int64_t(3)) >= static_cast<int64_t>(n_tok) * H) return;
   const bool live = vec < static_cast<int64_t>(n_tok) * H;
   const int h = live ? static_cast<int>(vec % H) : 0;
-  uint32_t sbits;
-  float mrow[4][16];
-  lane_blocks(params[h], q, sbits, mrow);
-  float v[16];
+  LaneConsts lc;
+  lane_consts(params[h], q, lc);
+  float2 a[8];
   if (live) {
-    load16(x + vec * kD + 16 * q, v);
+    RawA<T> raw;
+    load_a(x + vec * kD, q, raw);
+    unpack_a(raw, lc.sgn, a);
   } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+    for (int m = 0; m < 8; ++m) a[m] = make_float2(0.f, 0.f);
   }
-  const FastNorm fn = fast_norm(v);
-  fast_signs_wht(v, sbits, q);
-  float out[16];
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-#pragma unroll
-    for (int r = 0; r < 4; ++r) out[4 * k + r] = fn.ssf > 0.f ? fast_z(mrow, v, k, r, fn.inv) : 0.f;
+  const float ssf = group_sum(lane_squares(a));
+  // 1/n from the hardware reciprocal square root plus one Newton step
+  const float rs = rsqrtf(ssf);
+  const float inv = rs * (1.5f - 0.5f * ssf * rs * rs);
+  float y[16];
+  rotate_two_layouts(a, lc, tile[warp], grp, q, y);
   if (live) {
     float4 *dst = reinterpret_cast<float4 *>(z + vec * kD + 16 * q);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_float4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+    for (int i = 0; i < 4; ++i) {
+      float o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = ssf > 0.f ? y[4 * i + e] * inv : 0.f;
+      dst[i] = make_float4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -567,6 +582,7 @@ __global__ void __launch_bounds__(256) k_rotate_q(const RotateArgs g) {
 // rotate the queries.  Their latency chains overlap instead of adding up.
 template <typename T, int BITS>
 __global__ void __launch_bounds__(256) k_decode_prep(const CompressArgs c, const RotateArgs r, int nbc) {
+  __shared__ __align__(16) float tile[8][kTileFloats];
   pdl_trigger();
   pdl_wait();
   const uint32_t warp = threadIdx.x >> 5;
@@ -574,7 +590,7 @@ __global__ void __launch_bounds__(256) k_decode_prep(const CompressArgs c, const
   const int bx = static_cast<int>(blockIdx.x);
   if (bx < 2 * nbc) {
     const int kv = bx >= nbc ? 1 : 0;
-    compress_warp<T, BITS>(c, kv, static_cast<uint32_t>(bx - kv * nbc) * (blockDim.x >> 5) + warp, lane);
+    compress_warp<T, BITS>(c, kv, static_cast<uint32_t>(bx - kv * nbc) * (blockDim.x >> 5) + warp, lane, tile[warp]);
   } else {
     rotate_warp<T>(r, static_cast<uint32_t>(bx - 2 * nbc) * (blockDim.x >> 5) + warp, lane);
   }
