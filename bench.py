@@ -450,20 +450,36 @@ def _oracle_worker(job):
     return n, time.perf_counter() - t0
 
 
+def _compress_worker(job):
+    """One host process of the all-core bulk-compression leg: compress the
+    sample's vectors with the oracle until the budget is spent; returns the
+    vectors compressed and the time taken."""
+    import oracle
+    sample, start_at, budget_s, max_steps = job
+    while time.time() < start_at:
+        time.sleep(0.001)
+    n, t0 = 0, time.perf_counter()
+    while n < max_steps and (budget_s is None or time.perf_counter() - t0 < budget_s):
+        oracle.compress(sample["s"], sample["qt"], sample["x"], bits=sample["bits"])
+        n += 1
+    return n * len(sample["x"]), time.perf_counter() - t0
+
+
 class OraclePool:
     """`cores` spawned host processes, each running the oracle's decode step
-    on the sample (processes, not threads: the oracle is single-threaded C
-    behind ctypes; spawned, not forked, since the parent holds a CUDA
-    context)."""
+    (or, with `worker=_compress_worker`, its bulk compression) on the sample
+    (processes, not threads: the oracle is single-threaded C behind ctypes;
+    spawned, not forked, since the parent holds a CUDA context)."""
 
-    def __init__(self, sample, cores):
+    def __init__(self, sample, cores, worker=None):
         import multiprocessing as mp
         self.sample, self.cores = sample, cores
+        self.worker = worker or _oracle_worker
         self.pool = mp.get_context("spawn").Pool(cores)
 
     def run(self, budget_s=None, steps=1):
         start_at = time.time() + 0.5
-        res = self.pool.map(_oracle_worker, [(self.sample, start_at, budget_s, steps if budget_s is None else 1 << 40)]
+        res = self.pool.map(self.worker, [(self.sample, start_at, budget_s, steps if budget_s is None else 1 << 40)]
                             * self.cores, chunksize=1)
         return sum(r[0] for r in res), max(r[1] for r in res)
 
@@ -772,6 +788,46 @@ def run_prefill_attend(args):
     print(json.dumps(line))
 
 
+def compress_cpu_baseline(wl, cache, k, budget_s, n_vec=2048):
+    """The fp64 oracle's bulk compression, as it stands, on the host cores: a
+    bounded sample (the K vectors of the first n_vec tokens of KV head 0 of
+    layer 0, compressed again and again for budget_s) on one core and on
+    every core; plus the sample's codes and norms against the ones the GPU
+    wrote into layer 0's cache (mismatches, and coordinates within 1e-6 of a
+    threshold)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from compressed_space_decode_b200 import synthetic
+    signs, quats = synthetic.rotation_params(wl.seed, wl.kv_heads)
+    sample = {"s": signs[0].numpy(), "qt": quats[0].numpy(), "x": k[:n_vec, 0].double().cpu().numpy(), "bits": 3}
+    reps, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        oracle.compress(sample["s"], sample["qt"], sample["x"])
+        reps += 1
+    dt = time.perf_counter() - t0
+    one = {"value": reps * n_vec / dt, "unit": "vectors/s", "cores": 1, "sample": f"{reps} x {n_vec} vectors in {dt:.1f} s"}
+    cores = host_cores()
+    pool = OraclePool(sample, cores, worker=_compress_worker)
+    pool.run(steps=1)  # start-up, untimed
+    n, dt_all = pool.run(budget_s=budget_s)
+    pool.close()
+    oc, on, z, _ = oracle.compress(sample["s"], sample["qt"], sample["x"], want_z=True)
+    t = torch.arange(n_vec, device=cache.codes.device)
+    gc = cache.codes[t // 256, 0, 0, :, t % 256].to(torch.int64).cpu().numpy().astype(np.uint32)
+    gn = cache.norms[t // 256, 0, 0, t % 256].view(torch.int16).cpu().numpy().astype(np.uint16)
+    diff = (gc != oc).any(axis=1)
+    mism = int((oracle.unpack(gc[diff]) != oracle.unpack(oc[diff])).sum()) if diff.any() else 0
+    return {"value": n / dt_all, "unit": "vectors/s", "cores": cores, "kind": "oracle",
+            "sample": f"K vectors of tokens 0..{n_vec - 1}, KV head 0, layer 0 (bf16 in, 3-bit codes out); "
+                      f"{cores} host processes compressed {n} vectors in {dt_all:.1f} s",
+            "single_core": one,
+            "parity_sample": {"vectors": n_vec, "coords": n_vec * 128,
+                              "near_boundary_1e-6": int(oracle.near_boundary(z, 1e-6).sum()),
+                              "code_mismatches": mism, "norm_mismatches": int((gn != on).sum())}}
+
+
 def run_prefill(args):
     """Bulk compression of a long prompt: 32768 tokens x 8 KV heads x 48
     layers, K and V (isoquant_compress_kv per layer, one context per layer).
@@ -818,6 +874,7 @@ def run_prefill(args):
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1) / args.steps
+    cpu = None if args.no_cpu_baseline else compress_cpu_baseline(wl, caches[0], inputs[0][0], args.cpu_seconds)
     vectors = 2 * T * H * layers
     bytes_moved = vectors * (128 * 2 + 13 * 4 + 2)
     peak, peak_kind = peaks()
@@ -832,7 +889,7 @@ def run_prefill(args):
         "roofline": {"bound": "hbm", "kernel": "isoquant_compress_kv", "achieved": gbs, "peak": peak,
                      "unit": "GB/s", "frac": gbs / peak, "peak_kind": peak_kind,
                      "bytes_per_step": bytes_moved},
-        "gpu_launches": layers * args.steps, "clocks": clocks}))
+        "gpu_launches": layers * args.steps, "clocks": clocks, "cpu_baseline": cpu}))
 
 
 def main():

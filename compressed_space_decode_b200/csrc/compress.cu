@@ -491,7 +491,10 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
 #define ISOQUANT_COMPRESS_WARPS 4
 #endif
 constexpr int kCompressWarps = ISOQUANT_COMPRESS_WARPS;  // warps per k_compress block
-constexpr int kCompressBlocksPerSm = kCompressWarps == 8 ? 2 : 3;
+#ifndef ISOQUANT_COMPRESS_BLOCKS
+#define ISOQUANT_COMPRESS_BLOCKS (kCompressWarps == 8 ? 2 : 3)
+#endif
+constexpr int kCompressBlocksPerSm = ISOQUANT_COMPRESS_BLOCKS;
 template <typename T, int BITS>
 __global__ void __launch_bounds__(kCompressWarps * 32, kCompressBlocksPerSm) k_compress(const CompressArgs g) {
   __shared__ __align__(16) float tile[kCompressWarps][kTileFloats];
@@ -600,10 +603,22 @@ __global__ void __launch_bounds__(256) k_decode_prep(const CompressArgs c, const
 
 namespace {
 
-// Tokens per warp strip: long strips amortise loading a head's SO(4) blocks
-// in bulk compression; short ones spread a decode step's few tokens over
-// more warps.
-int strip_tokens(int n_tok) { return n_tok >= 4096 ? 16 : 4; }
+// Tokens per warp strip.  A strip loads its head's signs and SO(4) blocks
+// once, so long strips amortise that (bulk compression of 32768 x 8 vectors
+// per half: 0.187 ms per layer at 16 tokens, 0.162 at 32, 0.154 at 64); a
+// short batch (a decode step's few tokens) is spread over many warps
+// instead.  The strip is the longest multiple of 4, up to kMaxStrip, that
+// still gives each K/V half about as many warps as the SMs hold.
+#ifndef ISOQUANT_COMPRESS_STRIP
+#define ISOQUANT_COMPRESS_STRIP 64
+#endif
+constexpr int kMaxStrip = ISOQUANT_COMPRESS_STRIP;
+int strip_tokens(const isoquant_ctx *ctx, int n_tok) {
+  const int64_t vectors = static_cast<int64_t>(n_tok) * ctx->num_kv_heads;  // per K/V half
+  const int64_t resident = static_cast<int64_t>(ctx->num_sms) * 12;       // warps the SMs hold
+  const int64_t s = (vectors / resident) & ~int64_t(3);
+  return static_cast<int>(s < 4 ? 4 : (s > kMaxStrip ? kMaxStrip : s));
+}
 
 CompressArgs compress_args(const isoquant_ctx *ctx, const isoquant_cache *cache, const void *k, const void *v,
                            int n_tok, const int64_t *slot_mapping) {
@@ -621,14 +636,14 @@ CompressArgs compress_args(const isoquant_ctx *ctx, const isoquant_cache *cache,
   int ps_shift = 0;
   while ((1 << ps_shift) < cache->page_size) ++ps_shift;
   g.ps_shift = ps_shift;
-  g.strip = strip_tokens(n_tok);
+  g.strip = strip_tokens(ctx, n_tok);
   g.status = ctx->status;
   return g;
 }
 
-// compress blocks per K/V half (8 warps each, one strip per warp)
+// compress blocks per K/V half (warps_per_block warps each, one strip per warp)
 int64_t compress_blocks(const isoquant_ctx *ctx, int n_tok, int warps_per_block) {
-  const int strip = strip_tokens(n_tok);
+  const int strip = strip_tokens(ctx, n_tok);
   const int64_t warps = static_cast<int64_t>((n_tok + strip - 1) / strip) * ctx->num_kv_heads;
   return (warps + warps_per_block - 1) / warps_per_block;
 }
