@@ -150,6 +150,9 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": n}
 
 
+GRAPH_STEPS = 32  # decode steps (or attention calls) per CUDA graph under --graph
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -175,6 +178,11 @@ def run_ours(args):
     st = DecodeState(wl, growth=growth, device=dev, bits=args.bits)
     bytes_per_token_head = 2 * (csd.WORDS_FOR[args.bits] * 4 + 2)
     B, H, Hq, nq = st.B, st.H, st.Hq, wl.nq
+    if args.graph:
+        # graphs are captured on a side stream (not the legacy default one),
+        # which then stays the current stream for the whole run
+        torch.cuda.synchronize(dev)
+        torch.cuda.set_stream(torch.cuda.Stream(device=dev))
     stream = torch.cuda.current_stream(dev)
 
     # per-step inputs, generated up front (device-resident for the kernel metric)
@@ -227,14 +235,31 @@ def run_ours(args):
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid)
     launches[0] = 0
+    graphs = []
+    if args.graph:
+        # --graph: the timed steps are captured up front as CUDA graphs of
+        # GRAPH_STEPS consecutive steps each (every step its own inputs, so
+        # the context grows as without graphs) and replayed in order, so the
+        # host's per-call cost is off the timed path
+        attn_events = {}
+        for c0 in range(args.warmup, n_total, GRAPH_STEPS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for s in range(c0, min(c0 + GRAPH_STEPS, n_total)):
+                    step(s, k_all[s], v_all[s], q_all[s], slots_all[s], lens_all[s])
+            graphs.append(g)
     multi.barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for s in range(args.warmup, n_total):
-        step(s, k_all[s], v_all[s], q_all[s], slots_all[s], lens_all[s])
+    if args.graph:
+        for g in graphs:
+            g.replay()
+    else:
+        for s in range(args.warmup, n_total):
+            step(s, k_all[s], v_all[s], q_all[s], slots_all[s], lens_all[s])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
@@ -242,7 +267,7 @@ def run_ours(args):
     ms_local = t_start.elapsed_time(t_end)
     kernel_launches = launches[0]
     attn_ms = [e0.elapsed_time(e1) for e0, e1 in attn_events.values()]
-    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    attn_avg_ms = sum(attn_ms) / len(attn_ms) if attn_ms else ms_local / args.steps
 
     units_local = sum(int(lens_all[s].sum().item()) * H for s in range(args.warmup, n_total))
     ms = multi.max_over_ranks(ms_local, device=dev)
@@ -255,29 +280,44 @@ def run_ours(args):
     # over the cache as the timed loop left it (larger than L2)
     lens_last = lens_all[n_total - 1]
     n_attn = max(200, int(math.ceil(args.attn_seconds * 1e3 / max(attn_avg_ms, 1e-3))))
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_attn)]
     attn_launches = 0
+    if args.graph:
+        # the attention call GRAPH_STEPS times in one graph; events around
+        # each replay, per-call time = replay time / GRAPH_STEPS
+        ga = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ga, stream=stream):
+            for _ in range(GRAPH_STEPS):
+                csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, lens_last, ws, out,
+                                           causal=wl.causal, stream=stream)
+        n_attn = GRAPH_STEPS * max(1, n_attn // GRAPH_STEPS)
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_attn // GRAPH_STEPS if args.graph else n_attn)]
     multi.barrier()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(uuid)
     sampler.start()
     for ea, eb in attn_ev:
         ea.record(stream)
-        csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, lens_last, ws, out, causal=wl.causal,
-                                   stream=stream)
-        attn_launches += csd.isoquant_last_launch_count(st.ctx)
+        if args.graph:
+            ga.replay()
+        else:
+            csd.isoquant_attend_decode(st.ctx, st.cache, q_rot, st.page_table, lens_last, ws, out, causal=wl.causal,
+                                       stream=stream)
+            attn_launches += csd.isoquant_last_launch_count(st.ctx)
         eb.record(stream)
     torch.cuda.synchronize(dev)
     clocks_attn = sampler.stop()
     multi.barrier()
-    loop_ms = sorted(ea.elapsed_time(eb) for ea, eb in attn_ev)
+    per_call = GRAPH_STEPS if args.graph else 1
+    loop_ms = sorted(ea.elapsed_time(eb) / per_call for ea, eb in attn_ev)
     attn_med_ms = loop_ms[len(loop_ms) // 2]
 
     # roofline of the attention kernel: algorithmic bytes per launch / duration
     bytes_per_launch = bytes_per_token_head * int(lens_last.sum().item()) * H
     bytes_in_step = bytes_per_token_head * units_local / args.steps
     achieved = bytes_per_launch / (attn_med_ms / 1e3) / 1e9
-    achieved_in_step = bytes_in_step / (attn_avg_ms / 1e3) / 1e9
+    # (under --graph no events sit between a step's launches: no in-step figure)
+    achieved_in_step = bytes_in_step / (attn_avg_ms / 1e3) / 1e9 if attn_ms else None
     peak, peak_kind = peaks()
     # the profiled traffic is that of the 3-bit mma.sync kernel
     traffic = None  # set below once the kernel is known
@@ -356,6 +396,8 @@ def run_ours(args):
         "config": {"workload": wl.name.split("@")[0], "batch": B, "q_heads": Hq, "kv_heads": H, "head_dim": 128,
                    "context_start": lens0[0], "page_size": st.ps, "page_table": "shuffled",
                    "step": f"decode_prep (append {adv} token(s)/seq + rotate q, one launch) + attend_decode (split-K attention + combine); programmatic launches",
+                   "launch": (f"CUDA graphs of {GRAPH_STEPS} steps, replayed" if args.graph else
+                              "one library call per half step from the host"),
                    "l2": f"packed cache {bytes_per_launch / 1e6:.0f} MB > 126 MB L2; no flush",
                    "parallelism": f"dp{world} (independent shards)", "code_bits": args.bits,
                    "bytes_per_kv_token_head": bytes_per_token_head},
@@ -367,8 +409,10 @@ def run_ours(args):
                      "bytes_per_launch": bytes_per_launch, "avg_launch_ms": attn_med_ms,
                      "launches_timed": n_attn, "launch_ms_p10_p90": [loop_ms[len(loop_ms) // 10],
                                                                      loop_ms[(9 * len(loop_ms)) // 10]],
-                     "loop": f"{n_attn} attention calls back to back, CUDA events around each (median); "
-                             f"clocks sampled over the loop",
+                     "loop": (f"{n_attn} attention calls back to back in graphs of {GRAPH_STEPS}, CUDA events "
+                              f"around each replay (median per call); clocks sampled over the loop" if args.graph else
+                              f"{n_attn} attention calls back to back, CUDA events around each (median); "
+                              f"clocks sampled over the loop"),
                      "clocks": clocks_attn,
                      "achieved_in_step": achieved_in_step, "in_step_launches_timed": len(attn_ms),
                      "frac_of_8TBps": achieved / 8000.0},
@@ -907,6 +951,8 @@ def main():
     ap.add_argument("--attn-seconds", type=float, default=1.0,
                     help="length of the attention-only loop behind the roofline figure")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the timed decode steps (and the attention loop) as CUDA graphs and replay them")
     ap.add_argument("--bits", type=int, default=3, choices=[2, 3, 4],
                     help="code width of the decode workload (3: the method's; 2 and 4: other widths)")
     args = ap.parse_args()
