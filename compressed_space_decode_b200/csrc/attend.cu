@@ -533,25 +533,35 @@ __device__ __forceinline__ uint32_t k_pair(const uint4 (&kw)[4], int j, int k, u
 __device__ __forceinline__ int64_t cta_of_page(int64_t g, int64_t N, int64_t P) {
   return ((g + 1) * N + P - 1) / P - 1;
 }
-__device__ __forceinline__ bool cta_empty(int64_t c, int64_t N, int64_t P) {
-  return c * P / N == (c + 1) * P / N;
-}
+// The CTAs that hold a pair's pages [g0, g0 + np) of the P pages split over
+// N CTAs: with P >= N every CTA of the range c_lo..c_hi holds at least one
+// page; with fewer pages than CTAs each CTA holds at most one, so the owners
+// are the np pages' CTAs, and the many CTAs in between (empty ranges, no
+// record) are never visited.
+struct Owners {
+  int64_t c_lo, g0, N, P, count;
+  bool dense;
+  __device__ Owners(int64_t g0_, int np, int64_t N_, int64_t P_) : g0(g0_), N(N_), P(P_) {
+    c_lo = cta_of_page(g0, N, P);
+    dense = P >= N;
+    count = dense ? cta_of_page(g0 + np - 1, N, P) - c_lo + 1 : np;
+  }
+  __device__ int64_t at(int64_t j) const { return dense ? c_lo + j : cta_of_page(g0 + j, N, P); }
+};
 
-// Merge the records that CTAs c_lo..c_hi wrote for rows rr[0..NR) of
-// `pair`, divide by l and apply R^-1 = D Hn B^T of head parameters hp; the
-// warp stores row k's 128 outputs at dst[k] (lane holds dims 4 lane ..
-// 4 lane + 3), or skips row k when dst[k] is null.  CTAs with an empty page
-// range (possible only when there are fewer pages than CTAs) wrote no record
-// and are skipped.  Latency, not bandwidth, bounds this: lane i fetches the
-// (m, l) of record c_lo + i, and the o vectors are fetched 8 (record, row)
-// pairs at a time before any is used.  Records are read through L2
+// Merge the records that the owners of `pair`'s pages wrote for rows
+// rr[0..NR), divide by l and apply R^-1 = D Hn B^T of head parameters hp;
+// the warp stores row k's 128 outputs at dst[k] (lane holds dims 4 lane ..
+// 4 lane + 3), or skips row k when dst[k] is null.  Latency, not bandwidth,
+// bounds this: lane i fetches the (m, l) of owner i's record, and the o
+// vectors are fetched 8 (record, row) pairs at a time before any is used.  Records are read through L2
 // (ld.global.cg): in the fused path other CTAs of the running grid wrote
 // them.
 // Record of CTA c for the stream: slot (c + stream) * per + sub.
 template <int NR>
-__device__ __forceinline__ void merge_rows(const float *records, int64_t pair, int per, int sub, int64_t c_lo,
-                                           int64_t c_hi, int64_t N, int64_t total, const int (&rr)[NR],
-                                           float *const (&dst)[NR], const HeadParams &hp, int lane) {
+__device__ __forceinline__ void merge_rows(const float *records, int64_t pair, int per, int sub, const Owners &own,
+                                           const int (&rr)[NR], float *const (&dst)[NR], const HeadParams &hp,
+                                           int lane) {
   // this lane's rows of B^T, fetched first so that their latency overlaps
   const float4 *mb4 = reinterpret_cast<const float4 *>(hp.m32[lane]);
   const float4 mb[4] = {mb4[0], mb4[1], mb4[2], mb4[3]};
@@ -561,14 +571,15 @@ __device__ __forceinline__ void merge_rows(const float *records, int64_t pair, i
   float mr[NR], lr[NR], m0[NR];
 #pragma unroll
   for (int k = 0; k < NR; ++k) { mr[k] = -INFINITY; lr[k] = 0.f; m0[k] = -INFINITY; }
-  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
-    const int64_t c = c0 + lane;
-    if (c <= c_hi && !cta_empty(c, N, total)) {
-      const float *rec = records + ((c + pair) * per + sub) * kRecordFloats;
+  const int64_t count = own.count;
+  for (int64_t j0 = 0; j0 < count; j0 += 32) {
+    const int64_t j = j0 + lane;
+    if (j < count) {
+      const float *rec = records + ((own.at(j) + pair) * per + sub) * kRecordFloats;
 #pragma unroll
       for (int k = 0; k < NR; ++k) {
         const float2 ml = __ldcg(reinterpret_cast<const float2 *>(rec + 2 * rr[k]));
-        if (c0 == c_lo) m0[k] = ml.x;
+        if (j0 == 0) m0[k] = ml.x;
         if (ml.x > mr[k]) {
           lr[k] = lr[k] * ex2(mr[k] - ml.x) + ml.y;
           mr[k] = ml.x;
@@ -590,24 +601,27 @@ __device__ __forceinline__ void merge_rows(const float *records, int64_t pair, i
     o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
   }
   // pass 2: o = sum over records of 2^(m - M) o_c
-  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 32) {
-    const int64_t c = c0 + lane;
-    const bool mine = c <= c_hi && !cta_empty(c, N, total);
+  for (int64_t j0 = 0; j0 < count; j0 += 32) {
+    const int64_t j = j0 + lane;
+    const bool mine = j < count;
+    // this lane's owner (record slot), handed to the other lanes below
+    const int64_t slot = ((mine ? own.at(j) : own.c_lo) + pair) * per + sub;
     float sm[NR];
 #pragma unroll
     for (int k = 0; k < NR; ++k) {
       float mc = m0[k];
-      if (c0 != c_lo) mc = mine ? __ldcg(records + ((c + pair) * per + sub) * kRecordFloats + 2 * rr[k]) : -INFINITY;
+      if (j0 != 0) mc = mine ? __ldcg(records + slot * kRecordFloats + 2 * rr[k]) : -INFINITY;
       sm[k] = (!mine || M[k] == -INFINITY) ? 0.f : ex2(mc - M[k]);
     }
-    const int n = static_cast<int>(c_hi - c0 + 1 < 32 ? c_hi - c0 + 1 : 32);
+    const int n = static_cast<int>(count - j0 < 32 ? count - j0 : 32);
     constexpr int kBatch = 8 / NR;
     for (int i0 = 0; i0 < n; i0 += kBatch) {
       float sv[kBatch][NR];
       float4 v[kBatch][NR];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        const float *rec = records + ((c0 + i0 + u + pair) * per + sub) * kRecordFloats + 16 + 4 * lane;
+        const int64_t sl = __shfl_sync(0xffffffffu, slot, (i0 + u) & 31);
+        const float *rec = records + sl * kRecordFloats + 16 + 4 * lane;
 #pragma unroll
         for (int k = 0; k < NR; ++k) {
           sv[u][k] = __shfl_sync(0xffffffffu, sm[k], (i0 + u) & 31);
@@ -2298,10 +2312,9 @@ __global__ void __launch_bounds__(kCombineThreads) k_attend_combine(const Combin
     for (int k = 0; k < NR; ++k) *reinterpret_cast<float4 *>(dsts[k]) = make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
-  const int64_t N = p.n_cta;
-  const int64_t c_lo = cta_of_page(g0, N, total), c_hi = cta_of_page(g0 + np - 1, N, total);
+  const Owners own(g0, np, p.n_cta, total);
   const int64_t pair = (static_cast<int64_t>(rg) * p.B + b) * p.H + h;
-  merge_rows<NR>(p.records, pair, p.rps >> 3, sub, c_lo, c_hi, N, total, rows, dsts, p.params[h], lane);
+  merge_rows<NR>(p.records, pair, p.rps >> 3, sub, own, rows, dsts, p.params[h], lane);
 }
 
 }  // namespace
