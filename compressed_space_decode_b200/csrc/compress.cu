@@ -400,17 +400,20 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
 
     // ||x||^2 in fp32: squares of bf16/fp16 inputs are exact and the tree
     // (4 levels in the lane, 3 across the group) is within 7 * 2^-24
-    // relative; the fp16 norm is decided in fp32 unless n lies within 1e-6
-    // (relative) of a rounding midpoint, or is huge, tiny or not finite
+    // relative; n32 = sqrt of it by sqrt.approx (within 2^-22), so n32 is
+    // within ~5e-7 of the exact norm.  Its fp16 rounding is decided from
+    // n32's bits: fp16 keeps the top 10 of fp32's 23 mantissa bits, so the
+    // 13 below them place n32 inside an fp16 step, whose rounding midpoint
+    // is 0x1000.  A pattern 16 or more fp32 units from it lies at least
+    // 2^-20 (9.5e-7) relative from the midpoint, so the exact norm rounds
+    // the same way; closer, or outside the fp16 normal range below 65000
+    // (or not finite), the fp64 path decides.
     const float ssf = group_sum(lane_squares(a));
-    const float n32 = sqrtf(ssf);
-    const __half h32 = __float2half_rn(fminf(n32, 65504.f));
-    const float hv = __half2float(h32);
-    const uint16_t hb = __half_as_ushort(h32);
-    const float up = __half2float(__ushort_as_half(static_cast<uint16_t>(hb + 1)));
-    const float dn = hb > 0 ? __half2float(__ushort_as_half(static_cast<uint16_t>(hb - 1))) : 0.f;
-    const float mid = n32 >= hv ? 0.5f * (hv + up) : 0.5f * (hv + dn);
-    bool slow = !(ssf > 1e-30f && n32 < 65000.f && fabsf(n32 - mid) > 1e-6f * n32);
+    float n32;
+    asm("sqrt.approx.f32 %0, %1;" : "=f"(n32) : "f"(ssf));
+    const uint16_t hb = __half_as_ushort(__float2half_rn(fminf(n32, 65504.f)));
+    const int mid_off = static_cast<int>(__float_as_uint(n32) & 0x1FFFu) - 0x1000;
+    bool slow = !(n32 >= 6.103515625e-05f && n32 < 65000.f && (mid_off >= 16 || mid_off <= -16));
 
     float y[16];
     rotate_two_layouts(a, lc, tile, grp, q, y);
@@ -426,24 +429,51 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
     const float band = kRecheckBand * n32;
     uint64_t cbits = 0;
     float dmin = band;  // distance of the nearest coordinate to a threshold, capped
+    if constexpr (BITS == 3) {
+      // The code's three bits straight from sign bits: with s_k the sign bit
+      // of |y| - t_k n (t ascending, so s_1 <= s_2 <= s_3) and p = (y > 0),
+      // neg = s_1 + s_2 + s_3 has bit 0 = s_1 ^ s_2 ^ s_3 and bit 1 = s_2, so
+      // the code neg ^ (p ? 7 : 0) has bits (s_1^s_2^s_3^p, s_2^p, p).  Bit
+      // 31 of y is ~p, so the words below carry each bit inverted; funnel
+      // shifts collect bit 31 of each, coordinates 0..9 into one word and
+      // 10..15 into another (highest coordinate first, its bit 2 first), and
+      // one XOR per word undoes the inversion.
+      uint32_t wa = 0, wb = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float av = fabsf(y[i]);
-      uint32_t neg = 0;
-      float r[kPos];
-#pragma unroll
-      for (int j = 0; j < kPos; ++j) {
-        r[j] = av - thr[j];
-        neg += __float_as_uint(r[j]) >> 31;
+      for (int i = 15; i >= 0; --i) {
+        const float av = fabsf(y[i]);
+        const float r0 = av - thr[0], r1 = av - thr[1], r2 = av - thr[2];
+        const uint32_t yb = __float_as_uint(y[i]);
+        const uint32_t i0 = __float_as_uint(r0) ^ __float_as_uint(r1) ^ __float_as_uint(r2) ^ yb;
+        const uint32_t i1 = __float_as_uint(r1) ^ yb;
+        uint32_t &acc = i >= 10 ? wb : wa;
+        acc = __funnelshift_l(yb, acc, 1);
+        acc = __funnelshift_l(i1, acc, 1);
+        acc = __funnelshift_l(i0, acc, 1);
+        dmin = fmin3(dmin, fabsf(r0), fabsf(r1));
+        dmin = fmin3(dmin, fabsf(r2), av);
       }
-      const uint32_t c = neg ^ (kAll & ~static_cast<uint32_t>(__float_as_int(y[i]) >> 31));
-      cbits |= static_cast<uint64_t>(c) << (BITS * i);
-      if constexpr (kPos == 1) {
-        dmin = fmin3(dmin, fabsf(r[0]), av);
-      } else {
+      cbits = static_cast<uint64_t>(wa ^ 0x3FFFFFFFu) | (static_cast<uint64_t>(wb ^ 0x3FFFFu) << 30);
+    } else {
 #pragma unroll
-        for (int j = 0; j + 1 < kPos; j += 2) dmin = fmin3(dmin, fabsf(r[j]), fabsf(r[j + 1]));
-        dmin = fmin3(dmin, fabsf(r[kPos - 1]), av);
+      for (int i = 0; i < 16; ++i) {
+        const float av = fabsf(y[i]);
+        uint32_t neg = 0;
+        float r[kPos];
+#pragma unroll
+        for (int j = 0; j < kPos; ++j) {
+          r[j] = av - thr[j];
+          neg += __float_as_uint(r[j]) >> 31;
+        }
+        const uint32_t c = neg ^ (kAll & ~static_cast<uint32_t>(__float_as_int(y[i]) >> 31));
+        cbits |= static_cast<uint64_t>(c) << (BITS * i);
+        if constexpr (kPos == 1) {
+          dmin = fmin3(dmin, fabsf(r[0]), av);
+        } else {
+#pragma unroll
+          for (int j = 0; j + 1 < kPos; j += 2) dmin = fmin3(dmin, fabsf(r[j]), fabsf(r[j + 1]));
+          dmin = fmin3(dmin, fabsf(r[kPos - 1]), av);
+        }
       }
     }
     const bool near = dmin < band;

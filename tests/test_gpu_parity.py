@@ -119,6 +119,41 @@ def test_compress_bit_exact_all_dtypes(cuda_lib):
             print(dtype, h, stats)
 
 
+def test_compress_norms_at_fp16_midpoints(cuda_lib):
+    """Vectors scaled so that their norm sits on an fp16 rounding midpoint
+    (and a few fp32 units either side of it), across binades from 2^-13 to
+    2^15: the fp16 norm must still round as the oracle's fp64 norm does, so
+    these must take the re-check path where the fp32 norm cannot decide."""
+    from compressed_space_decode_b200 import synthetic
+    H, n = 1, 768
+    signs, quats = synthetic.rotation_params(81, H)
+    ctx = cuda_lib.isoquant_init(signs, quats)
+    cache = cuda_lib.PagedCache.allocate(H, (n + 255) // 256, 256)
+    rng = np.random.default_rng(82)
+    v = rng.standard_normal((n, D))
+    v /= np.linalg.norm(v, axis=1, keepdims=True)
+    # midpoint between two adjacent fp16 values of binade 2^e, nudged by k fp64 steps of 2^-24 relative
+    e = rng.integers(-13, 15, n)
+    m = rng.integers(0, 1023, n)
+    mid = (1.0 + (m + 0.5) / 1024.0) * np.exp2(e)
+    k = rng.integers(-12, 13, n)
+    target = mid * (1.0 + k * 2.0 ** -24)
+    x = torch.tensor((v * target[:, None])[:, None, :], dtype=torch.float32, device="cuda")
+    slots = torch.arange(n, dtype=torch.int64, device="cuda")
+    cuda_lib.isoquant_compress_kv(ctx, cache, x, x, slots)
+    torch.cuda.synchronize()
+    assert cuda_lib.isoquant_get_status(ctx) == 0
+    codes = cache.codes[:, 0, 0].permute(0, 2, 1).reshape(-1, 13)[:n]
+    norms = cache.norms[:, 0, 0].reshape(-1)[:n]
+    gc = codes.cpu().numpy().view(np.uint32)
+    gn = norms.cpu().numpy().view(np.uint16)
+    stats, _, _ = compare_compressed(x[:, 0].double().cpu().numpy(), signs[0].numpy(), quats[0].numpy(), gc, gn)
+    print(stats)
+    # the exemption band of compare_compressed is not needed: the re-check
+    # decides every one of them as the fp64 norm does
+    assert stats["norm_near_midpoint"] > n // 4 and stats["norm_mismatch"] == 0, stats
+
+
 def test_compress_slot_rules(cuda_lib):
     from compressed_space_decode_b200 import synthetic
     H = 1
