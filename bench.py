@@ -349,8 +349,11 @@ def run_ours(args):
     kd, vd = torch.empty_like(k_all[0]), torch.empty_like(v_all[0])
     qd, sd, ld = torch.empty_like(q_all[0]), torch.empty_like(slots_all[0]), torch.empty_like(lens_all[0])
     layout, row_bytes = stage_layout((kd, vd, qd, sd, ld))
-    stage_d = torch.empty(row_bytes, dtype=torch.uint8, device=dev)
-    kd, vd, qd, sd, ld = (stage_d[o:o + n].view(dt).view(shp) for o, n, dt, shp in layout)
+    # two device staging rows and two outputs, so that a step's copies overlap
+    # the neighbouring steps' kernels
+    stage_ds = [torch.empty(row_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dviews = [[sd_[o:o + n].view(dt).view(shp) for o, n, dt, shp in layout] for sd_ in stage_ds]
+    outs = [out, torch.empty_like(out)]
     stage_h = torch.zeros((e2e_steps, row_bytes), dtype=torch.uint8).pin_memory()
     host_views = [[stage_h[s, o:o + n].view(dt).view(shp) for o, n, dt, shp in layout] for s in range(e2e_steps)]
     lens_e2e = [[L + base + (s + 1) * adv for L in lens0] for s in range(e2e_steps)]
@@ -369,19 +372,92 @@ def run_ours(args):
     h2d = sum(n for _, n, _, _ in layout)
     d2h = out.numel() * 4
     ws_step = csd.alloc_step_workspace(st.ctx, B, nq, Hq, device=dev)
+    # copies on their own streams, one per direction (the link is full
+    # duplex): step s + 1's inputs go in while step s computes, step s's
+    # output comes back while step s + 1 computes; events order each buffer's
+    # reuse (inputs of step s + 2 after step s's kernels, its output after
+    # step s's read-back).  For steps of a few KB the extra stream and event
+    # calls cost the host more than the copies take, so those run in line.
+    overlap = h2d + d2h >= 65536
+    if overlap:
+        h2d_stream, d2h_stream = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    else:
+        h2d_stream = d2h_stream = stream
+    ev_in = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_out = [torch.cuda.Event() for _ in range(e2e_steps)]
+
+    def copy_in(s):
+        if s >= 2:
+            h2d_stream.wait_event(ev_done[s - 2])
+        with torch.cuda.stream(h2d_stream):
+            stage_ds[s % 2].copy_(stage_h[s], non_blocking=True)
+        ev_in[s].record(h2d_stream)
+
+    def step_in_line(s):
+        kd, vd, qd, sd, ld = dviews[s % 2]
+        stage_ds[s % 2].copy_(stage_h[s], non_blocking=True)
+        csd.isoquant_decode_step(st.ctx, st.cache, kd, vd, sd, qd.view(B, nq, Hq, 128), st.page_table, ld, ws_step,
+                                 outs[s % 2], causal=wl.causal, stream=stream)
+        out_h[s].copy_(outs[s % 2], non_blocking=True)
+
+    # --graph with in-line copies: the e2e steps, copies included, captured
+    # as graphs of GRAPH_STEPS steps and replayed
+    e2e_graphs = []
+    if args.graph and not overlap:
+        for c0 in range(0, e2e_steps, GRAPH_STEPS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for s in range(c0, min(c0 + GRAPH_STEPS, e2e_steps)):
+                    step_in_line(s)
+            e2e_graphs.append(g)
     multi.barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for s in range(e2e_steps):
-        stage_d.copy_(stage_h[s], non_blocking=True)
+    if overlap:
+        h2d_stream.wait_event(e0)
+        d2h_stream.wait_event(e0)
+        copy_in(0)
+    for g in e2e_graphs:
+        g.replay()
+    for s in range(e2e_steps if not e2e_graphs else 0):
+        kd, vd, qd, sd, ld = dviews[s % 2]
+        if overlap:
+            if s + 1 < e2e_steps:
+                copy_in(s + 1)
+            stream.wait_event(ev_in[s])
+            if s >= 2:
+                stream.wait_event(ev_out[s - 2])
+        else:
+            step_in_line(s)
+            continue
         # the one-call public API of a decode step
         csd.isoquant_decode_step(st.ctx, st.cache, kd, vd, sd, qd.view(B, nq, Hq, 128), st.page_table, ld, ws_step,
-                                 out, causal=wl.causal, stream=stream)
-        out_h[s].copy_(out, non_blocking=True)
+                                 outs[s % 2], causal=wl.causal, stream=stream)
+        if overlap:
+            ev_done[s].record(stream)
+            d2h_stream.wait_event(ev_done[s])
+            with torch.cuda.stream(d2h_stream):
+                out_h[s].copy_(outs[s % 2], non_blocking=True)
+            ev_out[s].record(d2h_stream)
+    if overlap:
+        stream.wait_event(ev_out[e2e_steps - 1])
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    # the overlapped steps against the same steps run one at a time on one
+    # stream (the kernels are deterministic: a race between the copies and
+    # the kernels would show as a difference)
+    e2e_checked = sorted({0, e2e_steps // 2, e2e_steps - 1})
+    e2e_identical = True
+    for s in e2e_checked:
+        stage_ds[0].copy_(stage_h[s])
+        kd, vd, qd, sd, ld = dviews[0]
+        csd.isoquant_decode_step(st.ctx, st.cache, kd, vd, sd, qd.view(B, nq, Hq, 128), st.page_table, ld, ws_step,
+                                 outs[0], causal=wl.causal, stream=stream)
+        torch.cuda.synchronize(dev)
+        e2e_identical = e2e_identical and bool(torch.equal(outs[0].cpu(), out_h[s]))
     e2e_ms = multi.max_over_ranks(e0.elapsed_time(e1), device=dev)
     e2e_units = multi.sum_over_ranks(sum(sum(lens_e2e[s]) * H for s in range(e2e_steps)), device=dev)
     e2e_value = e2e_units / (e2e_ms / 1e3)
@@ -420,7 +496,12 @@ def run_ours(args):
                    "parallelism": f"dp{world} (independent shards)", "code_bits": args.bits,
                    "bytes_per_kv_token_head": bytes_per_token_head},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps},
+                "steps": e2e_steps, "api": "isoquant_decode_step",
+                "copies": ("pinned host <-> device every step, each direction on its own stream, overlapping the "
+                           "neighbouring steps' kernels (double-buffered inputs and outputs)" if overlap else
+                           "pinned host <-> device every step, in line on the launching stream" +
+                           (f"; steps and copies replayed as CUDA graphs of {GRAPH_STEPS}" if e2e_graphs else "")),
+                "serial_recheck": {"steps": e2e_checked, "identical": e2e_identical}},
         "roofline": {"bound": "hbm", "kernel": f"isoquant_attend_decode ({partial_kernel} + k_attend_combine)",
                      "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
@@ -798,24 +879,49 @@ def run_prefill_attend(args):
     sh = slots.cpu().pin_memory()
     lh = st.seq_lens_dev.cpu().pin_memory()
     oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    kd, vd, qd, sd, ld = (torch.empty_like(ks), torch.empty_like(vs), torch.empty_like(qs[0]),
-                          torch.empty_like(slots), torch.empty_like(st.seq_lens_dev))
+    # two sets of device inputs and outputs: a step's copies (each direction
+    # on its own stream) overlap the neighbouring steps' kernels
+    bufs = [(torch.empty_like(ks), torch.empty_like(vs), torch.empty_like(qs[0]), torch.empty_like(slots),
+             torch.empty_like(st.seq_lens_dev), torch.empty_like(out)) for _ in range(2)]
     ws_step = csd.alloc_step_workspace(st.ctx, B, nq, Hq, device=dev)
+    kd, vd, qd, sd, ld, _ = bufs[0]
     h2d = (kd.numel() + vd.numel() + qd.numel()) * 2 + sd.numel() * 8 + ld.numel() * 4
     d2h = out.numel() * 4
     del ws
+    h2d_stream, d2h_stream = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_out = [torch.cuda.Event() for _ in range(e2e_steps)]
+
+    def copy_in(i):
+        if i >= 2:
+            h2d_stream.wait_event(ev_done[i - 2])
+        with torch.cuda.stream(h2d_stream):
+            for dst, src in zip(bufs[i % 2][:5], (kh, vh, qh, sh, lh)):
+                dst.copy_(src, non_blocking=True)
+        ev_in[i].record(h2d_stream)
+
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        qd.copy_(qh, non_blocking=True)
-        sd.copy_(sh, non_blocking=True)
-        ld.copy_(lh, non_blocking=True)
-        csd.isoquant_decode_step(st.ctx, st.cache, kd, vd, sd, qd, st.page_table, ld, ws_step, out, causal=True,
+    h2d_stream.wait_event(e0)
+    d2h_stream.wait_event(e0)
+    copy_in(0)
+    for i in range(e2e_steps):
+        if i + 1 < e2e_steps:
+            copy_in(i + 1)
+        kd, vd, qd, sd, ld, od = bufs[i % 2]
+        stream.wait_event(ev_in[i])
+        if i >= 2:
+            stream.wait_event(ev_out[i - 2])
+        csd.isoquant_decode_step(st.ctx, st.cache, kd, vd, sd, qd, st.page_table, ld, ws_step, od, causal=True,
                                  stream=stream)
-        oh.copy_(out, non_blocking=True)
+        ev_done[i].record(stream)
+        d2h_stream.wait_event(ev_done[i])
+        with torch.cuda.stream(d2h_stream):
+            oh.copy_(od, non_blocking=True)
+        ev_out[i].record(d2h_stream)
+    stream.wait_event(ev_out[e2e_steps - 1])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
@@ -833,7 +939,9 @@ def run_prefill_attend(args):
                            "attend_partial (tcgen05, causal horizon per 128-row stream) + attend_combine",
                    "l2": "two query sets of 268 MB alternate; no flush"},
         "e2e": {"value": flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps, "api": "isoquant_decode_step",
+                "copies": "pinned host <-> device every step, each direction on its own stream, overlapping the "
+                          "neighbouring steps' kernels (double-buffered inputs and outputs)"},
         "roofline": {"bound": "tensor", "kernel": "isoquant_attend_partial (k_attend_wide)", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": None, "avg_launch_ms": part_ms, "flops_per_launch": flops,
