@@ -477,7 +477,7 @@ __device__ __forceinline__ void compress_warp(const CompressArgs &g, int kv, uin
       }
     }
     const bool near = dmin < band;
-    // the group's verdict: any lane near a threshold sends the vector to
+    // the group's decision: any lane near a threshold sends the vector to
     // the fp64 path
     const uint32_t gmask = 0xFFu << (8 * grp);
     slow = (__ballot_sync(0xffffffffu, (near || slow) && valid) & gmask) != 0;
