@@ -288,9 +288,11 @@ int isoquant_attend_combine(isoquant_ctx *ctx, int batch, int nq,
 /* Debug export of the normalised rotated coordinates z that
  * isoquant_compress_kv quantizes: z_j = sqrt(128) * (R x)_j / ||x||_2, the
  * Walsh-Hadamard transform then the SO(4) blocks (RotaryQuant, Abstract),
- * as the compress kernels compute it on their fp32 fast path, before any
- * fp64 re-check (coordinates within 1e-5 of a decision threshold and norms
- * near an fp16 rounding midpoint are redone in fp64 when compressing).
+ * from the same fp32 rotation as the compress kernels' fast path, divided by
+ * the fp32 norm (the compress kernel itself compares |y| with t * ||x||
+ * rather than forming z), before any fp64 re-check (coordinates within 1e-5
+ * of a decision threshold and norms near an fp16 rounding midpoint are
+ * redone in fp64 when compressing).
  * Lets a test measure the fp32 error of z against an exact reference.  Not
  * on the decode path.
  *   x: device [n_tok][num_kv_heads][128] of dtype (F32, BF16, F16),
