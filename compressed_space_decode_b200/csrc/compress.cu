@@ -645,7 +645,7 @@ namespace {
 constexpr int kMaxStrip = ISOQUANT_COMPRESS_STRIP;
 int strip_tokens(const isoquant_ctx *ctx, int n_tok) {
   const int64_t vectors = static_cast<int64_t>(n_tok) * ctx->num_kv_heads;  // per K/V half
-  const int64_t resident = static_cast<int64_t>(ctx->num_sms) * 12;       // warps the SMs hold
+  const int64_t resident = static_cast<int64_t>(ctx->num_sms) * kCompressWarps * kCompressBlocksPerSm;  // warps the SMs hold
   const int64_t s = (vectors / resident) & ~int64_t(3);
   return static_cast<int>(s < 4 ? 4 : (s > kMaxStrip ? kMaxStrip : s));
 }
