@@ -495,6 +495,8 @@ def run_ours(args):
                    "l2": f"packed cache {bytes_per_launch / 1e6:.0f} MB > 126 MB L2; no flush",
                    "parallelism": f"dp{world} (independent shards)", "code_bits": args.bits,
                    "bytes_per_kv_token_head": bytes_per_token_head},
+        # the same rate per query head (each KV token-head serves G = Hq / H query heads)
+        "value_q_head_equivalent": {"value": value * (Hq // H), "unit": "KV-token·q-heads/s", "group": Hq // H},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "api": "isoquant_decode_step",
                 "copies": ("pinned host <-> device every step, each direction on its own stream, overlapping the "
