@@ -67,3 +67,33 @@ def test_oracle_step_rows_see_their_prefix(causal, nq):
         n = 45 + r // wl.group + 1
         ref = oracle.attend(o["s"], o["qt"], o["q"][r:r + 1], kc[:n], kn[:n], vc[:n], vn[:n], [n])
         assert np.allclose(out[r], ref[0], rtol=0, atol=1e-12 * np.abs(ref).max())
+
+
+def test_oracle_pools_run_their_samples():
+    """The all-core CPU-baseline legs: spawned processes that each run the
+    oracle's decode step (or its bulk compression) on the same sample, and
+    the counts the bench turns into rates."""
+    import numpy as np
+    from compressed_space_decode_b200 import synthetic
+    wl = Workload("t", 1, 4, 1, [100], nq=1, page_size=64, causal=False, seed=6)
+    o = bench.oracle_sample(wl, 0, 0, device="cpu")
+    pool = bench.OraclePool(o, 2)
+    n, dt = pool.run(steps=2)
+    pool.close()
+    assert n == 4 and dt > 0
+    signs, quats = synthetic.rotation_params(7, 1)
+    sample = {"s": signs[0].numpy(), "qt": quats[0].numpy(),
+              "x": np.random.default_rng(8).standard_normal((16, 128)), "bits": 3}
+    pool = bench.OraclePool(sample, 2, worker=bench._compress_worker)
+    n, dt = pool.run(steps=3)
+    pool.close()
+    assert n == 2 * 3 * 16 and dt > 0
+
+
+def test_clocks_resample_keeps_a_sampled_region():
+    """A timed region that nvidia-smi sampled keeps its own clocks (no
+    re-run); only an unsampled one is re-sampled over extra steps."""
+    c = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3}
+    calls = []
+    assert bench.clocks_or_resample(c, "GPU-x", lambda: calls.append(1), None) is c
+    assert not calls
